@@ -1,0 +1,429 @@
+"""Benchmark of the SAGA + Atop-N decode-attention step on B200.
+
+One step = one decode step of every layer of the workload: for each layer,
+append the new token's key/value rows, then the attention step (Atop-N
+threshold refresh on t % R == 0, else reuse).  The step runs as a CUDA graph
+replay; caches live in HBM.  Default workload: the Qwen2.5-1.5B-shaped SAGA
+configuration at 128K context (h_q=12, d=128, h_k=1, h_v=4, N=512, R=32,
+28 layers, batch 1 per GPU).
+
+Printed JSON (rank 0, one line):
+  value        whole-job algorithmic HBM GB/s (all ranks; bytes per the
+               key/value read model below), inputs already resident
+  ms_per_step  max over ranks of the mean step time
+  e2e          the same metric with this step's q/k_new/v_new copied from
+               pinned host memory and every layer's output copied back,
+               inside the timed region
+  roofline     the context-split attention kernel: algorithmic bytes of one
+               layer-step / its mean CUDA-event duration vs the measured HBM
+               copy bandwidth
+  cpu_baseline the CPU oracle on a bounded sample (rank 0, N=1)
+
+Algorithmic bytes of one layer-step:
+  2*B*d*(h_k*L + min(h_q*N, h_v*L)) + 2*B*h_q*d (q) + 4*B*h_q*d (fp32 out)
+(every cached key of every key head, N value rows per query head or each value
+row once when N covers the context, the query, the output).
+
+`--impl reference` times the CPU oracle as it stands on this host's cores
+(the reference arm; rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn µs/step and achieved HBM GB/s (% roofline) at 128K ctx, h_k=1..8"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "split_kernel_traffic.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def layer_bytes(wl, L):
+    n = L if wl.dense else wl.n_top
+    keys = wl.h_k * L
+    vals = min(wl.h_q * n, wl.h_v * L)
+    return 2 * wl.batch * wl.d * (keys + vals) + 2 * wl.batch * wl.h_q * wl.d + 4 * wl.batch * wl.h_q * wl.d
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("saga_kernels.cu", "saga_device.cuh", "saga_internal.h"):
+        with open(os.path.join(ROOT, "long_context_decoding_saga_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peak():
+    try:
+        with open(PEAKS_PATH) as f:
+            v = float(json.load(f)["hbm_gbs"])
+            return v, "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_traffic(workload_name):
+    try:
+        with open(TRAFFIC_PATH) as f:
+            t = json.load(f)
+        if t.get("kernel_hash") != kernel_source_hash() or t.get("workload") != workload_name:
+            return None
+        return float(t["bytes_per_launch"])
+    except Exception:  # noqa: BLE001
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:  # noqa: BLE001
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:  # noqa: BLE001
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        if not self.samples:
+            return None
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def oracle_threads():
+    """Threads the numpy oracle can use (its BLAS pool; sorts and exps are single-threaded)."""
+    n = len(os.sched_getaffinity(0))
+    try:
+        from threadpoolctl import threadpool_info
+        blas = [int(i.get("num_threads", 0)) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if blas:
+            n = max(blas)
+    except Exception:  # noqa: BLE001
+        pass
+    return n
+
+
+def cpu_baseline(wl, seconds_budget=20.0):
+    """The oracle as it stands, on a bounded sample: whole decode steps of single layers at full size."""
+    import numpy as np
+    import torch
+
+    from long_context_decoding_saga_b200 import workload
+    from oracle import saga_oracle
+
+    cores = oracle_threads()
+    inp = workload.make_layer(wl, 0, device="cpu", steps=2)
+    orc = saga_oracle.OracleLayer(inp["K0"].float().numpy(), inp["V0"].float().numpy(), wl.h_q,
+                                  wl.n_for_kernel(wl.l_kv + 2), wl.refresh, l_cap=wl.l_kv + 2)
+    t0 = time.perf_counter()
+    done, nbytes = 0, 0
+    kinds = []
+    for t in range(2):
+        orc.step(inp["q"][t].float().numpy(), inp["k_new"][t].float().numpy(), inp["v_new"][t].float().numpy())
+        done += 1
+        nbytes += layer_bytes(wl, wl.l_kv + t + 1)
+        kinds.append("refresh" if t % wl.refresh == 0 else "reuse")
+        if time.perf_counter() - t0 > seconds_budget:
+            break
+    dt = time.perf_counter() - t0
+    del torch, np
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} layer-steps of layer 0 ({'+'.join(kinds)}) at full size, numpy oracle",
+            "us_per_layer_step": dt / done * 1e6, "us_per_step_scaled": dt / done * 1e6 * wl.layers}
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return 0
+    # each step: a bounded sample of the workload (layer 0, one decode step, full size)
+    from long_context_decoding_saga_b200 import workload
+    from oracle import saga_oracle
+    inp = workload.make_layer(wl, 0, device="cpu", steps=args.warmup + args.steps)
+    l_cap = wl.l_kv + args.warmup + args.steps
+    orc = saga_oracle.OracleLayer(inp["K0"].float().numpy(), inp["V0"].float().numpy(), wl.h_q,
+                                  wl.n_for_kernel(l_cap), wl.refresh, l_cap=l_cap)
+    times, nbytes = [], 0
+    for t in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        orc.step(inp["q"][t].float().numpy(), inp["k_new"][t].float().numpy(), inp["v_new"][t].float().numpy())
+        dt = time.perf_counter() - t0
+        if t >= args.warmup:
+            times.append(dt)
+            nbytes += layer_bytes(wl, wl.l_kv + t + 1)
+    total = sum(times)
+    value = nbytes / total / 1e9
+    cores = oracle_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3 * wl.layers, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "l_kv": wl.l_kv, "h_q": wl.h_q, "h_k": wl.h_k,
+                   "h_v": wl.h_v, "d": wl.d, "n_top": wl.n_top, "refresh": wl.refresh, "layers": wl.layers},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": "each step: one decode step of layer 0 at full size (ms_per_step scaled to all "
+                                   "layers)"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_saga(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from long_context_decoding_saga_b200 import build as build_mod
+    from long_context_decoding_saga_b200 import saga, workload
+    from long_context_decoding_saga_b200.session import DecodeSession
+
+    build_mod.build()
+    saga.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+
+    W, K = args.warmup, args.steps
+    E = 0 if args.no_e2e else max(4, min(K, 16))
+    T = max(2, min(K, 8))  # kernel-timing replays
+    total_steps = 1 + W + K + E + T
+    l_cap = wl.l_kv + total_steps
+    n_top = wl.n_for_kernel(l_cap)
+    shape = saga.SagaShape.of(wl.batch, wl.h_q, wl.h_k, wl.h_v, wl.d, l_cap)
+    sess = DecodeSession(shape, wl.layers, n_top, wl.refresh, device=dev)
+    qs, ks, vs = [], [], []
+    for i in range(wl.layers):
+        inp = workload.make_layer(wl.with_(seed=wl.seed + 7919 * rank), i, device=dev, steps=total_steps)
+        sess.prefill(i, inp["K0"], inp["V0"])
+        qs.append(inp["q"])
+        ks.append(inp["k_new"])
+        vs.append(inp["v_new"])
+        del inp
+    q_all = torch.stack(qs, dim=1)  # [steps, layers, B, h_q, d]
+    k_all = torch.stack(ks, dim=1)
+    v_all = torch.stack(vs, dim=1)
+    del qs, ks, vs
+    torch.cuda.synchronize()
+
+    # step 0 eagerly (warms launch attributes), then record the step graphs
+    sess.step(q_all[0], k_all[0], v_all[0])
+    stream = torch.cuda.Stream(dev)
+    sess.capture(stream)
+    cur = 1
+
+    def replay_range(n):
+        nonlocal cur
+        for _ in range(n):
+            sess.stage(q_all[cur], k_all[cur], v_all[cur])
+            sess.replay()
+            cur += 1
+
+    replay_range(W)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    bytes_timed = 0
+    refresh_steps = 0
+    ev0.record()
+    for _ in range(K):
+        L = sess.length + 1
+        bytes_timed += wl.layers * layer_bytes(wl, L)
+        refresh_steps += int(sess.t % wl.refresh == 0)
+        sess.stage(q_all[cur], k_all[cur], v_all[cur])
+        sess.replay()
+        cur += 1
+    ev1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1)
+    launches = refresh_steps * sess.launches_per_step(True) + (K - refresh_steps) * sess.launches_per_step(False)
+    if world > 1:
+        dist.barrier()
+
+    # end to end: pinned host inputs in, every layer's output out, inside the timed region
+    e2e = None
+    if E > 0:
+        hq = [q_all[cur + s].cpu().pin_memory() for s in range(E)]
+        hk = [k_all[cur + s].cpu().pin_memory() for s in range(E)]
+        hv = [v_all[cur + s].cpu().pin_memory() for s in range(E)]
+        hout = torch.empty(sess.out.shape, dtype=sess.out.dtype, pin_memory=True)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e_bytes = 0
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for s in range(E):
+            e_bytes += wl.layers * layer_bytes(wl, sess.length + 1)
+            sess.stage(hq[s], hk[s], hv[s])
+            sess.replay()
+            hout.copy_(sess.out, non_blocking=True)
+        a1.record()
+        torch.cuda.synchronize()
+        e_ms = a0.elapsed_time(a1)
+        cur += E
+        h2d = (hq[0].numel() * 2 + hk[0].numel() * 2 + hv[0].numel() * 2)
+        d2h = hout.numel() * hout.element_size()
+        e2e = {"value": e_bytes / (e_ms / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / E}
+
+    # dominant kernel: the split-context attention kernel of reuse steps, bracketed by CUDA events on
+    # its stream inside freshly recorded graphs (one event pair per layer)
+    kernel_ms = []
+    if wl.refresh > 1 and T > 0:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(wl.layers)]
+        g = torch.cuda.CUDAGraph()
+        L_est = sess.length + 1
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            sess.seq_len_dev.add_(1)
+            for i in range(wl.layers):
+                saga.saga_kv_append(shape, sess.k_cache[i], sess.v_cache[i], sess.k_buf[i], sess.v_buf[i],
+                                    L_est - 1, seq_len_dev=sess.seq_len_dev)
+                saga.saga_trace_next_attention(*evs[i])
+                saga.saga_decode_attn(shape, sess.q_buf[i], sess.k_cache[i], sess.v_cache[i], L_est, n_top,
+                                      wl.refresh, 1, sess.tau[i], sess.out[i], sess.workspace,
+                                      seq_len_dev=sess.seq_len_dev)
+        sess.seq_len_dev.fill_(sess.length)
+        for _ in range(T):
+            if sess.t % wl.refresh == 0:  # keep the refresh schedule: run refresh steps with the step graphs
+                sess.stage(q_all[cur], k_all[cur], v_all[cur])
+                sess.replay()
+                cur += 1
+                continue
+            sess.stage(q_all[cur], k_all[cur], v_all[cur])
+            g.replay()
+            sess.length += 1
+            sess.t += 1
+            cur += 1
+            torch.cuda.synchronize()
+            kernel_ms.extend(a.elapsed_time(b) for a, b in evs)
+        del g
+    status = saga.saga_get_status(sess.workspace)
+
+    # ---- gather over ranks
+    stats = torch.tensor([ms, bytes_timed, e2e["value"] if e2e else 0.0], dtype=torch.float64, device=dev)
+    if world > 1:
+        gathered = [torch.zeros_like(stats) for _ in range(world)]
+        dist.all_gather(gathered, stats)
+        ms_max = max(float(x[0]) for x in gathered)
+        total_bytes = sum(float(x[1]) for x in gathered)
+        e2e_sum = sum(float(x[2]) for x in gathered)
+    else:
+        ms_max, total_bytes, e2e_sum = ms, bytes_timed, (e2e["value"] if e2e else 0.0)
+    if rank != 0:
+        return 0
+    value = total_bytes / (ms_max / 1e3) / 1e9
+    ms_per_step = ms_max / K
+    peak, peak_kind = load_peak()
+    roofline = None
+    if kernel_ms:
+        k_mean = statistics.mean(kernel_ms)
+        L_mid = sess.length
+        achieved = layer_bytes(wl, L_mid) / (k_mean / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": load_traffic(wl.name), "kernel": "saga_split_kernel (reuse step, per layer)",
+                    "kernel_us_mean": k_mean * 1e3, "launches_timed": len(kernel_ms), "peak_kind": peak_kind}
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "l_kv": wl.l_kv, "h_q": wl.h_q, "h_k": wl.h_k,
+                   "h_v": wl.h_v, "d": wl.d, "n_top": wl.n_top if not wl.dense else "dense", "refresh": wl.refresh,
+                   "layers": wl.layers, "parallelism": f"replicas{world}",
+                   "l2": "inputs exceed L2 (all layers' caches cycle through L2 each step)",
+                   "refresh_steps_timed": refresh_steps},
+        "roofline": roofline,
+        "e2e": ({"value": e2e_sum if world > 1 else e2e["value"], "unit": "GB/s",
+                 "h2d_bytes_per_step": e2e["h2d_bytes_per_step"] * world,
+                 "d2h_bytes_per_step": e2e["d2h_bytes_per_step"] * world} if e2e else None),
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "status_word": status,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=32)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="saga", choices=["saga", "reference"])
+    ap.add_argument("--workload", default="qwen2.5-1.5b_saga_128k")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from long_context_decoding_saga_b200 import workload
+    wl = workload.CONFIGS[args.workload]
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, wl, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        return run_saga(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

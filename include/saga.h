@@ -1,0 +1,160 @@
+/*
+ * saga.h - C ABI of libsaga: the SAGA + Atop-N single-token decode-attention
+ * step on NVIDIA B200 (sm_100a).
+ *
+ * Source of the operation: "More Value per Key: Asymmetric Sparse Attention
+ * for Faster LLM Decoding" (Elata, Lamprecht, Shechter, Ohayon, Hubara,
+ * Soudry).  One decode step of one attention layer:
+ *   - append the new token's key and value rows to the KV cache;
+ *   - score the token's queries against every cached key,
+ *     A = q K^T / sqrt(d)                                      (eq. 2);
+ *   - keep the positions whose score is at least a per-query-head threshold
+ *     (Atop-N step 1); every R steps that threshold is recomputed exactly as
+ *     the N-th largest score of the row and reused in between (Atop-N step 2);
+ *   - O = softmax(A[i]) V[i] over the kept positions i          (eq. 7);
+ *   - key and value head counts are independent, h_k != h_v     (SAGA).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library never allocates, frees or synchronizes; every call only
+ *     enqueues work on `stream` (a cudaStream_t passed as void*, NULL = the
+ *     legacy default stream) and returns.
+ *   - bf16 means IEEE bfloat16 stored as 16-bit words; fp32 is IEEE binary32.
+ *   - Layouts are dense and row-major in the order written:
+ *       q        bf16 [B, h_q, d]
+ *       k_cache  bf16 [B, h_k, l_cap, d]   (one buffer per layer)
+ *       v_cache  bf16 [B, h_v, l_cap, d]   (one buffer per layer)
+ *       k_new    bf16 [B, h_k, d]
+ *       v_new    bf16 [B, h_v, d]
+ *       tau      fp32 [B, h_q]
+ *       out      fp32 or bf16 [B, h_q, d]
+ *     Base addresses must be 16-byte aligned.
+ *   - Query head j reads key head floor(j*h_k/h_q) and value head
+ *     floor(j*h_v/h_q) (contiguous groups).  Requires h_q % h_k == 0,
+ *     h_q % h_v == 0 and (h_v % h_k == 0 or h_k % h_v == 0);
+ *     1 <= h_q/h_k <= 64; d in {64, 128}.
+ *   - Sequence length: `seq_len` is the number of valid cached tokens,
+ *     including the token appended this step (1 <= seq_len <= l_cap).  If
+ *     `seq_len_dev` is not NULL the kernels read the length from that device
+ *     int instead, when they run (use this inside CUDA graphs, where the
+ *     length changes between replays); `seq_len` must then still be a valid
+ *     host-side estimate, used only to size the launch.  A device length
+ *     outside [1, l_cap] is clamped and flagged in the workspace status word.
+ *   - Inputs must be finite (no NaN/Inf in q or the caches).
+ *   - Return value: SAGA_OK or a negative SAGA_ERR_* code.  Arguments are
+ *     validated before anything is enqueued; on an error nothing is
+ *     launched and saga_last_error() describes it.  SAGA_ERR_CUDA reports a
+ *     launch failure seen by cudaGetLastError after enqueueing.
+ */
+#ifndef SAGA_H
+#define SAGA_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define SAGA_API __attribute__((visibility("default")))
+#else
+#define SAGA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SAGA_OK 0
+#define SAGA_ERR_ARG (-1)         /* bad pointer, shape, length, N, R or dtype */
+#define SAGA_ERR_UNSUPPORTED (-2) /* valid but not implemented (e.g. d = 96)   */
+#define SAGA_ERR_WORKSPACE (-3)   /* workspace NULL or smaller than required    */
+#define SAGA_ERR_CUDA (-4)        /* CUDA runtime/driver error while enqueueing */
+
+#define SAGA_OUT_F32 0
+#define SAGA_OUT_BF16 1
+
+/* Bits of the workspace status word (see saga_get_status). */
+#define SAGA_STATUS_LEN_CLAMPED 0x1u /* a device-side length was outside [1, l_cap] */
+#define SAGA_STATUS_TIMEOUT 0x2u     /* a pipeline wait gave up (the result is invalid) */
+
+typedef struct saga_shape {
+  int batch; /* B */
+  int h_q;   /* query heads */
+  int h_k;   /* key heads   (SAGA: fewer key heads ...) */
+  int h_v;   /* value heads (... than value heads) */
+  int d;     /* head dimension: 64 or 128 */
+  int l_cap; /* capacity of each cache head, in tokens */
+} saga_shape;
+
+/* Bytes of scratch that atopn_refresh_threshold and saga_decode_attn need for
+ * this shape on the current device (split partials, the score rows of a
+ * refresh step, radix histograms, per-split index lists, a status word).
+ * The buffer is caller-owned device memory, 256-byte aligned, zero-filled
+ * once before first use; calls on one workspace must not overlap in time.
+ * Returns 0 for an invalid shape. */
+SAGA_API size_t saga_workspace_bytes(const saga_shape* s);
+
+/* KV cache append (the "KV cache" of the explainer's jargon list): writes
+ * k_new into k_cache[:, :, pos, :] and v_new into v_cache[:, :, pos, :].
+ * If seq_len_dev is not NULL, pos is read on the device as (*seq_len_dev - 1)
+ * and the host `pos` only needs to be in range.  0 <= pos < l_cap. */
+SAGA_API int saga_kv_append(const saga_shape* s, void* k_cache, void* v_cache, const void* k_new, const void* v_new, int pos,
+                   const int* seq_len_dev, void* stream);
+
+/* Atop-N threshold refresh (Atop-N step 1-2, "computed once every n
+ * tokens"): tau[b, j] = the n_top-th largest of the fp32 scores
+ * A[b, j, 0..seq_len) (eq. 2), counted with multiplicity; -inf when
+ * n_top >= seq_len.  Exact: radix selection over order-preserving 32-bit
+ * images of the scores, no sort.  n_top >= 1. */
+SAGA_API int atopn_refresh_threshold(const saga_shape* s, const void* q, const void* k_cache, int seq_len,
+                            const int* seq_len_dev, int n_top, float* tau, void* workspace, size_t ws_bytes,
+                            void* stream);
+
+/* The exact N-th-largest selection alone, over caller-provided fp32 rows:
+ * tau[r] = the n_top-th largest of scores[r*row_stride + 0 .. row_len), with
+ * multiplicity; -inf when n_top >= row_len.  rows >= 1, 1 <= row_len <=
+ * row_stride, row_stride % 4 == 0.  Workspace: at least
+ * atopn_select_workspace_bytes(rows). */
+SAGA_API size_t atopn_select_workspace_bytes(int rows);
+SAGA_API int atopn_select_threshold(const float* scores, int rows, int row_len, long long row_stride, int n_top, float* tau,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* One decode step of one layer (eqs. 2 and 7 with the Atop-N threshold).
+ *   step: decode step index t >= 0; when t % refresh_interval == 0 the
+ *         threshold is first recomputed exactly from this step's scores and
+ *         written to tau; otherwise tau is read (it must hold the threshold of
+ *         the last refresh step).
+ *   n_top: N >= 1.  n_top >= seq_len selects every token (dense attention);
+ *         pass n_top = l_cap for attention without a threshold.
+ *   out_dtype: SAGA_OUT_F32 or SAGA_OUT_BF16 (round to nearest even).
+ *   sel_count (nullable): int32 [B, h_q], number of kept positions.
+ *   sel_idx (nullable, needs sel_count): int32 [B, h_q, l_cap]; the first
+ *         sel_count[b, j] entries are the kept positions in ascending order.
+ * The kernels read the caches at positions < seq_len only. */
+SAGA_API int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, const void* v_cache, int seq_len,
+                     const int* seq_len_dev, int n_top, int refresh_interval, long long step, float* tau, void* out,
+                     int out_dtype, int* sel_count, int* sel_idx, void* workspace, size_t ws_bytes, void* stream);
+
+/* Tracing: the next saga_decode_attn call made on this host thread records
+ * ev_start on its stream just before its context-split attention kernels
+ * (after nothing else of that call) and ev_end just after them, before the
+ * cross-split combine.  On a reuse step that is the one fused split kernel;
+ * on a refresh step it spans score dump, radix select and the compare/gather
+ * pass.  The events are cudaEvent_t handles created by the caller (timing
+ * enabled); under stream capture they become external event-record nodes, so
+ * graph replays record them too.  One-shot: cleared by that call.  Passing
+ * NULLs cancels a pending request. */
+SAGA_API int saga_trace_next_attention(void* ev_start, void* ev_end);
+
+/* Reads the workspace status word (SAGA_STATUS_* bits ORed by the kernels
+ * since the workspace was zeroed) after synchronizing `stream`. */
+SAGA_API int saga_get_status(const void* workspace, void* stream, unsigned* status);
+
+/* Text of the last error reported on this host thread ("" if none). */
+SAGA_API const char* saga_last_error(void);
+
+/* ABI version (major * 100 + minor). */
+SAGA_API int saga_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGA_H */

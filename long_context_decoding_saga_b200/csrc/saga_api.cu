@@ -1,0 +1,476 @@
+// saga_api.cu - host side of libsaga: argument validation, workspace layout,
+// TMA descriptors, launch sizing and the extern "C" entry points of saga.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "saga.h"
+#include "saga_internal.h"
+
+namespace saga {
+cudaError_t launch_split(int D, int NP, bool dump, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p,
+                         dim3 grid, cudaStream_t st, int* occupancy_out);
+cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, cudaStream_t st);
+cudaError_t launch_combine(int D, const CombineParams& p, cudaStream_t st);
+cudaError_t launch_select(const SelectParams& p, int rows, cudaStream_t st);
+cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
+cudaError_t launch_fill(float* dst, float v, int n, cudaStream_t st);
+}  // namespace saga
+
+using namespace saga;
+
+namespace {
+
+thread_local char g_err[512] = "";
+thread_local cudaEvent_t g_trace_start = nullptr, g_trace_end = nullptr;
+
+cudaError_t trace_record(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  return cudaEventRecordWithFlags(ev, st, cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault);
+}
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int ok() {
+  g_err[0] = '\0';
+  return SAGA_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(SAGA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+struct DevInfo {
+  int sms = 0;
+  bool init = false;
+};
+DevInfo g_dev[128];
+std::mutex g_dev_mu;
+
+int device_sms(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 128) return fail(SAGA_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_dev[dev].init) {
+    int v = 0;
+    e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    g_dev[dev].sms = v;
+    g_dev[dev].init = true;
+  }
+  *sms = g_dev[dev].sms;
+  return SAGA_OK;
+}
+
+int np_for_group(int G) { return G <= 4 ? 4 : G <= 16 ? 16 : G <= 32 ? 32 : 64; }
+
+int validate_shape(const saga_shape* s) {
+  if (s == nullptr) return fail(SAGA_ERR_ARG, "shape is NULL");
+  if (s->batch < 1 || s->h_q < 1 || s->h_k < 1 || s->h_v < 1 || s->l_cap < 1)
+    return fail(SAGA_ERR_ARG, "shape fields must be >= 1 (batch=%d h_q=%d h_k=%d h_v=%d l_cap=%d)", s->batch, s->h_q,
+                s->h_k, s->h_v, s->l_cap);
+  if (s->d != 64 && s->d != 128) return fail(SAGA_ERR_UNSUPPORTED, "head dim d=%d not supported (64 or 128)", s->d);
+  if (s->h_q % s->h_k != 0 || s->h_q % s->h_v != 0)
+    return fail(SAGA_ERR_ARG, "h_q=%d must be a multiple of h_k=%d and h_v=%d", s->h_q, s->h_k, s->h_v);
+  if (s->h_v % s->h_k != 0 && s->h_k % s->h_v != 0)
+    return fail(SAGA_ERR_UNSUPPORTED, "one of h_k=%d, h_v=%d must divide the other", s->h_k, s->h_v);
+  const int G = s->h_q / s->h_k;
+  if (G > kMaxG) return fail(SAGA_ERR_UNSUPPORTED, "h_q/h_k=%d exceeds %d", G, kMaxG);
+  const int nvh = s->h_v >= s->h_k ? s->h_v / s->h_k : 1;
+  if (nvh > kMaxNvh) return fail(SAGA_ERR_UNSUPPORTED, "h_v/h_k=%d exceeds %d", nvh, kMaxNvh);
+  const int hpv = G / nvh;
+  const int P = nvh * (s->d / 4) * ((hpv + 3) / 4);
+  if (P > 4 * kEpiThreads) return fail(SAGA_ERR_UNSUPPORTED, "head layout too wide for one CTA (P=%d)", P);
+  if ((long long)s->batch * s->h_k * s->l_cap >= (1ll << 31) ||
+      (long long)s->batch * s->h_v * s->l_cap >= (1ll << 31) || (long long)s->batch * s->h_q >= (1 << 24))
+    return fail(SAGA_ERR_UNSUPPORTED, "cache too large for 32-bit row coordinates");
+  return SAGA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(const saga_shape* s, int sms) {
+  WsLayout w{};
+  const int groups = s->batch * s->h_k;
+  const long long rows = (long long)s->batch * s->h_q;
+  const int tiles_cap = (s->l_cap + kTile - 1) / kTile;
+  const long long by_sm = (32ll * kMaxCtasPerSm * sms + groups - 1) / groups;
+  w.s_cap = (int)std::max(1ll, std::min((long long)tiles_cap, by_sm));
+  w.ld_scores = ((long long)s->l_cap + 3) & ~3ll;
+  size_t off = 0;
+  w.status = off;
+  off = align256(off + 16);
+  w.part_o = off;
+  off = align256(off + (size_t)rows * w.s_cap * s->d * 4);
+  w.part_m = off;
+  off = align256(off + (size_t)rows * w.s_cap * 4);
+  w.part_l = off;
+  off = align256(off + (size_t)rows * w.s_cap * 4);
+  w.part_cnt = off;
+  off = align256(off + (size_t)rows * w.s_cap * 4);
+  w.scores = off;
+  off = align256(off + (size_t)rows * w.ld_scores * 4);
+  w.hist = off;
+  off = align256(off + (size_t)rows * 256 * 4);
+  w.idx = off;
+  off = align256(off + (size_t)rows * s->l_cap * 4);
+  w.total = off;
+  return w;
+}
+
+// Split count per (batch, key head): minimise waves / splits over the
+// resident-CTA slots of the device, at most one split per 128-token tile.
+int choose_splits(int groups, int L_est, int slots, int s_cap) {
+  const int tiles = std::max(1, (L_est + kTile - 1) / kTile);
+  const int smax = std::max(1, std::min(s_cap, tiles));
+  int best = 1;
+  double best_cost = 1e30;
+  for (int S = 1; S <= smax; ++S) {
+    const long long ctas = (long long)groups * S;
+    const long long waves = (ctas + slots - 1) / slots;
+    const double cost = (double)waves / S * (1.0 + 1e-3 * S);
+    if (cost < best_cost - 1e-12) {
+      best_cost = cost;
+      best = S;
+    }
+  }
+  return best;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D view of the key cache: rows = B*h_k*l_cap tokens, d bf16 columns;
+// boxes of 64 columns (one 128-byte swizzle atom) by `box_rows` rows.
+int make_key_map(CUtensorMap* m, const void* k_cache, const saga_shape* s, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (enc == nullptr) return fail(SAGA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
+  cuuint64_t dims[2] = {(cuuint64_t)s->d, (cuuint64_t)s->batch * s->h_k * s->l_cap};
+  cuuint64_t strides[1] = {(cuuint64_t)s->d * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k_cache), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SAGA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return SAGA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Prepared {
+  WsLayout ws;
+  int sms;
+  char* base;
+};
+
+int prepare_ws(const saga_shape* s, void* workspace, size_t ws_bytes, Prepared* out) {
+  int rc = device_sms(&out->sms);
+  if (rc) return rc;
+  out->ws = ws_layout(s, out->sms);
+  if (workspace == nullptr) return fail(SAGA_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(SAGA_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  if (ws_bytes < out->ws.total)
+    return fail(SAGA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, out->ws.total);
+  out->base = static_cast<char*>(workspace);
+  return SAGA_OK;
+}
+
+void fill_split_common(SplitParams& p, const saga_shape* s, const Prepared& pr, const void* q, int seq_len,
+                       const int* seq_len_dev) {
+  memset(&p, 0, sizeof(p));
+  p.q = static_cast<const uint16_t*>(q);
+  p.status = reinterpret_cast<unsigned*>(pr.base + pr.ws.status);
+  p.seq_len_dev = seq_len_dev;
+  p.seq_len = seq_len;
+  p.batch = s->batch;
+  p.h_q = s->h_q;
+  p.h_k = s->h_k;
+  p.h_v = s->h_v;
+  p.l_cap = s->l_cap;
+  p.s_cap = pr.ws.s_cap;
+  p.ld_scores = pr.ws.ld_scores;
+  p.G = s->h_q / s->h_k;
+  p.nvh = s->h_v >= s->h_k ? s->h_v / s->h_k : 1;
+  p.hpv = p.G / p.nvh;
+  p.scale = (float)(1.0 / sqrt((double)s->d));
+  p.part_o = reinterpret_cast<float*>(pr.base + pr.ws.part_o);
+  p.part_m = reinterpret_cast<float*>(pr.base + pr.ws.part_m);
+  p.part_l = reinterpret_cast<float*>(pr.base + pr.ws.part_l);
+  p.part_cnt = reinterpret_cast<int*>(pr.base + pr.ws.part_cnt);
+}
+
+int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, bool dump, const CUtensorMap& tf,
+               const CUtensorMap& tp, int* S) {
+  int occ = 0;
+  SplitParams dummy{};
+  cudaError_t e = launch_split(s->d, NP, dump, tf, tp, dummy, dim3(1), nullptr, &occ);
+  if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+  if (occ < 1) return fail(SAGA_ERR_UNSUPPORTED, "split kernel does not fit on an SM");
+  *S = choose_splits(s->batch * s->h_k, seq_len, occ * pr.sms, pr.ws.s_cap);
+  return SAGA_OK;
+}
+
+// Scores of every cached token, their top-byte histograms, and the exact
+// threshold (refresh).
+int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const void* k_cache, int seq_len,
+                const int* seq_len_dev, int n_top, float* tau, cudaStream_t st) {
+  const int G = s->h_q / s->h_k, NP = np_for_group(G);
+  CUtensorMap tf, tp;
+  int rc = make_key_map(&tf, k_cache, s, kTile);
+  if (rc) return rc;
+  rc = make_key_map(&tp, k_cache, s, kUnit);
+  if (rc) return rc;
+  int S = 1;
+  rc = splits_for(s, pr, seq_len, NP, true, tf, tp, &S);
+  if (rc) return rc;
+  const size_t rows = (size_t)s->batch * s->h_q;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(pr.base + pr.ws.hist);
+  cudaError_t e = cudaMemsetAsync(hist, 0, rows * 256 * 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(hist)");
+  SplitParams p;
+  fill_split_common(p, s, pr, q, seq_len, seq_len_dev);
+  p.scores_out = reinterpret_cast<float*>(pr.base + pr.ws.scores);
+  p.hist_out = hist;
+  p.nsplit = S;
+  e = launch_split(s->d, NP, true, tf, tp, p, dim3(S, s->h_k, s->batch), st, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "score dump launch");
+  SelectParams sp{};
+  sp.scores = p.scores_out;
+  sp.ld = pr.ws.ld_scores;
+  sp.hist = hist;
+  sp.tau = tau;
+  sp.status = p.status;
+  sp.seq_len_dev = seq_len_dev;
+  sp.row_len = seq_len;
+  sp.l_cap = s->l_cap;
+  sp.n_top = n_top;
+  e = launch_select(sp, (int)rows, st);
+  if (e != cudaSuccess) return cuda_fail(e, "radix select launch");
+  return SAGA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int saga_abi_version(void) { return 100; }
+
+const char* saga_last_error(void) { return g_err; }
+
+size_t saga_workspace_bytes(const saga_shape* s) {
+  if (validate_shape(s)) return 0;
+  int sms = 0;
+  if (device_sms(&sms)) return 0;
+  return ws_layout(s, sms).total;
+}
+
+size_t atopn_select_workspace_bytes(int rows) {
+  if (rows < 1) return 0;
+  return 256;
+}
+
+int saga_kv_append(const saga_shape* s, void* k_cache, void* v_cache, const void* k_new, const void* v_new, int pos,
+                   const int* seq_len_dev, void* stream) {
+  int rc = validate_shape(s);
+  if (rc) return rc;
+  if (!k_cache || !v_cache || !k_new || !v_new) return fail(SAGA_ERR_ARG, "NULL tensor pointer");
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) || !aligned16(v_new))
+    return fail(SAGA_ERR_ARG, "tensor pointers must be 16-byte aligned");
+  if (pos < 0 || pos >= s->l_cap) return fail(SAGA_ERR_ARG, "pos=%d outside [0, l_cap=%d)", pos, s->l_cap);
+  AppendParams p{};
+  p.k_cache = static_cast<uint16_t*>(k_cache);
+  p.v_cache = static_cast<uint16_t*>(v_cache);
+  p.k_new = static_cast<const uint16_t*>(k_new);
+  p.v_new = static_cast<const uint16_t*>(v_new);
+  p.seq_len_dev = seq_len_dev;
+  p.status = nullptr;
+  p.pos = pos;
+  p.batch = s->batch;
+  p.h_k = s->h_k;
+  p.h_v = s->h_v;
+  p.d = s->d;
+  p.l_cap = s->l_cap;
+  cudaError_t e = launch_append(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  return ok();
+}
+
+int atopn_refresh_threshold(const saga_shape* s, const void* q, const void* k_cache, int seq_len,
+                            const int* seq_len_dev, int n_top, float* tau, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  int rc = validate_shape(s);
+  if (rc) return rc;
+  if (!q || !k_cache || !tau) return fail(SAGA_ERR_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k_cache)) return fail(SAGA_ERR_ARG, "q and k_cache must be 16-byte aligned");
+  if (seq_len < 1 || seq_len > s->l_cap) return fail(SAGA_ERR_ARG, "seq_len=%d outside [1, l_cap=%d]", seq_len, s->l_cap);
+  if (n_top < 1) return fail(SAGA_ERR_ARG, "n_top=%d must be >= 1", n_top);
+  Prepared pr;
+  rc = prepare_ws(s, workspace, ws_bytes, &pr);
+  if (rc) return rc;
+  rc = run_refresh(s, pr, q, k_cache, seq_len, seq_len_dev, n_top, tau, static_cast<cudaStream_t>(stream));
+  if (rc) return rc;
+  return ok();
+}
+
+int atopn_select_threshold(const float* scores, int rows, int row_len, long long row_stride, int n_top, float* tau,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  if (!scores || !tau) return fail(SAGA_ERR_ARG, "NULL pointer");
+  if (rows < 1 || row_len < 1 || row_stride < row_len || (row_stride & 3) != 0)
+    return fail(SAGA_ERR_ARG, "bad rows=%d row_len=%d row_stride=%lld", rows, row_len, row_stride);
+  if (!aligned16(scores)) return fail(SAGA_ERR_ARG, "scores must be 16-byte aligned");
+  if (n_top < 1) return fail(SAGA_ERR_ARG, "n_top=%d must be >= 1", n_top);
+  if (workspace == nullptr || ws_bytes < atopn_select_workspace_bytes(rows))
+    return fail(SAGA_ERR_WORKSPACE, "workspace too small");
+  SelectParams sp{};
+  sp.scores = scores;
+  sp.ld = row_stride;
+  sp.hist = nullptr;
+  sp.tau = tau;
+  sp.status = static_cast<unsigned*>(workspace);
+  sp.seq_len_dev = nullptr;
+  sp.row_len = row_len;
+  sp.l_cap = row_len;
+  sp.n_top = n_top;
+  cudaError_t e = launch_select(sp, rows, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "radix select launch");
+  return ok();
+}
+
+int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, const void* v_cache, int seq_len,
+                     const int* seq_len_dev, int n_top, int refresh_interval, long long step, float* tau, void* out,
+                     int out_dtype, int* sel_count, int* sel_idx, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = validate_shape(s);
+  if (rc) return rc;
+  if (!q || !k_cache || !v_cache || !tau || !out) return fail(SAGA_ERR_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return fail(SAGA_ERR_ARG, "tensor pointers must be 16-byte aligned");
+  if (seq_len < 1 || seq_len > s->l_cap) return fail(SAGA_ERR_ARG, "seq_len=%d outside [1, l_cap=%d]", seq_len, s->l_cap);
+  if (n_top < 1) return fail(SAGA_ERR_ARG, "n_top=%d must be >= 1", n_top);
+  if (refresh_interval < 1) return fail(SAGA_ERR_ARG, "refresh_interval=%d must be >= 1", refresh_interval);
+  if (step < 0) return fail(SAGA_ERR_ARG, "step=%lld must be >= 0", step);
+  if (out_dtype != SAGA_OUT_F32 && out_dtype != SAGA_OUT_BF16) return fail(SAGA_ERR_ARG, "bad out_dtype %d", out_dtype);
+  if (sel_idx != nullptr && sel_count == nullptr) return fail(SAGA_ERR_ARG, "sel_idx requires sel_count");
+  Prepared pr;
+  rc = prepare_ws(s, workspace, ws_bytes, &pr);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G = s->h_q / s->h_k, NP = np_for_group(G);
+  const bool refresh = (step % refresh_interval) == 0;
+  const bool no_threshold = n_top >= s->l_cap;  // every possible length is covered by N
+  const int rows = s->batch * s->h_q;
+
+  CUtensorMap tf, tp;
+  rc = make_key_map(&tf, k_cache, s, kTile);
+  if (rc) return rc;
+  rc = make_key_map(&tp, k_cache, s, kUnit);
+  if (rc) return rc;
+
+  cudaEvent_t ev0 = g_trace_start, ev1 = g_trace_end;
+  g_trace_start = g_trace_end = nullptr;
+  if (ev0 != nullptr) {
+    cudaError_t et = trace_record(ev0, st);
+    if (et != cudaSuccess) return cuda_fail(et, "trace event record");
+  }
+
+  SplitParams p;
+  fill_split_common(p, s, pr, q, seq_len, seq_len_dev);
+  p.v_cache = static_cast<const uint16_t*>(v_cache);
+  p.tau = tau;
+  p.want_counts = sel_count != nullptr;
+  p.idxbuf = sel_idx != nullptr ? reinterpret_cast<int*>(pr.base + pr.ws.idx) : nullptr;
+  cudaError_t e;
+  int S = 1;
+  if (refresh && !no_threshold) {
+    rc = run_refresh(s, pr, q, k_cache, seq_len, seq_len_dev, n_top, tau, st);
+    if (rc) return rc;
+    rc = splits_for(s, pr, seq_len, NP, true, tf, tp, &S);
+    if (rc) return rc;
+    p.scores_in = reinterpret_cast<const float*>(pr.base + pr.ws.scores);
+    p.nsplit = S;
+    e = launch_from_scores(s->d, NP, p, dim3(S, s->h_k, s->batch), st);
+    if (e != cudaSuccess) return cuda_fail(e, "from-scores launch");
+  } else {
+    if (refresh) {
+      e = launch_fill(tau, -INFINITY, rows, st);
+      if (e != cudaSuccess) return cuda_fail(e, "threshold fill launch");
+    }
+    rc = splits_for(s, pr, seq_len, NP, false, tf, tp, &S);
+    if (rc) return rc;
+    p.nsplit = S;
+    e = launch_split(s->d, NP, false, tf, tp, p, dim3(S, s->h_k, s->batch), st, nullptr);
+    if (e != cudaSuccess) return cuda_fail(e, "split launch");
+  }
+  if (ev1 != nullptr) {
+    e = trace_record(ev1, st);
+    if (e != cudaSuccess) return cuda_fail(e, "trace event record");
+  }
+  CombineParams c{};
+  c.part_o = p.part_o;
+  c.part_m = p.part_m;
+  c.part_l = p.part_l;
+  c.part_cnt = p.part_cnt;
+  c.idxbuf = p.idxbuf;
+  c.out = out;
+  c.sel_count = sel_count;
+  c.sel_idx = sel_idx;
+  c.status = p.status;
+  c.seq_len_dev = seq_len_dev;
+  c.seq_len = seq_len;
+  c.rows = rows;
+  c.nsplit = S;
+  c.s_cap = pr.ws.s_cap;
+  c.l_cap = s->l_cap;
+  c.out_bf16 = out_dtype == SAGA_OUT_BF16;
+  e = launch_combine(s->d, c, st);
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  return ok();
+}
+
+int saga_trace_next_attention(void* ev_start, void* ev_end) {
+  if ((ev_start == nullptr) != (ev_end == nullptr)) return fail(SAGA_ERR_ARG, "pass both events or neither");
+  g_trace_start = static_cast<cudaEvent_t>(ev_start);
+  g_trace_end = static_cast<cudaEvent_t>(ev_end);
+  return ok();
+}
+
+int saga_get_status(const void* workspace, void* stream, unsigned* status) {
+  if (workspace == nullptr || status == nullptr) return fail(SAGA_ERR_ARG, "NULL pointer");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  e = cudaMemcpy(status, workspace, sizeof(unsigned), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+"""The C-ABI library on a machine without a GPU: it loads, it exports every
+entry point include/saga.h declares, and argument validation rejects bad
+calls before anything touches CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_decoding_saga_b200 import build as build_mod
+from long_context_decoding_saga_b200 import saga
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return saga.load()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "saga.h")).read()
+    return sorted(set(re.findall(r"SAGA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert set(declared_symbols()) == set(saga.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert lib.saga_abi_version() == 100
+
+
+def _shape(**kw):
+    base = dict(batch=1, h_q=8, h_k=1, h_v=8, d=64, l_cap=1024)
+    base.update(kw)
+    return saga.SagaShape.of(**base)
+
+
+FAKE = ctypes.c_void_p(0x100000)  # never dereferenced: validation fails first
+
+
+def _decode(lib, shape, seq_len=10, n_top=4, R=2, step=0, out_dtype=0, ptrs=True, sel_idx=None, sel_count=None):
+    p = FAKE if ptrs else None
+    return lib.saga_decode_attn(ctypes.byref(shape), p, p, p, seq_len, None, n_top, R, step, p, p, out_dtype,
+                                sel_count, sel_idx, p, 1 << 30, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), saga.SAGA_ERR_UNSUPPORTED),
+    (dict(h_q=6, h_k=4), saga.SAGA_ERR_ARG),
+    (dict(h_q=8, h_v=3), saga.SAGA_ERR_ARG),
+    (dict(h_q=12, h_k=3, h_v=2), saga.SAGA_ERR_UNSUPPORTED),
+    (dict(h_q=128, h_k=1), saga.SAGA_ERR_UNSUPPORTED),
+    (dict(batch=0), saga.SAGA_ERR_ARG),
+    (dict(l_cap=0), saga.SAGA_ERR_ARG),
+])
+def test_bad_shapes_rejected(lib, kw, code):
+    s = _shape(**kw)
+    assert _decode(lib, s) == code
+    assert lib.saga_last_error()
+    assert lib.saga_workspace_bytes(ctypes.byref(s)) == 0
+
+
+@pytest.mark.parametrize("kw", [dict(seq_len=0), dict(seq_len=1025), dict(n_top=0), dict(R=0), dict(step=-1),
+                                dict(out_dtype=7), dict(ptrs=False), dict(sel_idx=FAKE)])
+def test_bad_arguments_rejected(lib, kw):
+    assert _decode(lib, _shape(), **kw) == saga.SAGA_ERR_ARG
+    assert lib.saga_last_error()
+
+
+def test_append_and_select_validation(lib):
+    s = _shape()
+    assert lib.saga_kv_append(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, 1024, None, None) == saga.SAGA_ERR_ARG
+    assert lib.saga_kv_append(ctypes.byref(s), None, FAKE, FAKE, FAKE, 0, None, None) == saga.SAGA_ERR_ARG
+    assert lib.atopn_select_threshold(FAKE, 4, 10, 6, 3, FAKE, FAKE, 256, None) == saga.SAGA_ERR_ARG
+    assert lib.atopn_select_threshold(FAKE, 4, 10, 12, 0, FAKE, FAKE, 256, None) == saga.SAGA_ERR_ARG
+    assert lib.atopn_select_threshold(FAKE, 4, 10, 12, 3, FAKE, None, 0, None) == saga.SAGA_ERR_WORKSPACE
+    assert lib.atopn_refresh_threshold(ctypes.byref(s), FAKE, FAKE, 5, None, 0, FAKE, FAKE, 1, None) == saga.SAGA_ERR_ARG
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    s = _shape()
+    with pytest.raises(ValueError):
+        saga.saga_kv_append(s, torch.zeros(1, 1, 1024, 64, dtype=torch.bfloat16),
+                            torch.zeros(1, 8, 1024, 64, dtype=torch.bfloat16),
+                            torch.zeros(1, 1, 64, dtype=torch.bfloat16), torch.zeros(1, 8, 64, dtype=torch.bfloat16), 0)

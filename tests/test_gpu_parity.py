@@ -1,0 +1,191 @@
+"""Parity of the CUDA decode path with the CPU oracle (needs a B200)."""
+import numpy as np
+import pytest
+import torch
+
+from long_context_decoding_saga_b200 import saga, workload
+from oracle import saga_oracle
+from tests import gpu_harness
+
+pytestmark = pytest.mark.gpu
+
+W = workload.Workload
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from long_context_decoding_saga_b200 import build
+    build.build()
+    saga.load()
+
+
+def small(name, **kw):
+    base = dict(name=name, batch=1, h_q=8, h_k=1, h_v=8, d=64, l_kv=1000, layers=1, steps=12, n_top=40, refresh=4,
+                planted=0.02, q_mode="planted_mean", seed=7)
+    base.update(kw)
+    return W(**base)
+
+
+# Shapes spanning both scoring paths (CUDA cores for h_q/h_k <= 4, tcgen05 above), d = 64 and 128, value
+# heads above / equal to / below the key heads, batch > 1, ragged lengths (not multiples of 32 or 128).
+CASES = [
+    small("g8_d64", h_q=8, h_k=1, h_v=8, d=64, l_kv=1000),
+    small("g12_d128_hv4", h_q=12, h_k=1, h_v=4, d=128, l_kv=2085, n_top=50),
+    small("g16_d64_b2", batch=2, h_q=32, h_k=2, h_v=8, d=64, l_kv=1531, n_top=64),
+    small("g32_d64", h_q=32, h_k=1, h_v=8, d=64, l_kv=777, n_top=33),
+    small("g64_d64", h_q=64, h_k=1, h_v=16, d=64, l_kv=650, n_top=20),
+    small("g4_d64_gqa", h_q=32, h_k=8, h_v=8, d=64, l_kv=1100, n_top=30),
+    small("g2_d128_hv_lt_hk", h_q=8, h_k=4, h_v=2, d=128, l_kv=903, n_top=25),
+    small("g1_mha_d128", h_q=4, h_k=4, h_v=4, d=128, l_kv=300, n_top=9, batch=3),
+    small("g16_d128_r1", h_q=16, h_k=1, h_v=2, d=128, l_kv=1290, n_top=100, refresh=1, steps=5),
+    small("g8_n1", h_q=8, h_k=1, h_v=8, d=64, l_kv=500, n_top=1, refresh=3),
+    small("tiny_l", h_q=8, h_k=2, h_v=4, d=64, l_kv=5, n_top=3, refresh=2, steps=6),
+    small("n_gt_l", h_q=8, h_k=1, h_v=8, d=64, l_kv=40, n_top=60, refresh=2, steps=30),
+    small("dense_g4", h_q=16, h_k=4, h_v=4, d=64, l_kv=1500, n_top=workload.DENSE, refresh=1 << 30,
+          q_mode="gaussian", planted=0.0, steps=4),
+    small("dense_g12_d128", h_q=12, h_k=1, h_v=4, d=128, l_kv=700, n_top=workload.DENSE, refresh=1 << 30,
+          q_mode="gaussian", planted=0.0, steps=3),
+]
+
+
+@pytest.mark.parametrize("wl", CASES, ids=lambda w: w.name)
+def test_decode_matches_oracle(wl):
+    reports, _ = gpu_harness.run_parity(wl, wl.steps)
+    assert len(reports) == wl.steps
+    assert reports[0].refreshed
+
+
+def test_tiny_config_full():
+    """The tiny configuration, all 32 steps: 1 layer, l_kv=1024, h_q=8, h_k=1, h_v=8, N=64, R=8."""
+    reports, _ = gpu_harness.run_parity(workload.TINY, workload.TINY.steps)
+    assert sum(r.refreshed for r in reports) == 4
+
+
+def test_graph_replay_matches_oracle():
+    wl = small("graphs", h_q=12, h_k=1, h_v=4, d=128, l_kv=3001, n_top=70, refresh=3, steps=8)
+    reports, _ = gpu_harness.run_parity(wl, wl.steps, graphs=True)
+    assert len(reports) == wl.steps
+
+
+def test_bf16_output_is_rounded_fp32_output():
+    wl = small("bf16", h_q=12, h_k=1, h_v=4, d=128, l_kv=1200, n_top=40, steps=3)
+    _, s32 = gpu_harness.run_parity(wl, wl.steps)
+    _, s16 = gpu_harness.run_parity(wl, wl.steps, out_dtype=torch.bfloat16)
+    assert torch.equal(s32.out.to(torch.bfloat16), s16.out)
+
+
+def test_runs_are_bitwise_deterministic():
+    wl = small("det", h_q=32, h_k=2, h_v=8, d=64, l_kv=4000, n_top=64, steps=5)
+    _, a = gpu_harness.run_parity(wl, wl.steps)
+    _, b = gpu_harness.run_parity(wl, wl.steps)
+    assert torch.equal(a.out, b.out) and torch.equal(a.tau, b.tau) and torch.equal(a.sel_idx, b.sel_idx)
+
+
+def test_kv_append_bit_exact():
+    shape = saga.SagaShape.of(2, 8, 2, 4, 128, 64)
+    g = torch.Generator(device="cuda").manual_seed(3)
+    kc = torch.randn((2, 2, 64, 128), device="cuda", generator=g).to(torch.bfloat16)
+    vc = torch.randn((2, 4, 64, 128), device="cuda", generator=g).to(torch.bfloat16)
+    kn = torch.randn((2, 2, 128), device="cuda", generator=g).to(torch.bfloat16)
+    vn = torch.randn((2, 4, 128), device="cuda", generator=g).to(torch.bfloat16)
+    ref_k, ref_v = kc.clone(), vc.clone()
+    ref_k[:, :, 17] = kn
+    ref_v[:, :, 17] = vn
+    saga.saga_kv_append(shape, kc, vc, kn, vn, 17)
+    torch.cuda.synchronize()
+    assert torch.equal(kc, ref_k) and torch.equal(vc, ref_v)
+
+
+def _select_rows():
+    rng = np.random.default_rng(5)
+    rows = []
+    for n in (1, 2, 3, 5, 31, 32, 33, 1000, 4097, 65536 + 7):
+        rows.append(rng.standard_normal(n).astype(np.float32))
+    rows.append(np.round(rng.standard_normal(3000) * 4).astype(np.float32))   # heavy ties
+    rows.append(np.full(777, 1.25, np.float32))                              # all equal
+    z = rng.standard_normal(500).astype(np.float32)
+    z[::3] = 0.0
+    z[1::7] = -0.0
+    rows.append(z)                                                           # signed zeros
+    rows.append((rng.standard_normal(20000) * 1e-30).astype(np.float32))   # tiny magnitudes
+    rows.append(np.concatenate([rng.standard_normal(40000), 1e30 * rng.standard_normal(50)]).astype(np.float32))
+    return rows
+
+
+def test_radix_select_matches_oracle_nth_largest():
+    rows = _select_rows()
+    ws = torch.zeros(saga.load().atopn_select_workspace_bytes(1), dtype=torch.uint8, device="cuda")
+    for row in rows:
+        L = row.size
+        stride = (L + 3) // 4 * 4
+        buf = np.zeros((1, stride), np.float32)
+        buf[0, :L] = row
+        dev = torch.from_numpy(buf).cuda()
+        for n in sorted({1, 2, max(1, L // 3), max(1, L - 1), L, L + 5}):
+            tau = torch.zeros(1, device="cuda")
+            saga.atopn_select_threshold(dev, L, n, tau, ws)
+            torch.cuda.synchronize()
+            expect = saga_oracle.nth_largest(row, n)
+            got = float(tau.item())
+            assert (got == expect) or (np.isneginf(got) and np.isneginf(expect)), (L, n, got, expect)
+
+
+def test_refresh_threshold_entry_point():
+    wl = small("refresh_ep", h_q=12, h_k=1, h_v=4, d=128, l_kv=5000, n_top=77)
+    inp = workload.make_layer(wl, 0, steps=1)
+    shape = saga.SagaShape.of(1, 12, 1, 4, 128, 5000)
+    kc = inp["K0"].cuda().contiguous()
+    q = inp["q"][0].cuda().contiguous()
+    tau = torch.zeros((1, 12), device="cuda")
+    ws = saga.alloc_workspace(shape)
+    saga.atopn_refresh_threshold(shape, q, kc, 5000, 77, tau, ws)
+    torch.cuda.synchronize()
+    expect = saga_oracle.refresh_threshold(inp["q"][0].float().numpy(), inp["K0"].float().numpy(), 5000, 77)
+    assert np.max(np.abs(tau.cpu().numpy() - expect)) <= gpu_harness.BAND
+
+
+def test_empty_selection_gives_zero():
+    """A stale threshold above every score of a later step keeps nothing: output 0, count 0."""
+    shape = saga.SagaShape.of(1, 8, 1, 8, 64, 600)
+    g = torch.Generator(device="cuda").manual_seed(11)
+    sess_inp = {
+        "K0": torch.randn((1, 1, 598, 64), device="cuda", generator=g).to(torch.bfloat16),
+        "V0": torch.randn((1, 8, 598, 64), device="cuda", generator=g).to(torch.bfloat16),
+    }
+    from long_context_decoding_saga_b200.session import DecodeSession
+    s = DecodeSession(shape, 1, 1, 2, track_selection=True)
+    s.prefill(0, sess_inp["K0"], sess_inp["V0"])
+    q = torch.randn((1, 1, 8, 64), device="cuda", generator=g).to(torch.bfloat16)
+    kn = torch.zeros((1, 1, 1, 64), device="cuda", dtype=torch.bfloat16)
+    vn = torch.randn((1, 1, 8, 64), device="cuda", generator=g).to(torch.bfloat16)
+    s.step(q, kn, vn)
+    torch.cuda.synchronize()
+    assert (s.tau > 0).all() and (s.sel_count == 1).all()
+    s.step(torch.zeros_like(q), kn, vn)
+    torch.cuda.synchronize()
+    assert (s.sel_count == 0).all()
+    assert (s.out == 0).all()
+
+
+def test_workspace_too_small_is_rejected():
+    shape = saga.SagaShape.of(1, 8, 1, 8, 64, 256)
+    ws = torch.zeros(saga.saga_workspace_bytes(shape) - 256, dtype=torch.uint8, device="cuda")
+    z = lambda *s, dt=torch.bfloat16: torch.zeros(s, dtype=dt, device="cuda")  # noqa: E731
+    with pytest.raises(saga.SagaError) as e:
+        saga.saga_decode_attn(shape, z(1, 8, 64), z(1, 1, 256, 64), z(1, 8, 256, 64), 10, 4, 2, 0,
+                              z(1, 8, dt=torch.float32), z(1, 8, 64, dt=torch.float32), ws)
+    assert e.value.code == saga.SAGA_ERR_WORKSPACE
+
+
+def test_device_length_out_of_range_is_clamped_and_flagged():
+    shape = saga.SagaShape.of(1, 8, 1, 8, 64, 256)
+    ws = saga.alloc_workspace(shape)
+    z = lambda *s, dt=torch.bfloat16: torch.zeros(s, dtype=dt, device="cuda")  # noqa: E731
+    lens = torch.tensor([100000], dtype=torch.int32, device="cuda")
+    saga.saga_decode_attn(shape, z(1, 8, 64), z(1, 1, 256, 64), z(1, 8, 256, 64), 10, 4, 2, 0,
+                          z(1, 8, dt=torch.float32), z(1, 8, 64, dt=torch.float32), ws, seq_len_dev=lens)
+    st = saga.saga_get_status(ws)
+    assert st & saga.SAGA_STATUS_LEN_CLAMPED
+    assert not st & saga.SAGA_STATUS_TIMEOUT
