@@ -101,7 +101,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:  # noqa: BLE001
             self.proc = None
             return
@@ -269,6 +269,7 @@ def run_saga(args, wl, rank, world, local_rank):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     bytes_timed = 0
     refresh_steps = 0
+    torch.cuda.nvtx.range_push("bench_timed")
     ev0.record()
     for _ in range(K):
         L = sess.length + 1
@@ -278,6 +279,7 @@ def run_saga(args, wl, rank, world, local_rank):
         sess.replay()
         cur += 1
     ev1.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     clocks = sampler.stop()
     ms = ev0.elapsed_time(ev1)
@@ -401,9 +403,12 @@ def main():
     ap.add_argument("--workload", default="qwen2.5-1.5b_saga_128k")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     args = ap.parse_args()
     from long_context_decoding_saga_b200 import workload
     wl = workload.CONFIGS[args.workload]
+    if args.layers > 0:
+        wl = wl.with_(layers=args.layers)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -32,7 +32,7 @@
  *   - Query head j reads key head floor(j*h_k/h_q) and value head
  *     floor(j*h_v/h_q) (contiguous groups).  Requires h_q % h_k == 0,
  *     h_q % h_v == 0 and (h_v % h_k == 0 or h_k % h_v == 0);
- *     1 <= h_q/h_k <= 64; d in {64, 128}.
+ *     1 <= h_q/h_k <= 64 (<= 32 when d = 128); d in {64, 128}; h_v/h_k <= 32.
  *   - Sequence length: `seq_len` is the number of valid cached tokens,
  *     including the token appended this step (1 <= seq_len <= l_cap).  If
  *     `seq_len_dev` is not NULL the kernels read the length from that device

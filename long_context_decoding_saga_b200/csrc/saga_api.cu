@@ -92,11 +92,9 @@ int validate_shape(const saga_shape* s) {
     return fail(SAGA_ERR_UNSUPPORTED, "one of h_k=%d, h_v=%d must divide the other", s->h_k, s->h_v);
   const int G = s->h_q / s->h_k;
   if (G > kMaxG) return fail(SAGA_ERR_UNSUPPORTED, "h_q/h_k=%d exceeds %d", G, kMaxG);
+  if (s->d == 128 && G > 32) return fail(SAGA_ERR_UNSUPPORTED, "d=128 supports h_q/h_k <= 32 (got %d)", G);
   const int nvh = s->h_v >= s->h_k ? s->h_v / s->h_k : 1;
   if (nvh > kMaxNvh) return fail(SAGA_ERR_UNSUPPORTED, "h_v/h_k=%d exceeds %d", nvh, kMaxNvh);
-  const int hpv = G / nvh;
-  const int P = nvh * (s->d / 4) * ((hpv + 3) / 4);
-  if (P > 4 * kEpiThreads) return fail(SAGA_ERR_UNSUPPORTED, "head layout too wide for one CTA (P=%d)", P);
   if ((long long)s->batch * s->h_k * s->l_cap >= (1ll << 31) ||
       (long long)s->batch * s->h_v * s->l_cap >= (1ll << 31) || (long long)s->batch * s->h_q >= (1 << 24))
     return fail(SAGA_ERR_UNSUPPORTED, "cache too large for 32-bit row coordinates");
@@ -244,7 +242,7 @@ int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, boo
 // Scores of every cached token, their top-byte histograms, and the exact
 // threshold (refresh).
 int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const void* k_cache, int seq_len,
-                const int* seq_len_dev, int n_top, float* tau, cudaStream_t st) {
+                const int* seq_len_dev, int n_top, float* tau, cudaStream_t st, cudaEvent_t ev_start = nullptr) {
   const int G = s->h_q / s->h_k, NP = np_for_group(G);
   CUtensorMap tf, tp;
   int rc = make_key_map(&tf, k_cache, s, kTile);
@@ -256,6 +254,10 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   if (rc) return rc;
   const size_t rows = (size_t)s->batch * s->h_q;
   uint32_t* hist = reinterpret_cast<uint32_t*>(pr.base + pr.ws.hist);
+  if (ev_start != nullptr) {
+    cudaError_t et = trace_record(ev_start, st);
+    if (et != cudaSuccess) return cuda_fail(et, "trace event record");
+  }
   cudaError_t e = cudaMemsetAsync(hist, 0, rows * 256 * 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(hist)");
   SplitParams p;
@@ -398,10 +400,6 @@ int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, co
 
   cudaEvent_t ev0 = g_trace_start, ev1 = g_trace_end;
   g_trace_start = g_trace_end = nullptr;
-  if (ev0 != nullptr) {
-    cudaError_t et = trace_record(ev0, st);
-    if (et != cudaSuccess) return cuda_fail(et, "trace event record");
-  }
 
   SplitParams p;
   fill_split_common(p, s, pr, q, seq_len, seq_len_dev);
@@ -412,7 +410,7 @@ int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, co
   cudaError_t e;
   int S = 1;
   if (refresh && !no_threshold) {
-    rc = run_refresh(s, pr, q, k_cache, seq_len, seq_len_dev, n_top, tau, st);
+    rc = run_refresh(s, pr, q, k_cache, seq_len, seq_len_dev, n_top, tau, st, ev0);
     if (rc) return rc;
     rc = splits_for(s, pr, seq_len, NP, true, tf, tp, &S);
     if (rc) return rc;
@@ -421,13 +419,17 @@ int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, co
     e = launch_from_scores(s->d, NP, p, dim3(S, s->h_k, s->batch), st);
     if (e != cudaSuccess) return cuda_fail(e, "from-scores launch");
   } else {
+    rc = splits_for(s, pr, seq_len, NP, false, tf, tp, &S);
+    if (rc) return rc;
+    p.nsplit = S;
+    if (ev0 != nullptr) {
+      e = trace_record(ev0, st);
+      if (e != cudaSuccess) return cuda_fail(e, "trace event record");
+    }
     if (refresh) {
       e = launch_fill(tau, -INFINITY, rows, st);
       if (e != cudaSuccess) return cuda_fail(e, "threshold fill launch");
     }
-    rc = splits_for(s, pr, seq_len, NP, false, tf, tp, &S);
-    if (rc) return rc;
-    p.nsplit = S;
     e = launch_split(s->d, NP, false, tf, tp, p, dim3(S, s->h_k, s->batch), st, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "split launch");
   }

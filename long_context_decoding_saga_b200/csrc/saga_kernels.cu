@@ -23,6 +23,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "saga_device.cuh"
@@ -56,305 +57,400 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   }
 }
 
-template <int D>
-__host__ __device__ constexpr int split_stages() { return D == 128 ? 4 : 6; }
+template <int D, int NP>
+__host__ __device__ constexpr int split_stages() { return D == 128 ? (NP >= 64 ? 3 : 4) : 6; }
 
 template <int NP>
 __host__ __device__ constexpr uint32_t tmem_cols() { return (2 * NP <= 32) ? 32u : (2 * NP <= 64) ? 64u : 128u; }
 
 // ============================================================================ epilogue
-// Per-tile staging: union rows (tokens kept by at least one query head of the
-// group), their value-head bits and softmax weights, written in phase A of a
-// tile and consumed by phase B one tile later (so the L2 prefetch of the
-// value rows issued in phase A overlaps the next tile's key stream).
-template <int NP>
-struct EpiSlot {
-  float w[kTile][NP];
-  int tok[kTile];
-  uint32_t vmask[kTile];
-  float factor[NP];
-  int nrows;
-  int active;
-};
+// Each of the four epilogue warps owns 32 token rows of every tile (its TMEM
+// lane quarter) and keeps its own online softmax, so no barrier couples the
+// warps inside the tile loop.  Per tile a warp only compares its scores with
+// the Atop-N thresholds (step 1) and, when some of its rows are kept, appends
+// them (token, scores, head mask) to a warp-private list and starts copying
+// their value rows into shared memory.  The softmax and the value sum of
+// eq. 7 run per batch: when a list buffer is full (double-buffered, one
+// refill behind) and at the end.  The four warps' partials are merged last.
+constexpr int kBatch = 32;  // rows per list buffer
 
-constexpr int kRedFloats = 2048;  // G*D bound when row groups are reduced (see EpiCtx)
+template <int NP>
+struct WarpList {
+  float sc[kBatch][NP];   // scores of the row for every head; overwritten by the weights
+  uint64_t keep[kBatch];  // heads that keep the row
+  int tok[kBatch];
+};
 
 template <int NP>
 struct EpiShared {
-  EpiSlot<NP> slot[2];
-  float tau[NP];
-  float m_run[NP];
-  float wmax[4][NP];
-  int wrows[4];
-  int hcnt[4][NP];
-  int cnt_run[NP];
-  float red_o[kRedFloats];
-  float red_l[kMaxG];
+  WarpList<NP> list[4][2];
+  alignas(16) float tau[NP];  // Atop-N thresholds (+inf for padding heads)
+  int vu[NP];                 // local value head of each query head of the group
+  int hcnt[4][NP];            // counting mode: per-warp kept counts of the current tile
+  int cnt_run[NP];            // counting mode: kept so far in this split
 };
 
-constexpr int kPT = 4;  // phase-B ownership slots per thread
+// Bytes of value rows each warp stages per list buffer.
+template <int NP>
+__host__ __device__ constexpr int vstage_warp_bytes() { return NP >= 64 ? 2048 : 4096; }
 
-// Phase-B ownership: thread et accumulates, for pair (value head u, 4-dim
-// chunk c, block hb of up to 4 query heads of u) and row group rg, the
-// running numerator and denominator of eq. 7.
-template <int D>
-struct EpiCtx {
-  int et, q, lane, erow;
-  int G, nvh, hpv, hb_n, P, RG;
-  int valid[kPT], u[kPT], c[kPT], hb[kPT], rg[kPT];
+struct EpiArgs {
+  const uint16_t* vgroup;  // V of the group's first value head, batch b
+  int l_cap, G, hpv, nvh;
+  int rcapw;  // rows per list buffer whose value rows are staged in shared memory
+  int cpr;    // 16-byte chunks of one row over the group's value heads
+  int hmul;   // ceil(65536 / hpv): (j * hmul) >> 16 == j / hpv for j < 64
+};
 
-  __device__ void init(int et_, int G_, int nvh_, int hpv_) {
-    et = et_;
-    lane = et_ & 31;
-    q = (threadIdx.x >> 5) & 3;
-    erow = 32 * q + lane;
-    G = G_;
-    nvh = nvh_;
-    hpv = hpv_;
-    hb_n = (hpv + 3) / 4;
-    P = nvh * (D / 4) * hb_n;
-    RG = P < kEpiThreads ? kEpiThreads / P : 1;
-    const int W = P * RG;
+// Per-lane online-softmax state: lane owns dims [lane*DPL, lane*DPL+DPL) of every head.
+template <int D, int NP>
+struct WarpAcc {
+  static constexpr int DPL = D / 32;
+  float m[NP];
+  float l[NP];
+  float o[NP][DPL];
+  __device__ __forceinline__ void init() {
 #pragma unroll
-    for (int i = 0; i < kPT; ++i) {
-      const int s = et + kEpiThreads * i;
-      valid[i] = s < W;
-      const int pair = s % P;
-      rg[i] = s / P;
-      c[i] = pair % (D / 4);
-      const int rest = pair / (D / 4);
-      hb[i] = rest % hb_n;
-      u[i] = rest / hb_n;
+    for (int j = 0; j < NP; ++j) {
+      m[j] = -INFINITY;
+      l[j] = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) o[j][e] = 0.f;
     }
   }
 };
 
-struct EpiAcc {
-  float o[kPT][4][4];
-  float l[kPT][4];
-  __device__ void zero() {
-#pragma unroll
-    for (int i = 0; i < kPT; ++i)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        l[i][k] = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[i][k][e] = 0.f;
-      }
-  }
+// A warp's list state: current buffer, its rows, and the full buffer waiting
+// to be reduced (-1 if none).
+struct ListState {
+  int cur, n, pend, npend;
 };
 
-template <int NP>
-__device__ void epi_setup(EpiShared<NP>& es, int et, const SplitParams& p, int b, int j0, bool load_tau) {
-  if (et < NP) {
-    es.tau[et] = (load_tau && et < p.G) ? p.tau[(size_t)b * p.h_q + j0 + et] : INFINITY;
-    es.m_run[et] = -INFINITY;
-    es.cnt_run[et] = 0;
-  }
-  for (int i = et; i < kRedFloats; i += kEpiThreads) es.red_o[i] = 0.f;
-  if (et < kMaxG) es.red_l[et] = 0.f;
+template <int D, int NP>
+__device__ __forceinline__ EpiArgs epi_args(const SplitParams& p, int b, int j0) {
+  EpiArgs ea;
+  const int v_base = (int)(((long long)j0 * p.h_v) / p.h_q);
+  ea.vgroup = p.v_cache + ((size_t)b * p.h_v + v_base) * (size_t)p.l_cap * D;
+  ea.l_cap = p.l_cap;
+  ea.G = p.G;
+  ea.hpv = p.hpv;
+  ea.nvh = p.nvh;
+  ea.rcapw = min(kBatch, vstage_warp_bytes<NP>() / (p.nvh * D * 2));
+  ea.cpr = p.nvh * D / 8;
+  ea.hmul = (65536 + p.hpv - 1) / p.hpv;
+  return ea;
 }
 
-// Phase A of tile `slot_i`: threshold compare (Atop-N step 1), per-head tile
-// max, compaction of the union rows, softmax weights, L2 prefetch of the
-// value rows, and (optionally) per-head counts and ascending index lists.
-template <int D, int NP>
-__device__ void phase_a(EpiShared<NP>& es, int slot_i, const float (&sc)[NP], int tok, bool valid, const EpiCtx<D>& cx,
-                        const SplitParams& p, int b, int j0, int chunk_start, const uint16_t* vgroup) {
-  EpiSlot<NP>& sl = es.slot[slot_i];
+template <int NP>
+__device__ __forceinline__ void epi_setup(EpiShared<NP>& es, int et, const SplitParams& p, int b, int j0,
+                                          bool load_tau) {
+  if (et < NP) {
+    es.tau[et] = (load_tau && et < p.G) ? __ldg(p.tau + (size_t)b * p.h_q + j0 + et) : INFINITY;
+    es.vu[et] = et < p.G ? et / p.hpv : 0;
+    es.cnt_run[et] = 0;
+  }
+}
+
+// Atop-N step 1 for the lane's token: bit j set when query head j keeps it.
+template <int NP>
+__device__ __forceinline__ uint64_t keep_mask(const EpiShared<NP>& es, const float (&sc)[NP], bool valid) {
   uint64_t keep = 0;
 #pragma unroll
-  for (int jl = 0; jl < NP; ++jl)
-    if (jl < cx.G && valid && sc[jl] >= es.tau[jl]) keep |= 1ull << jl;
-  const bool any = named_bar_or(1, kEpiThreads, keep != 0);
-  if (!any) {
-    if (cx.et == 0) sl.active = 0;
-    return;
+  for (int j4 = 0; j4 < NP / 4; ++j4) {
+    const float4 tv = *reinterpret_cast<const float4*>(&es.tau[4 * j4]);
+    if (sc[4 * j4 + 0] >= tv.x) keep |= 1ull << (4 * j4 + 0);
+    if (sc[4 * j4 + 1] >= tv.y) keep |= 1ull << (4 * j4 + 1);
+    if (sc[4 * j4 + 2] >= tv.z) keep |= 1ull << (4 * j4 + 2);
+    if (sc[4 * j4 + 3] >= tv.w) keep |= 1ull << (4 * j4 + 3);
+  }
+  return valid ? keep : 0ull;
+}
+
+// Softmax and value sum over list buffer bi (n rows) of this warp.
+template <int D, int NP>
+__device__ __forceinline__ void reduce_batch(EpiShared<NP>& es, WarpAcc<D, NP>& acc, const EpiArgs& ea, int q,
+                                             int lane, int bi, int n, const uint16_t* vstage_w, bool newest_pending) {
+  constexpr int DPL = WarpAcc<D, NP>::DPL;
+  if (newest_pending) {
+    asm volatile("cp.async.wait_group 1;" ::: "memory");  // the newest group belongs to the other buffer
+  } else {
+    cp_async_wait_all();
+  }
+  __syncwarp();
+  WarpList<NP>& li = es.list[q][bi];
+  const bool mine = lane < n;
+  const uint64_t keep = mine ? li.keep[lane] : 0ull;
+  float s[NP];
+#pragma unroll
+  for (int j4 = 0; j4 < NP / 4; ++j4) {
+    float4 v = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    if (mine) v = *reinterpret_cast<const float4*>(&li.sc[lane][4 * j4]);
+    s[4 * j4 + 0] = v.x;
+    s[4 * j4 + 1] = v.y;
+    s[4 * j4 + 2] = v.z;
+    s[4 * j4 + 3] = v.w;
+  }
+  // batch maximum per head (one reduction over order-preserving keys); raise
+  // the running maxima and rescale the running sums (warp-uniform branches)
+#pragma unroll
+  for (int jl = 0; jl < NP; ++jl) {
+    const uint32_t k = ((keep >> jl) & 1ull) ? float_key(s[jl]) : 0u;
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, k);
+    if (kmax != 0u) {
+      const float tm = key_float(kmax);
+      if (tm > acc.m[jl]) {
+        const float f = (acc.m[jl] == -INFINITY) ? 0.f : __expf(acc.m[jl] - tm);
+        acc.l[jl] *= f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc.o[jl][e] *= f;
+        acc.m[jl] = tm;
+      }
+    }
+  }
+  // weights of the lane's row, written over its scores
+  if (mine) {
+#pragma unroll
+    for (int j4 = 0; j4 < NP / 4; ++j4) {
+      float4 w;
+      w.x = ((keep >> (4 * j4 + 0)) & 1ull) ? __expf(s[4 * j4 + 0] - acc.m[4 * j4 + 0]) : 0.f;
+      w.y = ((keep >> (4 * j4 + 1)) & 1ull) ? __expf(s[4 * j4 + 1] - acc.m[4 * j4 + 1]) : 0.f;
+      w.z = ((keep >> (4 * j4 + 2)) & 1ull) ? __expf(s[4 * j4 + 2] - acc.m[4 * j4 + 2]) : 0.f;
+      w.w = ((keep >> (4 * j4 + 3)) & 1ull) ? __expf(s[4 * j4 + 3] - acc.m[4 * j4 + 3]) : 0.f;
+      *reinterpret_cast<float4*>(&li.sc[lane][4 * j4]) = w;
+    }
+  }
+  __syncwarp();
+  for (int r = 0; r < n; ++r) {
+    float w[NP];
+#pragma unroll
+    for (int j4 = 0; j4 < NP / 4; ++j4) {
+      const float4 v4 = *reinterpret_cast<const float4*>(&li.sc[r][4 * j4]);
+      w[4 * j4 + 0] = v4.x;
+      w[4 * j4 + 1] = v4.y;
+      w[4 * j4 + 2] = v4.z;
+      w[4 * j4 + 3] = v4.w;
+    }
+    if (r < ea.rcapw) {
+      // staged row: every value head of the group is in shared memory, so the
+      // loads need no branch (heads that do not keep the row have w = 0)
+      const uint16_t* vrow = vstage_w + ((size_t)bi * ea.rcapw + r) * ea.nvh * D + lane * DPL;
+#pragma unroll
+      for (int jl = 0; jl < NP; ++jl) {
+        if (jl < ea.G) {
+          const uint16_t* src = vrow + ((jl * ea.hmul) >> 16) * D;
+          float v[DPL];
+          if constexpr (DPL == 4) {
+            const uint2 raw = *reinterpret_cast<const uint2*>(src);
+            v[0] = bf16_lo(raw.x);
+            v[1] = bf16_hi(raw.x);
+            v[2] = bf16_lo(raw.y);
+            v[3] = bf16_hi(raw.y);
+          } else {
+            const uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
+            v[0] = bf16_lo(raw);
+            v[1] = bf16_hi(raw);
+          }
+          acc.l[jl] += w[jl];
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) acc.o[jl][e] = fmaf(w[jl], v[e], acc.o[jl][e]);
+        }
+      }
+    } else {
+      const uint16_t* vrow = ea.vgroup + (size_t)li.tok[r] * D + lane * DPL;
+#pragma unroll
+      for (int jl = 0; jl < NP; ++jl) {
+        if (w[jl] != 0.f) {  // same value in every lane
+          const uint16_t* src = vrow + (size_t)((jl * ea.hmul) >> 16) * ea.l_cap * D;
+          float v[DPL];
+          if constexpr (DPL == 4) {
+            const uint2 raw = __ldg(reinterpret_cast<const uint2*>(src));
+            v[0] = bf16_lo(raw.x);
+            v[1] = bf16_hi(raw.x);
+            v[2] = bf16_lo(raw.y);
+            v[3] = bf16_hi(raw.y);
+          } else {
+            const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(src));
+            v[0] = bf16_lo(raw);
+            v[1] = bf16_hi(raw);
+          }
+          acc.l[jl] += w[jl];
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) acc.o[jl][e] = fmaf(w[jl], v[e], acc.o[jl][e]);
+        }
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// Appends the warp's kept rows of one tile to its list (reducing a full
+// buffer one refill later) and starts staging their value rows.
+template <int D, int NP>
+__device__ __forceinline__ void append_rows(EpiShared<NP>& es, WarpAcc<D, NP>& acc, const EpiArgs& ea, ListState& ls,
+                                            int q, int lane, uint32_t bal, uint64_t keep, const float (&sc)[NP],
+                                            int tok, uint16_t* vstage_w) {
+  const int nnew = __popc(bal);
+  if (ls.n + nnew > kBatch) {
+    if (ls.pend >= 0) reduce_batch<D, NP>(es, acc, ea, q, lane, ls.pend, ls.npend, vstage_w, true);
+    ls.pend = ls.cur;
+    ls.npend = ls.n;
+    ls.cur ^= 1;
+    ls.n = 0;
+  }
+  WarpList<NP>& li = es.list[q][ls.cur];
+  if (keep != 0ull) {
+    const int pos = ls.n + __popc(bal & ((1u << lane) - 1u));
+    li.tok[pos] = tok;
+    li.keep[pos] = keep;
+#pragma unroll
+    for (int j4 = 0; j4 < NP / 4; ++j4)
+      *reinterpret_cast<float4*>(&li.sc[pos][4 * j4]) =
+          make_float4(sc[4 * j4 + 0], sc[4 * j4 + 1], sc[4 * j4 + 2], sc[4 * j4 + 3]);
+  }
+  __syncwarp();
+  // value rows (every value head of the group) of the new list entries:
+  // staged in shared memory while the buffer has room, otherwise warmed in L2
+  const int r0 = ls.n, r1 = ls.n + nnew;
+  const int rs = min(r1, ea.rcapw);
+  for (int it = lane; it < max(0, rs - r0) * ea.cpr; it += 32) {
+    const int ri = r0 + it / ea.cpr, ch = it % ea.cpr;
+    const int u = ch / (D / 8), cc = ch - u * (D / 8);
+    cp_async16(vstage_w + (((size_t)ls.cur * ea.rcapw + ri) * ea.nvh + u) * D + cc * 8,
+                 ea.vgroup + ((size_t)u * ea.l_cap + li.tok[ri]) * D + cc * 8);
+  }
+  for (int it = lane; it < max(0, r1 - max(r0, rs)) * ea.nvh * (D / 64); it += 32) {
+    const int per = ea.nvh * (D / 64);
+    const int ri = max(r0, rs) + it / per, rem = it % per;
+    const int u = rem / (D / 64), line = rem % (D / 64);
+    const char* src = reinterpret_cast<const char*>(ea.vgroup + ((size_t)u * ea.l_cap + li.tok[ri]) * D) + line * 128;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(src));
+  }
+  cp_async_commit();
+  ls.n = r1;
+}
+
+// Reduces whatever is left in the warp's lists.
+template <int D, int NP>
+__device__ __forceinline__ void flush_lists(EpiShared<NP>& es, WarpAcc<D, NP>& acc, const EpiArgs& ea, ListState& ls,
+                                            int q, int lane, const uint16_t* vstage_w) {
+  // the newest cp.async group belongs to the current buffer only if it holds rows
+  if (ls.pend >= 0) reduce_batch<D, NP>(es, acc, ea, q, lane, ls.pend, ls.npend, vstage_w, ls.n > 0);
+  if (ls.n > 0) reduce_batch<D, NP>(es, acc, ea, q, lane, ls.cur, ls.n, vstage_w, false);
+  ls.pend = -1;
+  ls.n = 0;
+}
+
+// Counting mode (kept counts and ascending index lists requested): the four
+// warps go through each tile together; per-head ballots give each kept
+// token its position in the split's list.
+template <int NP>
+__device__ __forceinline__ void count_tile(EpiShared<NP>& es, uint64_t keep, int q, int lane, int et, int tok,
+                                           const SplitParams& p, int b, int j0, int chunk_start) {
+#pragma unroll
+  for (int jl = 0; jl < NP; ++jl) {
+    if (jl < p.G) {
+      const uint32_t bl = __ballot_sync(0xffffffffu, (keep >> jl) & 1ull);
+      if (lane == 0) es.hcnt[q][jl] = __popc(bl);
+    }
+  }
+  named_bar_sync(1, kEpiThreads);
+  if (p.idxbuf != nullptr) {
+#pragma unroll
+    for (int jl = 0; jl < NP; ++jl) {
+      if (jl < p.G) {
+        const bool kb = (keep >> jl) & 1ull;
+        const uint32_t bl = __ballot_sync(0xffffffffu, kb);
+        if (kb) {
+          int off = es.cnt_run[jl];
+          for (int qq = 0; qq < q; ++qq) off += es.hcnt[qq][jl];
+          off += __popc(bl & ((1u << lane) - 1u));
+          p.idxbuf[((size_t)b * p.h_q + j0 + jl) * p.l_cap + chunk_start + off] = tok;
+        }
+      }
+    }
+  }
+  named_bar_sync(1, kEpiThreads);
+  if (et < p.G) es.cnt_run[et] += es.hcnt[0][et] + es.hcnt[1][et] + es.hcnt[2][et] + es.hcnt[3][et];
+}
+
+// Per tile of one warp: threshold compare, optional counting, list append.
+template <int D, int NP>
+__device__ __forceinline__ void tile_epilogue(EpiShared<NP>& es, WarpAcc<D, NP>& acc, const EpiArgs& ea,
+                                              ListState& ls, int q, int lane, int et, const float (&sc)[NP], int tok,
+                                              bool valid, bool counting, const SplitParams& p, int b, int j0,
+                                              int chunk_start, uint16_t* vstage_w) {
+  const uint64_t keep = keep_mask<NP>(es, sc, valid);
+  const uint32_t bal = __ballot_sync(0xffffffffu, keep != 0ull);
+  if (counting) count_tile<NP>(es, keep, q, lane, et, tok, p, b, j0, chunk_start);
+  if (bal != 0u) append_rows<D, NP>(es, acc, ea, ls, q, lane, bal, keep, sc, tok, vstage_w);
+}
+
+// Merges the four warps' (m, l, o) and writes the split's partial: every
+// warp writes its state, one thread per head forms the merge factors, and all
+// threads combine.  mrg holds 4 * NP * (D + 2) + 4 * NP floats, 16-byte
+// aligned.  Deterministic (fixed warp order in every sum).
+template <int D, int NP>
+__host__ __device__ constexpr int merge_floats() { return 4 * NP * (D + 2) + 4 * NP; }
+
+template <int D, int NP>
+__device__ __forceinline__ void merge_and_store(const EpiShared<NP>& es, float* mrg, WarpAcc<D, NP>& acc, int q,
+                                                int lane, int et, const SplitParams& p, int b, int j0, int s) {
+  constexpr int DPL = WarpAcc<D, NP>::DPL;
+  constexpr int REG = NP * (D + 2);
+  float* mine = mrg + q * REG;  // m[NP], l[NP], o[NP][D]
+  float* fac = mrg + 4 * REG;   // [4][NP]
+  if (lane == 0) {
+#pragma unroll
+    for (int j4 = 0; j4 < NP / 4; ++j4) {
+      *reinterpret_cast<float4*>(&mine[4 * j4]) =
+          make_float4(acc.m[4 * j4], acc.m[4 * j4 + 1], acc.m[4 * j4 + 2], acc.m[4 * j4 + 3]);
+      *reinterpret_cast<float4*>(&mine[NP + 4 * j4]) =
+          make_float4(acc.l[4 * j4], acc.l[4 * j4 + 1], acc.l[4 * j4 + 2], acc.l[4 * j4 + 3]);
+    }
   }
 #pragma unroll
   for (int jl = 0; jl < NP; ++jl) {
-    if (jl < cx.G) {
-      float v = ((keep >> jl) & 1ull) ? sc[jl] : -INFINITY;
-      v = warp_max(v);
-      if (cx.lane == 0) es.wmax[cx.q][jl] = v;
+    float* dst = &mine[2 * NP + jl * D + lane * DPL];
+    if constexpr (DPL == 4) {
+      *reinterpret_cast<float4*>(dst) = make_float4(acc.o[jl][0], acc.o[jl][1], acc.o[jl][2], acc.o[jl][3]);
+    } else {
+      *reinterpret_cast<float2*>(dst) = make_float2(acc.o[jl][0], acc.o[jl][1]);
     }
   }
-  const bool isrow = keep != 0;
-  const uint32_t bal = __ballot_sync(0xffffffffu, isrow);
-  if (cx.lane == 0) es.wrows[cx.q] = __popc(bal);
   named_bar_sync(1, kEpiThreads);
-  if (cx.et < cx.G) {
-    const int jl = cx.et;
-    const float tmax = fmaxf(fmaxf(es.wmax[0][jl], es.wmax[1][jl]), fmaxf(es.wmax[2][jl], es.wmax[3][jl]));
-    const float mold = es.m_run[jl];
-    const float mnew = fmaxf(mold, tmax);
-    sl.factor[jl] = (mnew == -INFINITY) ? 1.f : __expf(mold - mnew);
-    es.m_run[jl] = mnew;
-  }
-  int base = 0;
-  for (int qq = 0; qq < cx.q; ++qq) base += es.wrows[qq];
-  const int total = es.wrows[0] + es.wrows[1] + es.wrows[2] + es.wrows[3];
-  named_bar_sync(1, kEpiThreads);
-  if (isrow) {
-    const int pos = base + __popc(bal & ((1u << cx.lane) - 1u));
-    sl.tok[pos] = tok;
-    uint32_t vm = 0;
-#pragma unroll
-    for (int jl = 0; jl < NP; ++jl) {
-      if (jl < cx.G) {
-        float w = 0.f;
-        if ((keep >> jl) & 1ull) {
-          w = __expf(sc[jl] - es.m_run[jl]);
-          vm |= 1u << (jl / cx.hpv);
-        }
-        sl.w[pos][jl] = w;
-      }
-    }
-    sl.vmask[pos] = vm;
-    uint32_t bits = vm;
-    while (bits) {
-      const int u = __ffs(bits) - 1;
-      bits &= bits - 1;
-      prefetch_l2_bulk(vgroup + ((size_t)u * p.l_cap + tok) * D, D * 2);
-    }
-  }
-  if (cx.et == 0) {
-    sl.nrows = total;
-    sl.active = 1;
-  }
-  if (p.want_counts) {
-#pragma unroll
-    for (int jl = 0; jl < NP; ++jl) {
-      if (jl < cx.G) {
-        const uint32_t bl = __ballot_sync(0xffffffffu, (keep >> jl) & 1ull);
-        if (cx.lane == 0) es.hcnt[cx.q][jl] = __popc(bl);
-      }
-    }
-    named_bar_sync(1, kEpiThreads);
-    if (p.idxbuf != nullptr) {
-#pragma unroll
-      for (int jl = 0; jl < NP; ++jl) {
-        if (jl < cx.G) {
-          const bool kb = (keep >> jl) & 1ull;
-          const uint32_t bl = __ballot_sync(0xffffffffu, kb);
-          if (kb) {
-            int off = es.cnt_run[jl];
-            for (int qq = 0; qq < cx.q; ++qq) off += es.hcnt[qq][jl];
-            off += __popc(bl & ((1u << cx.lane) - 1u));
-            p.idxbuf[((size_t)b * p.h_q + j0 + jl) * p.l_cap + chunk_start + off] = tok;
-          }
-        }
-      }
-    }
-    named_bar_sync(1, kEpiThreads);
-    if (cx.et < cx.G)
-      es.cnt_run[cx.et] += es.hcnt[0][cx.et] + es.hcnt[1][cx.et] + es.hcnt[2][cx.et] + es.hcnt[3][cx.et];
-  }
-}
-
-// Phase B of tile `slot_i`: rescale the running sums to the new maxima and
-// add w * V[row] for every kept (row, query head) this thread owns.
-template <int D, int NP>
-__device__ void phase_b(EpiShared<NP>& es, int slot_i, const EpiCtx<D>& cx, const uint16_t* vgroup, int l_cap,
-                        EpiAcc& acc) {
-  EpiSlot<NP>& sl = es.slot[slot_i];
-  if (!sl.active) return;
-  const int nrows = sl.nrows;
-#pragma unroll
-  for (int i = 0; i < kPT; ++i) {
-    if (!cx.valid[i]) continue;
-    const int u = cx.u[i];
-    const int jb = u * cx.hpv + cx.hb[i] * 4;
-    const int nk = min(4, cx.hpv - cx.hb[i] * 4);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      if (k < nk) {
-        const float f = sl.factor[jb + k];
-        acc.l[i][k] *= f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc.o[i][k][e] *= f;
-      }
-    }
-    const uint16_t* vb = vgroup + (size_t)u * l_cap * D + cx.c[i] * 4;
-    const int step = cx.RG;
-    for (int r0 = cx.rg[i]; r0 < nrows; r0 += 4 * step) {
-      uint2 raw[4];
-      bool use[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const int r = r0 + t * step;
-        use[t] = (r < nrows) && ((sl.vmask[r] >> u) & 1u);
-        if (use[t]) raw[t] = __ldg(reinterpret_cast<const uint2*>(vb + (size_t)sl.tok[r] * D));
-      }
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        if (!use[t]) continue;
-        const int r = r0 + t * step;
-        const float v0 = bf16_lo(raw[t].x), v1 = bf16_hi(raw[t].x), v2 = bf16_lo(raw[t].y), v3 = bf16_hi(raw[t].y);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (k < nk) {
-            const float w = sl.w[r][jb + k];
-            acc.l[i][k] += w;
-            acc.o[i][k][0] = fmaf(w, v0, acc.o[i][k][0]);
-            acc.o[i][k][1] = fmaf(w, v1, acc.o[i][k][1]);
-            acc.o[i][k][2] = fmaf(w, v2, acc.o[i][k][2]);
-            acc.o[i][k][3] = fmaf(w, v3, acc.o[i][k][3]);
-          }
-        }
-      }
-    }
-  }
-}
-
-// Writes this split's partial (running max m, denominator l, numerator o)
-// for every query head of the group.
-template <int D, int NP>
-__device__ void epi_finish(EpiShared<NP>& es, const EpiCtx<D>& cx, EpiAcc& acc, const SplitParams& p, int b, int j0,
-                           int s) {
   const size_t row0 = (size_t)b * p.h_q + j0;
-  if (cx.RG > 1) {
+  if (et < p.G) {
+    float m4[4], M = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < kPT; ++i) {
-      if (!cx.valid[i]) continue;
-      const int jb = cx.u[i] * cx.hpv + cx.hb[i] * 4;
-      const int nk = min(4, cx.hpv - cx.hb[i] * 4);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (k < nk) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) atomicAdd(&es.red_o[(jb + k) * D + cx.c[i] * 4 + e], acc.o[i][k][e]);
-          if (cx.c[i] == 0) atomicAdd(&es.red_l[jb + k], acc.l[i][k]);
-        }
-      }
+    for (int w = 0; w < 4; ++w) {
+      m4[w] = mrg[w * REG + et];
+      M = fmaxf(M, m4[w]);
     }
-    named_bar_sync(1, kEpiThreads);
-    for (int idx = cx.et; idx < cx.G * (D / 4); idx += kEpiThreads) {
-      const int jl = idx / (D / 4), c4 = idx % (D / 4);
-      const float4 v = *reinterpret_cast<const float4*>(&es.red_o[jl * D + c4 * 4]);
-      *reinterpret_cast<float4*>(&p.part_o[((row0 + jl) * p.s_cap + s) * D + c4 * 4]) = v;
-    }
-    if (cx.et < cx.G) p.part_l[(row0 + cx.et) * p.s_cap + s] = es.red_l[cx.et];
-  } else {
+    float lsum = 0.f;
 #pragma unroll
-    for (int i = 0; i < kPT; ++i) {
-      if (!cx.valid[i]) continue;
-      const int jb = cx.u[i] * cx.hpv + cx.hb[i] * 4;
-      const int nk = min(4, cx.hpv - cx.hb[i] * 4);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (k < nk) {
-          const size_t r = (row0 + jb + k) * p.s_cap + s;
-          *reinterpret_cast<float4*>(&p.part_o[r * D + cx.c[i] * 4]) =
-              make_float4(acc.o[i][k][0], acc.o[i][k][1], acc.o[i][k][2], acc.o[i][k][3]);
-          if (cx.c[i] == 0) p.part_l[r] = acc.l[i][k];
-        }
-      }
+    for (int w = 0; w < 4; ++w) {
+      const float f = (m4[w] == -INFINITY) ? 0.f : __expf(m4[w] - M);
+      fac[w * NP + et] = f;
+      lsum += f * mrg[w * REG + NP + et];
     }
+    p.part_m[(row0 + et) * p.s_cap + s] = M;
+    p.part_l[(row0 + et) * p.s_cap + s] = lsum;
+    p.part_cnt[(row0 + et) * p.s_cap + s] = es.cnt_run[et];
   }
-  if (cx.et < cx.G) {
-    p.part_m[(row0 + cx.et) * p.s_cap + s] = es.m_run[cx.et];
-    p.part_cnt[(row0 + cx.et) * p.s_cap + s] = es.cnt_run[cx.et];
+  named_bar_sync(1, kEpiThreads);
+  for (int idx = et; idx < p.G * (D / 4); idx += kEpiThreads) {
+    const int jl = idx / (D / 4), c4 = idx % (D / 4);
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float f = fac[w * NP + jl];
+      const float4 v = *reinterpret_cast<const float4*>(&mrg[w * REG + 2 * NP + jl * D + c4 * 4]);
+      o.x = fmaf(f, v.x, o.x);
+      o.y = fmaf(f, v.y, o.y);
+      o.z = fmaf(f, v.z, o.z);
+      o.w = fmaf(f, v.w, o.w);
+    }
+    *reinterpret_cast<float4*>(&p.part_o[((row0 + jl) * p.s_cap + s) * D + c4 * 4]) = o;
   }
 }
 
@@ -363,17 +459,45 @@ template <int D, int NP, bool UMMA>
 struct SplitSmem {
   static constexpr int NATOM = D / 64;
   static constexpr int STAGE_BYTES = kTile * D * 2;
-  static constexpr int NSTAGE = split_stages<D>();
+  static constexpr int NSTAGE = split_stages<D, NP>();
   static constexpr int QBYTES = UMMA ? NATOM * NP * 128 : NP * D * 4;
   static constexpr int Q_OFF = NSTAGE * STAGE_BYTES;
   static constexpr int EPI_OFF = Q_OFF + ((QBYTES + 1023) / 1024) * 1024;
-  static constexpr int BAR_OFF = EPI_OFF + ((int)sizeof(EpiShared<NP>) + 15) / 16 * 16;
+  static constexpr int VST_OFF = EPI_OFF + ((int)sizeof(EpiShared<NP>) + 127) / 128 * 128;
+  static constexpr int BAR_OFF = VST_OFF + 4 * 2 * vstage_warp_bytes<NP>();
   static constexpr int NBARS = 2 * NSTAGE + 5;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
+  static_assert(merge_floats<D, NP>() * 4 <= NSTAGE * STAGE_BYTES, "merge buffer must fit in the key stages");
+  static_assert(NP * 256 * 4 <= (int)sizeof(WarpList<NP>) * 8, "dump histogram must fit in the warp lists");
 };
 
+// One key tile: 128 rows (or the rows left in the split, as 32-row boxes)
+// of every 64-column swizzle atom, into stage t % NSTAGE.
+template <int NATOM, int NSTAGE, int STAGE_BYTES>
+__device__ __forceinline__ void issue_key_tile(int t, int start, int end, int row_base, uint8_t* kst, uint64_t* full,
+                                               const CUtensorMap* tmap_full, const CUtensorMap* tmap_part) {
+  const int stage = t % NSTAGE;
+  const int r0 = start + t * kTile;
+  const int rows = min(kTile, end - r0);
+  uint8_t* dst = kst + stage * STAGE_BYTES;
+  if (rows == kTile) {
+    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+#pragma unroll
+    for (int a = 0; a < NATOM; ++a) tma_load_2d(dst + a * 16384, tmap_full, &full[stage], a * 64, row_base + r0);
+  } else {
+    const int nsub = (rows + kUnit - 1) / kUnit;
+    mbar_arrive_expect_tx(&full[stage], nsub * kUnit * 128 * NATOM);
+    for (int i = 0; i < nsub; ++i)
+#pragma unroll
+      for (int a = 0; a < NATOM; ++a)
+        tma_load_2d(dst + a * 16384 + i * kUnit * 128, tmap_part, &full[stage], a * 64, row_base + r0 + i * kUnit);
+  }
+}
+
+// Warp roles: 0 = TMA producer, 1 = tcgen05 MMA issuer (idle on the
+// CUDA-core path), 2..5 = epilogue (one thread per token row of a tile).
 template <int D, int NP, bool UMMA, bool DUMP>
 __global__ void __launch_bounds__(192, 1)
     saga_split_kernel(const __grid_constant__ CUtensorMap tmap_full, const __grid_constant__ CUtensorMap tmap_part,
@@ -390,7 +514,8 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* kst = smem;
   uint8_t* qsm = smem + SM::Q_OFF;
   EpiShared<NP>& es = *reinterpret_cast<EpiShared<NP>*>(smem + SM::EPI_OFF);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(&es.slot[0]);  // dump mode: [NP][256]
+  uint16_t* vstage = reinterpret_cast<uint16_t*>(smem + SM::VST_OFF);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(&es.list[0][0]);  // dump mode: [NP][256]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFF);
   uint64_t* empty = full + NSTAGE;
   uint64_t* accf = empty + NSTAGE;
@@ -409,6 +534,7 @@ __global__ void __launch_bounds__(192, 1)
   const int row_base = (b * p.h_k + h) * p.l_cap;  // first cache row of this (batch, key head)
 
   // ---------------------------------------------------------------- setup
+  int issued = 0;  // producer: tiles issued
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int i = 0; i < NSTAGE; ++i) {
@@ -421,10 +547,11 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(fin, 1);
     mbar_init_fence();
-  }
-  if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmap_full);
     tma_prefetch_desc(&tmap_part);
+    // the first stages go out before the rest of the setup
+    for (; issued < ntiles && issued < NSTAGE; ++issued)
+      issue_key_tile<NATOM, NSTAGE, STAGE_BYTES>(issued, start, end, row_base, kst, full, &tmap_full, &tmap_part);
   }
   if (UMMA && warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -459,29 +586,13 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = UMMA ? *tmem_slot : 0u;
 
-  int issued = 0;  // producer: tiles issued
   // ---------------------------------------------------------------- roles
   if (warp == 0) {
     if (lane == 0) {
-      for (int t = 0; t < ntiles; ++t) {
+      for (int t = issued; t < ntiles; ++t) {
         const int stage = t % NSTAGE, round = t / NSTAGE;
         if (round > 0 && !mbar_wait(&empty[stage], (round - 1) & 1, abort_flag)) break;
-        const int r0 = start + t * kTile;
-        const int rows = min(kTile, end - r0);
-        uint8_t* dst = kst + stage * STAGE_BYTES;
-        if (rows == kTile) {
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-#pragma unroll
-          for (int a = 0; a < NATOM; ++a) tma_load_2d(dst + a * 16384, &tmap_full, &full[stage], a * 64, row_base + r0);
-        } else {
-          const int nsub = (rows + kUnit - 1) / kUnit;
-          mbar_arrive_expect_tx(&full[stage], nsub * kUnit * 128 * NATOM);
-          for (int i = 0; i < nsub; ++i)
-#pragma unroll
-            for (int a = 0; a < NATOM; ++a)
-              tma_load_2d(dst + a * 16384 + i * kUnit * 128, &tmap_part, &full[stage], a * 64,
-                          row_base + r0 + i * kUnit);
-        }
+        issue_key_tile<NATOM, NSTAGE, STAGE_BYTES>(t, start, end, row_base, kst, full, &tmap_full, &tmap_part);
         issued = t + 1;
       }
     }
@@ -514,24 +625,26 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int et = threadIdx.x - 64;
-    EpiCtx<D> cx;
-    const int v_base = (int)(((long long)j0 * p.h_v) / p.h_q);
-    cx.init(et, p.G, p.nvh, p.hpv);
-    EpiAcc acc;
-    acc.zero();
-    const uint16_t* vgroup = p.v_cache + ((size_t)b * p.h_v + v_base) * (size_t)p.l_cap * D;
+    const int q = warp & 3;           // TMEM lane quarter: rows 32q .. 32q+31 of every tile
+    const int erow = 32 * q + lane;
+    const bool counting = p.want_counts != 0;
+    const EpiArgs ea = epi_args<D, NP>(p, b, j0);
+    uint16_t* vstage_w = vstage + (size_t)q * 2 * (vstage_warp_bytes<NP>() / 2);
+    WarpAcc<D, NP> acc;
+    acc.init();
+    ListState ls{0, 0, -1, 0};
     const size_t srow = ((size_t)b * p.h_q + j0) * (size_t)p.ld_scores;
-    bool ok = true;
     int t = 0;
     for (; t < ntiles; ++t) {
       float sc[NP];
+      bool ok;
       if (UMMA) {
         const int abuf = t & 1;
-        ok = mbar_wait(&accf[abuf], (t >> 1) & 1, abort_flag);
-        ok = named_bar_and(1, kEpiThreads, ok);
+        ok = __all_sync(0xffffffffu, mbar_wait(&accf[abuf], (t >> 1) & 1, abort_flag));
+        if (counting) ok = named_bar_and(1, kEpiThreads, ok);  // warps leave together (barriers below)
         if (!ok) break;
         tc_fence_after();
-        const uint32_t taddr = tmem_base + ((uint32_t)(32 * cx.q) << 16) + (uint32_t)(abuf * NP);
+        const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * NP);
 #pragma unroll
         for (int i = 0; i < NP / 16; ++i) tmem_ld16(taddr + 16 * i, sc + 16 * i);
         tc_fence_before();
@@ -539,10 +652,10 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) mbar_arrive(&acce[abuf]);
       } else {
         const int stage = t % NSTAGE;
-        ok = mbar_wait(&full[stage], (t / NSTAGE) & 1, abort_flag);
-        ok = named_bar_and(1, kEpiThreads, ok);
+        ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], (t / NSTAGE) & 1, abort_flag));
+        if (counting) ok = named_bar_and(1, kEpiThreads, ok);
         if (!ok) break;
-        const uint8_t* rowp = kst + stage * STAGE_BYTES + cx.erow * 128;
+        const uint8_t* rowp = kst + stage * STAGE_BYTES + erow * 128;
         const float* qf = reinterpret_cast<const float*>(qsm);
 #pragma unroll
         for (int n = 0; n < NP; ++n) sc[n] = 0.f;
@@ -550,7 +663,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int a = 0; a < NATOM; ++a) {
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(rowp + a * 16384 + ((c ^ (cx.erow & 7)) << 4));
+            const uint4 raw = *reinterpret_cast<const uint4*>(rowp + a * 16384 + ((c ^ (erow & 7)) << 4));
             const float kv[8] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y),
                                  bf16_lo(raw.z), bf16_hi(raw.z), bf16_lo(raw.w), bf16_hi(raw.w)};
 #pragma unroll
@@ -575,7 +688,7 @@ __global__ void __launch_bounds__(192, 1)
       }
 #pragma unroll
       for (int n = 0; n < NP; ++n) sc[n] *= p.scale;
-      const int tok = start + t * kTile + cx.erow;
+      const int tok = start + t * kTile + erow;
       const bool valid = tok < end;
       if (DUMP) {
 #pragma unroll
@@ -588,17 +701,14 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       } else {
-        phase_a<D, NP>(es, t & 1, sc, tok, valid, cx, p, b, j0, start, vgroup);
-        if (t > 0) phase_b<D, NP>(es, (t - 1) & 1, cx, vgroup, p.l_cap, acc);
+        tile_epilogue<D, NP>(es, acc, ea, ls, q, lane, et, sc, tok, valid, counting, p, b, j0, start, vstage_w);
       }
     }
     if (!DUMP) {
-      if (ok && ntiles > 0) {
-        named_bar_sync(1, kEpiThreads);
-        phase_b<D, NP>(es, (ntiles - 1) & 1, cx, vgroup, p.l_cap, acc);
-      }
-      named_bar_sync(1, kEpiThreads);
-      epi_finish<D, NP>(es, cx, acc, p, b, j0, s);
+      if (t == ntiles) flush_lists<D, NP>(es, acc, ea, ls, q, lane, vstage_w);
+      cp_async_wait_all();
+      named_bar_sync(1, kEpiThreads);  // every warp is done with the key stages (merge buffer below)
+      merge_and_store<D, NP>(es, reinterpret_cast<float*>(kst), acc, q, lane, et, p, b, j0, s);
     }
   }
 
@@ -629,53 +739,59 @@ __global__ void __launch_bounds__(192, 1)
 
 // ============================================================================ from-scores kernel
 // Refresh steps: the scores were dumped before the exact threshold was known;
-// compare and gather from them (same epilogue as the split kernel).
+// compare and gather from them with the same per-warp epilogue.
+template <int NP>
+__device__ __forceinline__ void load_scores(float (&dst)[NP], const float* srow, long long ld, int G, int tok, int end) {
+#pragma unroll
+  for (int jl = 0; jl < NP; ++jl) dst[jl] = (jl < G && tok < end) ? __ldg(srow + (size_t)jl * ld + tok) : -INFINITY;
+}
+
+template <int D, int NP>
+struct FromScoresSmem {
+  static constexpr int VST_OFF = ((int)sizeof(EpiShared<NP>) + 127) / 128 * 128;
+  static constexpr int MRG_OFF = VST_OFF + 4 * 2 * vstage_warp_bytes<NP>();
+  static constexpr int BYTES = MRG_OFF + merge_floats<D, NP>() * 4;
+};
+
 template <int D, int NP>
 __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const SplitParams p) {
-  extern __shared__ uint8_t smem_raw[];
+  using SM = FromScoresSmem<D, NP>;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
   EpiShared<NP>& es = *reinterpret_cast<EpiShared<NP>*>(smem_raw);
+  uint16_t* vstage = reinterpret_cast<uint16_t*>(smem_raw + SM::VST_OFF);
+  float* mrg = reinterpret_cast<float*>(smem_raw + SM::MRG_OFF);
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int et = threadIdx.x;
+  const int et = threadIdx.x, q = et >> 5, lane = et & 31;
   const int j0 = h * p.G;
   const int L = device_seq_len(p.seq_len_dev, p.seq_len, p.l_cap, nullptr);
   int start, end;
   split_range(L, p.nsplit, s, &start, &end);
   const int ntiles = (end - start + kTile - 1) / kTile;
+  const bool counting = p.want_counts != 0;
 
   epi_setup<NP>(es, et, p, b, j0, true);
-  EpiCtx<D> cx;
-  cx.init(et, p.G, p.nvh, p.hpv);
-  EpiAcc acc;
-  acc.zero();
-  const int v_base = (int)(((long long)j0 * p.h_v) / p.h_q);
-  const uint16_t* vgroup = p.v_cache + ((size_t)b * p.h_v + v_base) * (size_t)p.l_cap * D;
+  const EpiArgs ea = epi_args<D, NP>(p, b, j0);
+  uint16_t* vstage_w = vstage + (size_t)q * 2 * (vstage_warp_bytes<NP>() / 2);
+  WarpAcc<D, NP> acc;
+  acc.init();
+  ListState ls{0, 0, -1, 0};
   const float* srow = p.scores_in + ((size_t)b * p.h_q + j0) * (size_t)p.ld_scores;
   __syncthreads();
 
   float nxt[NP];
-  auto load = [&](int t, float (&dst)[NP]) {
-    const int tok = start + t * kTile + cx.erow;
-#pragma unroll
-    for (int jl = 0; jl < NP; ++jl)
-      dst[jl] = (jl < p.G && tok < end) ? __ldg(srow + (size_t)jl * p.ld_scores + tok) : -INFINITY;
-  };
-  if (ntiles > 0) load(0, nxt);
+  if (ntiles > 0) load_scores<NP>(nxt, srow, p.ld_scores, p.G, start + et, end);
   for (int t = 0; t < ntiles; ++t) {
     float sc[NP];
 #pragma unroll
     for (int jl = 0; jl < NP; ++jl) sc[jl] = nxt[jl];
-    if (t + 1 < ntiles) load(t + 1, nxt);
-    const int tok = start + t * kTile + cx.erow;
-    named_bar_sync(1, kEpiThreads);
-    phase_a<D, NP>(es, t & 1, sc, tok, tok < end, cx, p, b, j0, start, vgroup);
-    if (t > 0) phase_b<D, NP>(es, (t - 1) & 1, cx, vgroup, p.l_cap, acc);
+    if (t + 1 < ntiles) load_scores<NP>(nxt, srow, p.ld_scores, p.G, start + (t + 1) * kTile + et, end);
+    const int tok = start + t * kTile + et;
+    tile_epilogue<D, NP>(es, acc, ea, ls, q, lane, et, sc, tok, tok < end, counting, p, b, j0, start, vstage_w);
   }
-  if (ntiles > 0) {
-    named_bar_sync(1, kEpiThreads);
-    phase_b<D, NP>(es, (ntiles - 1) & 1, cx, vgroup, p.l_cap, acc);
-  }
+  flush_lists<D, NP>(es, acc, ea, ls, q, lane, vstage_w);
+  cp_async_wait_all();
   named_bar_sync(1, kEpiThreads);
-  epi_finish<D, NP>(es, cx, acc, p, b, j0, s);
+  merge_and_store<D, NP>(es, mrg, acc, q, lane, et, p, b, j0, s);
 }
 
 // ============================================================================ combine kernel
@@ -948,57 +1064,62 @@ __global__ void saga_fill_kernel(float* dst, float v, int n) {
 
 // ============================================================================ launchers
 template <int D, int NP, bool UMMA, bool DUMP>
-static cudaError_t prep_split() {
-  static bool done = false;
-  if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(saga_split_kernel<D, NP, UMMA, DUMP>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SplitSmem<D, NP, UMMA>::ALLOC);
-  if (e == cudaSuccess) done = true;
-  return e;
-}
-
-template <int D, int NP, bool UMMA, bool DUMP>
 static cudaError_t run_split(const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p, dim3 grid,
                              cudaStream_t st, int* occ) {
-  cudaError_t e = prep_split<D, NP, UMMA, DUMP>();
-  if (e != cudaSuccess) return e;
+  using K = SplitSmem<D, NP, UMMA>;
+  static bool prepared = false;
+  if (!prepared) {
+    cudaError_t e = cudaFuncSetAttribute(saga_split_kernel<D, NP, UMMA, DUMP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, K::ALLOC);
+    if (e != cudaSuccess) return e;
+    prepared = true;
+  }
   if (occ != nullptr)
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, saga_split_kernel<D, NP, UMMA, DUMP>, 192,
-                                                         SplitSmem<D, NP, UMMA>::ALLOC);
-  saga_split_kernel<D, NP, UMMA, DUMP><<<grid, 192, SplitSmem<D, NP, UMMA>::ALLOC, st>>>(tf, tp, p);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, saga_split_kernel<D, NP, UMMA, DUMP>, 192, K::ALLOC);
+  saga_split_kernel<D, NP, UMMA, DUMP><<<grid, 192, K::ALLOC, st>>>(tf, tp, p);
   return cudaGetLastError();
 }
 
-template <int D, bool DUMP>
-static cudaError_t dispatch_np(int NP, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p, dim3 g,
-                               cudaStream_t st, int* occ) {
+template <int D>
+static cudaError_t dispatch_np(int NP, bool dump, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p,
+                               dim3 g, cudaStream_t st, int* occ) {
+#define SAGA_NP(NN, UM)                                                                \
+  case NN:                                                                            \
+    return dump ? run_split<D, NN, UM, true>(tf, tp, p, g, st, occ)                   \
+                : run_split<D, NN, UM, false>(tf, tp, p, g, st, occ);
   switch (NP) {
-    case 4: return run_split<D, 4, false, DUMP>(tf, tp, p, g, st, occ);
-    case 16: return run_split<D, 16, true, DUMP>(tf, tp, p, g, st, occ);
-    case 32: return run_split<D, 32, true, DUMP>(tf, tp, p, g, st, occ);
-    case 64: return run_split<D, 64, true, DUMP>(tf, tp, p, g, st, occ);
-    default: return cudaErrorInvalidValue;
+    SAGA_NP(4, false)
+    SAGA_NP(16, true)
+    SAGA_NP(32, true)
+    case 64:
+      if constexpr (D == 64) {
+        return dump ? run_split<D, 64, true, true>(tf, tp, p, g, st, occ)
+                    : run_split<D, 64, true, false>(tf, tp, p, g, st, occ);
+      } else {
+        return cudaErrorInvalidValue;  // d = 128 supports at most 32 query heads per key head
+      }
+    default:
+      return cudaErrorInvalidValue;
   }
+#undef SAGA_NP
 }
 
 cudaError_t launch_split(int D, int NP, bool dump, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p,
                          dim3 grid, cudaStream_t st, int* occupancy_out) {
-  if (D == 64) return dump ? dispatch_np<64, true>(NP, tf, tp, p, grid, st, occupancy_out)
-                           : dispatch_np<64, false>(NP, tf, tp, p, grid, st, occupancy_out);
-  if (D == 128) return dump ? dispatch_np<128, true>(NP, tf, tp, p, grid, st, occupancy_out)
-                            : dispatch_np<128, false>(NP, tf, tp, p, grid, st, occupancy_out);
+  if (D == 64) return dispatch_np<64>(NP, dump, tf, tp, p, grid, st, occupancy_out);
+  if (D == 128) return dispatch_np<128>(NP, dump, tf, tp, p, grid, st, occupancy_out);
   return cudaErrorInvalidValue;
 }
 
 template <int D, int NP>
 static cudaError_t run_from_scores(const SplitParams& p, dim3 grid, cudaStream_t st) {
-  static bool done = false;
-  const int bytes = (int)sizeof(EpiShared<NP>);
-  if (!done) {
-    cudaError_t e = cudaFuncSetAttribute(saga_from_scores_kernel<D, NP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         bytes);
+  static bool prepared = false;
+  const int bytes = FromScoresSmem<D, NP>::BYTES;
+  if (!prepared) {
+    cudaError_t e =
+        cudaFuncSetAttribute(saga_from_scores_kernel<D, NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    done = true;
+    prepared = true;
   }
   saga_from_scores_kernel<D, NP><<<grid, kEpiThreads, bytes, st>>>(p);
   return cudaGetLastError();
@@ -1008,7 +1129,7 @@ cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, c
 #define SAGA_FS(DD, NN) \
   if (D == DD && NP == NN) return run_from_scores<DD, NN>(p, grid, st);
   SAGA_FS(64, 4) SAGA_FS(64, 16) SAGA_FS(64, 32) SAGA_FS(64, 64)
-  SAGA_FS(128, 4) SAGA_FS(128, 16) SAGA_FS(128, 32) SAGA_FS(128, 64)
+  SAGA_FS(128, 4) SAGA_FS(128, 16) SAGA_FS(128, 32)
 #undef SAGA_FS
   return cudaErrorInvalidValue;
 }
@@ -1041,16 +1162,6 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t st) {
 cudaError_t launch_fill(float* dst, float v, int n, cudaStream_t st) {
   saga_fill_kernel<<<(n + 255) / 256, 256, 0, st>>>(dst, v, n);
   return cudaGetLastError();
-}
-
-int epi_shared_bytes(int NP) {
-  switch (NP) {
-    case 4: return (int)sizeof(EpiShared<4>);
-    case 16: return (int)sizeof(EpiShared<16>);
-    case 32: return (int)sizeof(EpiShared<32>);
-    case 64: return (int)sizeof(EpiShared<64>);
-  }
-  return 0;
 }
 
 }  // namespace saga

@@ -41,7 +41,7 @@ CASES = [
     small("g1_mha_d128", h_q=4, h_k=4, h_v=4, d=128, l_kv=300, n_top=9, batch=3),
     small("g16_d128_r1", h_q=16, h_k=1, h_v=2, d=128, l_kv=1290, n_top=100, refresh=1, steps=5),
     small("g8_n1", h_q=8, h_k=1, h_v=8, d=64, l_kv=500, n_top=1, refresh=3),
-    small("tiny_l", h_q=8, h_k=2, h_v=4, d=64, l_kv=5, n_top=3, refresh=2, steps=6),
+    small("tiny_l", h_q=8, h_k=2, h_v=4, d=64, l_kv=5, n_top=3, refresh=2, steps=6, q_mode="gaussian", planted=0.0),
     small("n_gt_l", h_q=8, h_k=1, h_v=8, d=64, l_kv=40, n_top=60, refresh=2, steps=30),
     small("dense_g4", h_q=16, h_k=4, h_v=4, d=64, l_kv=1500, n_top=workload.DENSE, refresh=1 << 30,
           q_mode="gaussian", planted=0.0, steps=4),
