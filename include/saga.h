@@ -143,6 +143,31 @@ SAGA_API int saga_decode_attn(const saga_shape* s, const void* q, const void* k_
  * NULLs cancels a pending request. */
 SAGA_API int saga_trace_next_attention(void* ev_start, void* ev_end);
 
+/* Allocation-free variant of saga_decode_attn (the paper has no counterpart:
+ * this is an integration aid).  Same arguments and results, without the
+ * workspace: the scratch is a fixed array of SAGA_NOALLOC_SCRATCH_BYTES in
+ * the library's device image, which every device that loads the library
+ * holds until the process exits.  For callers that cannot allocate device
+ * memory around the call (their memory is owned by another allocator, or an
+ * allocation is not allowed at that point).
+ *   - Shapes whose saga_workspace_bytes exceeds the scratch are rejected with
+ *     SAGA_ERR_WORKSPACE and a message; use saga_decode_attn for those.
+ *   - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
+ *   - The first call on a device looks up the scratch's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call on a device shares the one scratch array, which keeps the
+ *     previous call's contents; each call clears the status word it uses.
+ *     Calls whose work overlaps on the GPU (other streams, other host
+ *     threads) race on the scratch: serialize them.
+ * saga_noalloc_last_error() describes the last failure of this entry point. */
+#define SAGA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+SAGA_API size_t saga_noalloc_scratch_bytes(void);
+SAGA_API int saga_decode_attn_noalloc(const saga_shape* s, const void* q, const void* k_cache, const void* v_cache,
+                                      int seq_len, const int* seq_len_dev, int n_top, int refresh_interval,
+                                      long long step, float* tau, void* out, int out_dtype, int* sel_count,
+                                      int* sel_idx, void* stream);
+SAGA_API const char* saga_noalloc_last_error(void);
+
 /* Reads the workspace status word (SAGA_STATUS_* bits ORed by the kernels
  * since the workspace was zeroed) after synchronizing `stream`. */
 SAGA_API int saga_get_status(const void* workspace, void* stream, unsigned* status);

@@ -28,7 +28,8 @@ SAGA_STATUS_LEN_CLAMPED = 0x1
 SAGA_STATUS_TIMEOUT = 0x2
 
 EXPORTED = ("saga_workspace_bytes", "saga_kv_append", "atopn_refresh_threshold", "atopn_select_workspace_bytes",
-            "atopn_select_threshold", "saga_decode_attn", "saga_trace_next_attention", "saga_get_status", "saga_last_error", "saga_abi_version")
+            "atopn_select_threshold", "saga_decode_attn", "saga_trace_next_attention", "saga_get_status", "saga_last_error", "saga_abi_version",
+            "saga_noalloc_scratch_bytes", "saga_decode_attn_noalloc", "saga_noalloc_last_error")
 
 
 class SagaError(RuntimeError):
@@ -85,6 +86,13 @@ def load(path: Optional[str] = None):
     lib.saga_last_error.restype = ctypes.c_char_p
     lib.saga_abi_version.argtypes = []
     lib.saga_abi_version.restype = _I
+    lib.saga_noalloc_scratch_bytes.argtypes = []
+    lib.saga_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.saga_decode_attn_noalloc.argtypes = [sp, _P, _P, _P, _I, _P, _I, _I, ctypes.c_longlong, _P, _P, _I, _P, _P,
+                                             _P]
+    lib.saga_decode_attn_noalloc.restype = _I
+    lib.saga_noalloc_last_error.argtypes = []
+    lib.saga_noalloc_last_error.restype = ctypes.c_char_p
     _lib = lib
     return lib
 
@@ -207,6 +215,35 @@ def saga_trace_next_attention(ev_start: Optional[torch.cuda.Event], ev_end: Opti
         if ev.cuda_event == 0:  # torch creates the event on first record
             ev.record()
     _check(load().saga_trace_next_attention(ctypes.c_void_p(ev_start.cuda_event), ctypes.c_void_p(ev_end.cuda_event)))
+
+
+def saga_decode_attn_noalloc(shape: SagaShape, q, k_cache, v_cache, seq_len: int, n_top: int, refresh_interval: int,
+                             step: int, tau, out, sel_count=None, sel_idx=None, seq_len_dev=None, stream=None):
+    """saga_decode_attn with the library's built-in scratch instead of a caller workspace (allocates nothing)."""
+    B, hq, hk, hv, d, lc = shape.astuple()
+    _expect(q, "q", torch.bfloat16, (B, hq, d))
+    _expect(k_cache, "k_cache", torch.bfloat16, (B, hk, lc, d))
+    _expect(v_cache, "v_cache", torch.bfloat16, (B, hv, lc, d))
+    _expect(tau, "tau", torch.float32, (B, hq))
+    if out.dtype == torch.float32:
+        out_dtype = SAGA_OUT_F32
+    elif out.dtype == torch.bfloat16:
+        out_dtype = SAGA_OUT_BF16
+    else:
+        raise TypeError("out must be float32 or bfloat16")
+    _expect(out, "out", out.dtype, (B, hq, d))
+    if sel_count is not None:
+        _expect(sel_count, "sel_count", torch.int32, (B, hq))
+    if sel_idx is not None:
+        _expect(sel_idx, "sel_idx", torch.int32, (B, hq, lc))
+    if seq_len_dev is not None:
+        _expect(seq_len_dev, "seq_len_dev", torch.int32)
+    lib = load()
+    rc = lib.saga_decode_attn_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), int(seq_len),
+                                      _ptr(seq_len_dev), int(n_top), int(refresh_interval), int(step), _ptr(tau),
+                                      _ptr(out), out_dtype, _ptr(sel_count), _ptr(sel_idx), _stream(stream))
+    if rc != SAGA_OK:
+        raise SagaError(rc, lib.saga_noalloc_last_error().decode(errors="replace"))
 
 
 def saga_get_status(workspace, stream=None) -> int:
