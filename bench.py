@@ -1,8 +1,9 @@
 """Benchmark of the SAGA + Atop-N decode-attention step on B200.
 
 One step = one decode step of every layer of the workload: for each layer,
-append the new token's key/value rows, then the attention step (Atop-N
-threshold refresh on t % R == 0, else reuse).  The step runs as a CUDA graph
+one saga_decode_step call (the new token's key/value rows are appended by
+the attention kernels, then the attention step: Atop-N threshold refresh on
+t % R == 0, else reuse).  The step runs as a CUDA graph
 replay; caches live in HBM.  Default workload: the Qwen2.5-1.5B-shaped SAGA
 configuration at 128K context (h_q=12, d=128, h_k=1, h_v=4, N=512, R=32,
 28 layers, batch 1 per GPU).
@@ -175,6 +176,26 @@ def cpu_baseline(wl, seconds_budget=20.0):
             "us_per_layer_step": dt / done * 1e6, "us_per_step_scaled": dt / done * 1e6 * wl.layers}
 
 
+def gather_rank_stats(local, world):
+    """Every rank's timing record, in rank order (one all_gather over the process group: NCCL or gloo)."""
+    if world == 1:
+        return [local]
+    import torch.distributed as dist
+    out = [None] * world
+    dist.all_gather_object(out, local)
+    return out
+
+
+def combine_rank_stats(per_rank, steps):
+    """Whole-job figures under weak scaling: the bytes of all ranks over the slowest rank's time."""
+    ms_max = max(r["ms"] for r in per_rank)
+    total = sum(r["bytes"] for r in per_rank)
+    e_ms = max(r["e2e_ms"] for r in per_rank)
+    e_total = sum(r["e2e_bytes"] for r in per_rank)
+    return {"value": total / (ms_max / 1e3) / 1e9, "ms_max": ms_max, "ms_per_step": ms_max / steps,
+            "e2e_value": e_total / (e_ms / 1e3) / 1e9 if e_ms > 0 else None}
+
+
 def run_reference(args, wl, rank, world):
     if rank != 0:
         return 0
@@ -314,8 +335,9 @@ def run_saga(args, wl, rank, world, local_rank):
         e2e = {"value": e_bytes / (e_ms / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / E}
 
-    # dominant kernel: the split-context attention kernel of reuse steps, bracketed by CUDA events on
-    # its stream inside freshly recorded graphs (one event pair per layer)
+    # dominant kernel: the split-context attention kernel of reuse steps (with the fused append),
+    # bracketed by CUDA events on its stream inside a freshly recorded graph (one event pair per layer;
+    # the events serialise the kernels, so this is the kernel's own duration without launch overlap)
     kernel_ms = []
     if wl.refresh > 1 and T > 0:
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(wl.layers)]
@@ -325,12 +347,10 @@ def run_saga(args, wl, rank, world, local_rank):
         with torch.cuda.graph(g, stream=stream):
             sess.seq_len_dev.add_(1)
             for i in range(wl.layers):
-                saga.saga_kv_append(shape, sess.k_cache[i], sess.v_cache[i], sess.k_buf[i], sess.v_buf[i],
-                                    L_est - 1, seq_len_dev=sess.seq_len_dev)
                 saga.saga_trace_next_attention(*evs[i])
-                saga.saga_decode_attn(shape, sess.q_buf[i], sess.k_cache[i], sess.v_cache[i], L_est, n_top,
-                                      wl.refresh, 1, sess.tau[i], sess.out[i], sess.workspace,
-                                      seq_len_dev=sess.seq_len_dev)
+                saga.saga_decode_step(shape, sess.q_buf[i], sess.k_buf[i], sess.v_buf[i], sess.k_cache[i],
+                                      sess.v_cache[i], L_est, n_top, wl.refresh, 1, sess.tau[i], sess.out[i],
+                                      sess.workspace, seq_len_dev=sess.seq_len_dev)
         sess.seq_len_dev.fill_(sess.length)
         for _ in range(T):
             if sess.t % wl.refresh == 0:  # keep the refresh schedule: run refresh steps with the step graphs
@@ -348,20 +368,14 @@ def run_saga(args, wl, rank, world, local_rank):
         del g
     status = saga.saga_get_status(sess.workspace)
 
-    # ---- gather over ranks
-    stats = torch.tensor([ms, bytes_timed, e2e["value"] if e2e else 0.0], dtype=torch.float64, device=dev)
-    if world > 1:
-        gathered = [torch.zeros_like(stats) for _ in range(world)]
-        dist.all_gather(gathered, stats)
-        ms_max = max(float(x[0]) for x in gathered)
-        total_bytes = sum(float(x[1]) for x in gathered)
-        e2e_sum = sum(float(x[2]) for x in gathered)
-    else:
-        ms_max, total_bytes, e2e_sum = ms, bytes_timed, (e2e["value"] if e2e else 0.0)
+    # ---- gather over ranks (every rank takes part, whatever it measured)
+    local = {"ms": ms, "bytes": bytes_timed, "e2e_ms": e2e["ms_per_step"] * E if e2e else 0.0,
+             "e2e_bytes": e_bytes if e2e else 0.0}
+    job = combine_rank_stats(gather_rank_stats(local, world), K)
     if rank != 0:
         return 0
-    value = total_bytes / (ms_max / 1e3) / 1e9
-    ms_per_step = ms_max / K
+    value = job["value"]
+    ms_per_step = job["ms_per_step"]
     peak, peak_kind = load_peak()
     roofline = None
     if kernel_ms:
@@ -381,7 +395,7 @@ def run_saga(args, wl, rank, world, local_rank):
                    "l2": "inputs exceed L2 (all layers' caches cycle through L2 each step)",
                    "refresh_steps_timed": refresh_steps},
         "roofline": roofline,
-        "e2e": ({"value": e2e_sum if world > 1 else e2e["value"], "unit": "GB/s",
+        "e2e": ({"value": job["e2e_value"], "unit": "GB/s",
                  "h2d_bytes_per_step": e2e["h2d_bytes_per_step"] * world,
                  "d2h_bytes_per_step": e2e["d2h_bytes_per_step"] * world} if e2e else None),
         "gpu_launches": launches,

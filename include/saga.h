@@ -38,8 +38,20 @@
  *     `seq_len_dev` is not NULL the kernels read the length from that device
  *     int instead, when they run (use this inside CUDA graphs, where the
  *     length changes between replays); `seq_len` must then still be a valid
- *     host-side estimate, used only to size the launch.  A device length
- *     outside [1, l_cap] is clamped and flagged in the workspace status word.
+ *     host-side estimate: it sizes the launch and places the context-split
+ *     boundaries, and the last split also covers any tokens beyond it (so a
+ *     graph captured at length P stays correct for every later length; pass
+ *     the capture-time length).  A device length outside [1, l_cap] is
+ *     clamped and flagged in the workspace status word.
+ *   - The kernels are launched with programmatic dependent launch
+ *     (cudaLaunchAttributeProgrammaticStreamSerialization): each may start
+ *     while the previous kernel on the stream finishes, but reads and writes
+ *     nothing that kernel can touch before it has completed (its early work
+ *     is barrier and TMEM setup and an L2 prefetch of key rows).  Set
+ *     SAGA_PDL=0 in the environment for plain stream order.
+ *   - Reads of the caches: key rows are loaded in 32-row units, so rows up
+ *     to the next multiple of 32 past seq_len - 1 (always below l_cap) may be
+ *     read and are ignored.
  *   - Inputs must be finite (no NaN/Inf in q or the caches).
  *   - Return value: SAGA_OK or a negative SAGA_ERR_* code.  Arguments are
  *     validated before anything is enqueued; on an error nothing is
@@ -127,12 +139,25 @@ SAGA_API int atopn_select_threshold(const float* scores, int rows, int row_len, 
  *   sel_count (nullable): int32 [B, h_q], number of kept positions.
  *   sel_idx (nullable, needs sel_count): int32 [B, h_q, l_cap]; the first
  *         sel_count[b, j] entries are the kept positions in ascending order.
- * The kernels read the caches at positions < seq_len only. */
+ * The new token's rows must already be in the caches at seq_len - 1
+ * (saga_kv_append), or use saga_decode_step. */
 SAGA_API int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, const void* v_cache, int seq_len,
                      const int* seq_len_dev, int n_top, int refresh_interval, long long step, float* tau, void* out,
                      int out_dtype, int* sel_count, int* sel_idx, void* workspace, size_t ws_bytes, void* stream);
 
-/* Tracing: the next saga_decode_attn call made on this host thread records
+/* Append and attend in one call: saga_kv_append(k_new, v_new, pos =
+ * seq_len - 1) followed by saga_decode_attn, with the append done inside
+ * the attention kernels (the context split that holds row seq_len - 1
+ * writes the key and value rows before it loads them), so a decode step of
+ * a layer costs no separate launch for it.  Same arguments and results as
+ * saga_decode_attn plus k_new bf16 [B, h_k, d] and v_new bf16 [B, h_v, d];
+ * the caches are written. */
+SAGA_API int saga_decode_step(const saga_shape* s, const void* q, const void* k_new, const void* v_new, void* k_cache,
+                     void* v_cache, int seq_len, const int* seq_len_dev, int n_top, int refresh_interval,
+                     long long step, float* tau, void* out, int out_dtype, int* sel_count, int* sel_idx,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/* Tracing: the next saga_decode_attn (or saga_decode_step) call made on this host thread records
  * ev_start on its stream just before its context-split attention kernels
  * (after nothing else of that call) and ev_end just after them, before the
  * cross-split combine.  On a reuse step that is the one fused split kernel;

@@ -14,7 +14,7 @@
 #include "saga_internal.h"
 
 namespace saga {
-cudaError_t launch_split(int D, int NP, bool dump, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p,
+cudaError_t launch_split(int D, int NP, int mode, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p,
                          dim3 grid, cudaStream_t st, int* occupancy_out);
 cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, cudaStream_t st);
 cudaError_t launch_combine(int D, const CombineParams& p, cudaStream_t st);
@@ -204,10 +204,19 @@ int prepare_ws(const saga_shape* s, void* workspace, size_t ws_bytes, Prepared* 
   return SAGA_OK;
 }
 
-void fill_split_common(SplitParams& p, const saga_shape* s, const Prepared& pr, const void* q, int seq_len,
-                       const int* seq_len_dev) {
+// New token's rows for the fused append (all null: no append).
+struct NewRows {
+  uint16_t* k_cache = nullptr;
+  uint16_t* v_cache = nullptr;
+  const uint16_t* k_new = nullptr;
+  const uint16_t* v_new = nullptr;
+};
+
+void fill_split_common(SplitParams& p, const saga_shape* s, const Prepared& pr, const void* q, const void* k_cache,
+                       int seq_len, const int* seq_len_dev) {
   memset(&p, 0, sizeof(p));
   p.q = static_cast<const uint16_t*>(q);
+  p.k_cache = static_cast<const uint16_t*>(k_cache);
   p.status = reinterpret_cast<unsigned*>(pr.base + pr.ws.status);
   p.seq_len_dev = seq_len_dev;
   p.seq_len = seq_len;
@@ -228,11 +237,11 @@ void fill_split_common(SplitParams& p, const saga_shape* s, const Prepared& pr, 
   p.part_cnt = reinterpret_cast<int*>(pr.base + pr.ws.part_cnt);
 }
 
-int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, bool dump, const CUtensorMap& tf,
+int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, int mode, const CUtensorMap& tf,
                const CUtensorMap& tp, int* S) {
   int occ = 0;
   SplitParams dummy{};
-  cudaError_t e = launch_split(s->d, NP, dump, tf, tp, dummy, dim3(1), nullptr, &occ);
+  cudaError_t e = launch_split(s->d, NP, mode, tf, tp, dummy, dim3(1), nullptr, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
   if (occ < 1) return fail(SAGA_ERR_UNSUPPORTED, "split kernel does not fit on an SM");
   *S = choose_splits(s->batch * s->h_k, seq_len, occ * pr.sms, pr.ws.s_cap);
@@ -242,7 +251,8 @@ int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, boo
 // Scores of every cached token, their top-byte histograms, and the exact
 // threshold (refresh).
 int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const void* k_cache, int seq_len,
-                const int* seq_len_dev, int n_top, float* tau, cudaStream_t st, cudaEvent_t ev_start = nullptr) {
+                const int* seq_len_dev, int n_top, float* tau, cudaStream_t st, cudaEvent_t ev_start = nullptr,
+                const NewRows& nr = NewRows()) {
   const int G = s->h_q / s->h_k, NP = np_for_group(G);
   CUtensorMap tf, tp;
   int rc = make_key_map(&tf, k_cache, s, kTile);
@@ -250,7 +260,7 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   rc = make_key_map(&tp, k_cache, s, kUnit);
   if (rc) return rc;
   int S = 1;
-  rc = splits_for(s, pr, seq_len, NP, true, tf, tp, &S);
+  rc = splits_for(s, pr, seq_len, NP, kSplitDump, tf, tp, &S);
   if (rc) return rc;
   const size_t rows = (size_t)s->batch * s->h_q;
   uint32_t* hist = reinterpret_cast<uint32_t*>(pr.base + pr.ws.hist);
@@ -261,11 +271,15 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   cudaError_t e = cudaMemsetAsync(hist, 0, rows * 256 * 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(hist)");
   SplitParams p;
-  fill_split_common(p, s, pr, q, seq_len, seq_len_dev);
+  fill_split_common(p, s, pr, q, k_cache, seq_len, seq_len_dev);
+  p.k_cache_w = nr.k_cache;
+  p.v_cache_w = nr.v_cache;
+  p.k_new = nr.k_new;
+  p.v_new = nr.v_new;
   p.scores_out = reinterpret_cast<float*>(pr.base + pr.ws.scores);
   p.hist_out = hist;
   p.nsplit = S;
-  e = launch_split(s->d, NP, true, tf, tp, p, dim3(S, s->h_k, s->batch), st, nullptr);
+  e = launch_split(s->d, NP, kSplitDump, tf, tp, p, dim3(S, s->h_k, s->batch), st, nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "score dump launch");
   SelectParams sp{};
   sp.scores = p.scores_out;
@@ -369,9 +383,16 @@ int atopn_select_threshold(const float* scores, int rows, int row_len, long long
   return ok();
 }
 
-int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, const void* v_cache, int seq_len,
-                     const int* seq_len_dev, int n_top, int refresh_interval, long long step, float* tau, void* out,
-                     int out_dtype, int* sel_count, int* sel_idx, void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// One attention step; with nr set, the new token's rows are appended at
+// seq_len - 1 by the attention kernels themselves.
+int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const void* v_cache, int seq_len,
+                const int* seq_len_dev, int n_top, int refresh_interval, long long step, float* tau, void* out,
+                int out_dtype, int* sel_count, int* sel_idx, void* workspace, size_t ws_bytes, void* stream,
+                const NewRows& nr) {
   int rc = validate_shape(s);
   if (rc) return rc;
   if (!q || !k_cache || !v_cache || !tau || !out) return fail(SAGA_ERR_ARG, "NULL tensor pointer");
@@ -402,7 +423,7 @@ int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, co
   g_trace_start = g_trace_end = nullptr;
 
   SplitParams p;
-  fill_split_common(p, s, pr, q, seq_len, seq_len_dev);
+  fill_split_common(p, s, pr, q, k_cache, seq_len, seq_len_dev);
   p.v_cache = static_cast<const uint16_t*>(v_cache);
   p.tau = tau;
   p.want_counts = sel_count != nullptr;
@@ -410,16 +431,17 @@ int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, co
   cudaError_t e;
   int S = 1;
   if (refresh && !no_threshold) {
-    rc = run_refresh(s, pr, q, k_cache, seq_len, seq_len_dev, n_top, tau, st, ev0);
+    rc = run_refresh(s, pr, q, k_cache, seq_len, seq_len_dev, n_top, tau, st, ev0, nr);
     if (rc) return rc;
-    rc = splits_for(s, pr, seq_len, NP, true, tf, tp, &S);
+    rc = splits_for(s, pr, seq_len, NP, kSplitDump, tf, tp, &S);
     if (rc) return rc;
     p.scores_in = reinterpret_cast<const float*>(pr.base + pr.ws.scores);
     p.nsplit = S;
     e = launch_from_scores(s->d, NP, p, dim3(S, s->h_k, s->batch), st);
     if (e != cudaSuccess) return cuda_fail(e, "from-scores launch");
   } else {
-    rc = splits_for(s, pr, seq_len, NP, false, tf, tp, &S);
+    const int mode = no_threshold ? kSplitDense : kSplitSparse;
+    rc = splits_for(s, pr, seq_len, NP, mode, tf, tp, &S);
     if (rc) return rc;
     p.nsplit = S;
     if (ev0 != nullptr) {
@@ -430,7 +452,12 @@ int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, co
       e = launch_fill(tau, -INFINITY, rows, st);
       if (e != cudaSuccess) return cuda_fail(e, "threshold fill launch");
     }
-    e = launch_split(s->d, NP, false, tf, tp, p, dim3(S, s->h_k, s->batch), st, nullptr);
+    if (no_threshold) p.tau = nullptr;  // every token kept; the threshold is not read
+    p.k_cache_w = nr.k_cache;
+    p.v_cache_w = nr.v_cache;
+    p.k_new = nr.k_new;
+    p.v_new = nr.v_new;
+    e = launch_split(s->d, NP, mode, tf, tp, p, dim3(S, s->h_k, s->batch), st, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "split launch");
   }
   if (ev1 != nullptr) {
@@ -457,6 +484,32 @@ int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, co
   e = launch_combine(s->d, c, st);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int saga_decode_attn(const saga_shape* s, const void* q, const void* k_cache, const void* v_cache, int seq_len,
+                     const int* seq_len_dev, int n_top, int refresh_interval, long long step, float* tau, void* out,
+                     int out_dtype, int* sel_count, int* sel_idx, void* workspace, size_t ws_bytes, void* stream) {
+  return decode_impl(s, q, k_cache, v_cache, seq_len, seq_len_dev, n_top, refresh_interval, step, tau, out, out_dtype,
+                     sel_count, sel_idx, workspace, ws_bytes, stream, NewRows());
+}
+
+int saga_decode_step(const saga_shape* s, const void* q, const void* k_new, const void* v_new, void* k_cache,
+                     void* v_cache, int seq_len, const int* seq_len_dev, int n_top, int refresh_interval,
+                     long long step, float* tau, void* out, int out_dtype, int* sel_count, int* sel_idx,
+                     void* workspace, size_t ws_bytes, void* stream) {
+  if (k_new == nullptr || v_new == nullptr) return fail(SAGA_ERR_ARG, "NULL k_new / v_new");
+  if (!aligned16(k_new) || !aligned16(v_new)) return fail(SAGA_ERR_ARG, "k_new and v_new must be 16-byte aligned");
+  NewRows nr;
+  nr.k_cache = static_cast<uint16_t*>(k_cache);
+  nr.v_cache = static_cast<uint16_t*>(v_cache);
+  nr.k_new = static_cast<const uint16_t*>(k_new);
+  nr.v_new = static_cast<const uint16_t*>(v_new);
+  return decode_impl(s, q, k_cache, v_cache, seq_len, seq_len_dev, n_top, refresh_interval, step, tau, out, out_dtype,
+                     sel_count, sel_idx, workspace, ws_bytes, stream, nr);
 }
 
 int saga_trace_next_attention(void* ev_start, void* ev_end) {

@@ -96,6 +96,21 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* gptr, uint32_t byte
                : "memory");
 }
 
+// Generic-proxy global writes made visible to later TMA (async-proxy) reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// pdl_wait: returns once the grids this one depends on have completed and
+// their writes are visible (immediately when launched without the
+// programmatic-serialization attribute).  Nothing a preceding kernel writes
+// may be read, and nothing a preceding kernel reads may be written, before it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// pdl_trigger: lets the next kernel on the stream start launching its CTAs
+// (they run up to their own pdl_wait).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- cp.async (16-byte, L2 only)
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),

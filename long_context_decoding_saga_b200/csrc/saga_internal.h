@@ -9,6 +9,9 @@
 
 namespace saga {
 
+// Split-kernel modes: attend with every token kept (N covers every length),
+// attend with the Atop-N threshold, or dump scores for a refresh.
+constexpr int kSplitDense = 0, kSplitSparse = 1, kSplitDump = 2;
 constexpr int kTile = 128;       // tokens per pipeline tile (UMMA M)
 constexpr int kUnit = 32;        // split boundaries fall on multiples of 32 tokens
 constexpr int kEpiThreads = 128; // epilogue warps: one thread per token of a tile
@@ -18,15 +21,30 @@ constexpr int kMaxCtasPerSm = 4; // bound used to size the split partials
 constexpr int kSelectThreads = 1024;
 constexpr int kSelectCap = 16384; // radix-select candidates kept in shared memory
 
-// Token range [start, end) of split s out of S over a row of L tokens.
-__host__ __device__ inline void split_range(int L, int S, int s, int* start, int* end) {
-  const long long U = (L + kUnit - 1) / kUnit;
+// Token range [start, end) of split s out of S.  The boundaries partition P
+// tokens (the host's length at launch, fixed for a captured graph) at
+// multiples of kUnit; the range is then clamped to the device length L, and
+// the last split also takes any tokens in [P, L).
+__host__ __device__ inline void split_range(int P, int S, int s, int L, int* start, int* end) {
+  const long long U = (P + kUnit - 1) / kUnit;
   const long long a = (s * U) / S, b = ((s + 1) * U) / S;
-  long long st = a * kUnit, en = b * kUnit;
+  long long st = a * kUnit, en = (s == S - 1) ? (long long)L : b * kUnit;
   if (en > L) en = L;
   if (st > L) st = L;
   *start = (int)st;
   *end = (int)en;
+}
+
+// Rows split s may cover whatever the device length is: [start, cap_end),
+// within the cache capacity (used for prefetching before the length is read).
+__host__ __device__ inline void split_cap_range(int P, int S, int s, int l_cap, int* start, int* cap_end) {
+  const long long U = (P + kUnit - 1) / kUnit;
+  const long long a = (s * U) / S, b = ((s + 1) * U) / S;
+  long long st = a * kUnit, en = (s == S - 1) ? (long long)l_cap : b * kUnit;
+  if (en > l_cap) en = l_cap;
+  if (st > l_cap) st = l_cap;
+  *start = (int)st;
+  *cap_end = (int)en;
 }
 
 // Byte offsets of the workspace regions (each 256-byte aligned).
@@ -46,7 +64,12 @@ struct WsLayout {
 
 struct SplitParams {
   const uint16_t* q;        // bf16 [B, h_q, d]
+  const uint16_t* k_cache;  // bf16 [B, h_k, l_cap, d] (also behind the tensor maps)
   const uint16_t* v_cache;  // bf16 [B, h_v, l_cap, d]
+  uint16_t* k_cache_w;      // fused append: caches written at row L - 1
+  uint16_t* v_cache_w;
+  const uint16_t* k_new;    // fused append (nullable): bf16 [B, h_k, d]
+  const uint16_t* v_new;    //                          bf16 [B, h_v, d]
   const float* tau;         // [B, h_q]
   const float* scores_in;   // from-scores mode: [B*h_q, ld_scores]
   float* scores_out;        // dump mode
@@ -59,7 +82,7 @@ struct SplitParams {
   unsigned* status;
   const int* seq_len_dev;   // nullable
   long long ld_scores;
-  int seq_len;
+  int seq_len;   // host length: the length when seq_len_dev is null, and the partition length P
   int batch, h_q, h_k, h_v, l_cap;
   int nsplit;    // splits per (batch, key head)
   int s_cap;     // partials stride

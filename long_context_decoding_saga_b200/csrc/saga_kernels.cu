@@ -26,6 +26,11 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <stdlib.h>
+
+#include <atomic>
+#include <utility>
+
 #include "saga_device.cuh"
 #include "saga_internal.h"
 
@@ -34,6 +39,43 @@ namespace saga {
 // ============================================================================ helpers
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// N = 2 or 4 consecutive bf16 values (8- or 4-byte aligned) as floats.
+template <int N>
+__device__ __forceinline__ void load_bf16(const uint16_t* src, float (&v)[N]) {
+  if constexpr (N == 4) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(src);
+    v[0] = bf16_lo(raw.x);
+    v[1] = bf16_hi(raw.x);
+    v[2] = bf16_lo(raw.y);
+    v[3] = bf16_hi(raw.y);
+  } else {
+    const uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
+    v[0] = bf16_lo(raw);
+    v[1] = bf16_hi(raw);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void load_bf16_global(const uint16_t* src, float (&v)[N]) {
+  if constexpr (N == 4) {
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(src));
+    v[0] = bf16_lo(raw.x);
+    v[1] = bf16_hi(raw.x);
+    v[2] = bf16_lo(raw.y);
+    v[3] = bf16_hi(raw.y);
+  } else {
+    const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(src));
+    v[0] = bf16_lo(raw);
+    v[1] = bf16_hi(raw);
+  }
+}
 
 __device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
   uint32_t out;
@@ -57,8 +99,6 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   }
 }
 
-template <int D, int NP>
-__host__ __device__ constexpr int split_stages() { return D == 128 ? (NP >= 64 ? 3 : 4) : 6; }
 
 template <int NP>
 __host__ __device__ constexpr uint32_t tmem_cols() { return (2 * NP <= 32) ? 32u : (2 * NP <= 64) ? 64u : 128u; }
@@ -88,6 +128,8 @@ struct EpiShared {
   int vu[NP];                 // local value head of each query head of the group
   int hcnt[4][NP];            // counting mode: per-warp kept counts of the current tile
   int cnt_run[NP];            // counting mode: kept so far in this split
+  int tail_buf[4][2];         // tail: each warp's unreduced list buffers ...
+  int tail_n[4][2];           // ... and their row counts
 };
 
 // Bytes of value rows each warp stages per list buffer.
@@ -141,11 +183,21 @@ __device__ __forceinline__ EpiArgs epi_args(const SplitParams& p, int b, int j0)
   return ea;
 }
 
+// Thresholds: read from p.tau; every token kept (-inf) when p.tau is null
+// (N covers every length); nothing compared in dump mode.  Padding heads keep
+// nothing (+inf).  The load is separate from the shared-memory setup so that
+// a kernel can issue all of its setup loads back to back.
 template <int NP>
-__device__ __forceinline__ void epi_setup(EpiShared<NP>& es, int et, const SplitParams& p, int b, int j0,
-                                          bool load_tau) {
+__device__ __forceinline__ float load_tau(int et, const SplitParams& p, int b, int j0, bool compare) {
+  float tv = INFINITY;
+  if (compare && et < p.G) tv = p.tau != nullptr ? __ldg(p.tau + (size_t)b * p.h_q + j0 + et) : -INFINITY;
+  return tv;
+}
+
+template <int NP>
+__device__ __forceinline__ void epi_setup(EpiShared<NP>& es, int et, const SplitParams& p, float tv) {
   if (et < NP) {
-    es.tau[et] = (load_tau && et < p.G) ? __ldg(p.tau + (size_t)b * p.h_q + j0 + et) : INFINITY;
+    es.tau[et] = tv;
     es.vu[et] = et < p.G ? et / p.hpv : 0;
     es.cnt_run[et] = 0;
   }
@@ -329,17 +381,6 @@ __device__ __forceinline__ void append_rows(EpiShared<NP>& es, WarpAcc<D, NP>& a
   ls.n = r1;
 }
 
-// Reduces whatever is left in the warp's lists.
-template <int D, int NP>
-__device__ __forceinline__ void flush_lists(EpiShared<NP>& es, WarpAcc<D, NP>& acc, const EpiArgs& ea, ListState& ls,
-                                            int q, int lane, const uint16_t* vstage_w) {
-  // the newest cp.async group belongs to the current buffer only if it holds rows
-  if (ls.pend >= 0) reduce_batch<D, NP>(es, acc, ea, q, lane, ls.pend, ls.npend, vstage_w, ls.n > 0);
-  if (ls.n > 0) reduce_batch<D, NP>(es, acc, ea, q, lane, ls.cur, ls.n, vstage_w, false);
-  ls.pend = -1;
-  ls.n = 0;
-}
-
 // Counting mode (kept counts and ascending index lists requested): the four
 // warps go through each tile together; per-head ballots give each kept
 // token its position in the split's list.
@@ -385,20 +426,26 @@ __device__ __forceinline__ void tile_epilogue(EpiShared<NP>& es, WarpAcc<D, NP>&
   if (bal != 0u) append_rows<D, NP>(es, acc, ea, ls, q, lane, bal, keep, sc, tok, vstage_w);
 }
 
-// Merges the four warps' (m, l, o) and writes the split's partial: every
-// warp writes its state, one thread per head forms the merge factors, and all
-// threads combine.  mrg holds 4 * NP * (D + 2) + 4 * NP floats, 16-byte
-// aligned.  Deterministic (fixed warp order in every sum).
+// Tail of a split: merges the four warps' running (m, l, o) with the rows
+// still waiting, unreduced, in their lists, and writes the split's partial.
+// Each warp publishes its state (in mrg: 4 * NP * (D + 2) floats, 16-byte
+// aligned) and its list descriptors.  After one barrier the unreduced rows
+// of all warps form one pool; each warp takes whole heads: its lanes first
+// hold one pool row each (weight, one max reduction per head), then the
+// columns while the rows are accumulated from shuffled weights.
+// Deterministic (fixed order in every sum).
 template <int D, int NP>
-__host__ __device__ constexpr int merge_floats() { return 4 * NP * (D + 2) + 4 * NP; }
+__host__ __device__ constexpr int merge_floats() { return 4 * NP * (D + 2); }
 
 template <int D, int NP>
-__device__ __forceinline__ void merge_and_store(const EpiShared<NP>& es, float* mrg, WarpAcc<D, NP>& acc, int q,
-                                                int lane, int et, const SplitParams& p, int b, int j0, int s) {
+__device__ __forceinline__ void tail_merge(EpiShared<NP>& es, float* mrg, const WarpAcc<D, NP>& acc,
+                                           const ListState& ls, const EpiArgs& ea, const uint16_t* vstage, int q,
+                                           int lane, int et, const SplitParams& p, int b, int j0, int s,
+                                           bool drop_lists) {
   constexpr int DPL = WarpAcc<D, NP>::DPL;
   constexpr int REG = NP * (D + 2);
-  float* mine = mrg + q * REG;  // m[NP], l[NP], o[NP][D]
-  float* fac = mrg + 4 * REG;   // [4][NP]
+  constexpr int VWE = vstage_warp_bytes<NP>();  // elements of one warp's staging area (two buffers)
+  float* mine = mrg + q * REG;                  // m[NP], l[NP], o[NP][D]
   if (lane == 0) {
 #pragma unroll
     for (int j4 = 0; j4 < NP / 4; ++j4) {
@@ -407,6 +454,10 @@ __device__ __forceinline__ void merge_and_store(const EpiShared<NP>& es, float* 
       *reinterpret_cast<float4*>(&mine[NP + 4 * j4]) =
           make_float4(acc.l[4 * j4], acc.l[4 * j4 + 1], acc.l[4 * j4 + 2], acc.l[4 * j4 + 3]);
     }
+    es.tail_buf[q][0] = ls.pend & 1;
+    es.tail_n[q][0] = (ls.pend >= 0 && !drop_lists) ? ls.npend : 0;
+    es.tail_buf[q][1] = ls.cur & 1;
+    es.tail_n[q][1] = drop_lists ? 0 : ls.n;
   }
 #pragma unroll
   for (int jl = 0; jl < NP; ++jl) {
@@ -417,61 +468,157 @@ __device__ __forceinline__ void merge_and_store(const EpiShared<NP>& es, float* 
       *reinterpret_cast<float2*>(dst) = make_float2(acc.o[jl][0], acc.o[jl][1]);
     }
   }
+  cp_async_wait_all();  // this thread's staged value rows; the barrier publishes everyone's
   named_bar_sync(1, kEpiThreads);
+
+  // the unreduced rows of all warps form one pool: (warp, buffer) lists in order
+  int off[9];
+  off[0] = 0;
+#pragma unroll
+  for (int wk = 0; wk < 8; ++wk) off[wk + 1] = off[wk] + es.tail_n[wk >> 1][wk & 1];
+  const int npool = off[8];
   const size_t row0 = (size_t)b * p.h_q + j0;
-  if (et < p.G) {
-    float m4[4], M = -INFINITY;
+  // warp q takes heads q, q+4, ...; lanes hold columns [lane*DPL, lane*DPL+DPL)
+  for (int jl = q; jl < p.G; jl += 4) {
+    const int u = (jl * ea.hmul) >> 16;  // the head's value head within the group
+    float mw[4], M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      m4[w] = mrg[w * REG + et];
-      M = fmaxf(M, m4[w]);
+      mw[w] = mrg[w * REG + jl];
+      M = fmaxf(M, mw[w]);
     }
+    for (int base = 0; base < npool; base += 32) {  // pool maximum, one row per lane
+      const int k = base + lane;
+      float sc = -INFINITY;
+      if (k < npool) {
+        int wk = 0, r = k;
+#pragma unroll
+        for (int i = 1; i < 8; ++i)
+          if (k >= off[i]) {
+            wk = i;
+            r = k - off[i];
+          }
+        const WarpList<NP>& li = es.list[wk >> 1][es.tail_buf[wk >> 1][wk & 1]];
+        if ((li.keep[r] >> jl) & 1ull) sc = li.sc[r][jl];
+      }
+      M = fmaxf(M, warp_max(sc));
+    }
+    float o[DPL];
     float lsum = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float f = (m4[w] == -INFINITY) ? 0.f : __expf(m4[w] - M);
-      fac[w * NP + et] = f;
-      lsum += f * mrg[w * REG + NP + et];
-    }
-    p.part_m[(row0 + et) * p.s_cap + s] = M;
-    p.part_l[(row0 + et) * p.s_cap + s] = lsum;
-    p.part_cnt[(row0 + et) * p.s_cap + s] = es.cnt_run[et];
-  }
-  named_bar_sync(1, kEpiThreads);
-  for (int idx = et; idx < p.G * (D / 4); idx += kEpiThreads) {
-    const int jl = idx / (D / 4), c4 = idx % (D / 4);
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = 0; e < DPL; ++e) o[e] = 0.f;
+    if (M != -INFINITY) {
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float f = fac[w * NP + jl];
-      const float4 v = *reinterpret_cast<const float4*>(&mrg[w * REG + 2 * NP + jl * D + c4 * 4]);
-      o.x = fmaf(f, v.x, o.x);
-      o.y = fmaf(f, v.y, o.y);
-      o.z = fmaf(f, v.z, o.z);
-      o.w = fmaf(f, v.w, o.w);
+      for (int w = 0; w < 4; ++w) {
+        const float f = (mw[w] == -INFINITY) ? 0.f : __expf(mw[w] - M);
+        lsum = fmaf(f, mrg[w * REG + NP + jl], lsum);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) o[e] = fmaf(f, mrg[w * REG + 2 * NP + jl * D + lane * DPL + e], o[e]);
+      }
+      for (int base = 0; base < npool; base += 32) {
+        // lane k: its pool row's weight and where its value row is (shared
+        // memory offset, or -(token + 1) for a row that was not staged)
+        const int k = base + lane;
+        float wgt = 0.f;
+        int loc = 0;
+        if (k < npool) {
+          int wk = 0, r = k;
+#pragma unroll
+          for (int i = 1; i < 8; ++i)
+            if (k >= off[i]) {
+              wk = i;
+              r = k - off[i];
+            }
+          const int bi = es.tail_buf[wk >> 1][wk & 1];
+          const WarpList<NP>& li = es.list[wk >> 1][bi];
+          if ((li.keep[r] >> jl) & 1ull) wgt = __expf(li.sc[r][jl] - M);
+          loc = r < ea.rcapw ? (wk >> 1) * VWE + ((bi * ea.rcapw + r) * ea.nvh + u) * D : -(li.tok[r] + 1);
+        }
+        lsum += warp_sum(wgt);
+        const int nrow = min(32, npool - base);
+#pragma unroll 4
+        for (int i = 0; i < nrow; ++i) {
+          const float w = __shfl_sync(0xffffffffu, wgt, i);
+          const int li_loc = __shfl_sync(0xffffffffu, loc, i);
+          if (w == 0.f) continue;  // warp-uniform
+          float v[DPL];
+          if (li_loc >= 0) {
+            load_bf16<DPL>(vstage + li_loc + lane * DPL, v);
+          } else {
+            load_bf16_global<DPL>(ea.vgroup + ((size_t)u * ea.l_cap + (size_t)(-li_loc - 1)) * D + lane * DPL, v);
+          }
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) o[e] = fmaf(w, v[e], o[e]);
+        }
+      }
     }
-    *reinterpret_cast<float4*>(&p.part_o[((row0 + jl) * p.s_cap + s) * D + c4 * 4]) = o;
+    float* dst = &p.part_o[((row0 + jl) * p.s_cap + s) * D + lane * DPL];
+    if constexpr (DPL == 4) {
+      *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+    } else {
+      *reinterpret_cast<float2*>(dst) = make_float2(o[0], o[1]);
+    }
+    if (lane == 0) {
+      p.part_m[(row0 + jl) * p.s_cap + s] = M;
+      p.part_l[(row0 + jl) * p.s_cap + s] = lsum;
+      p.part_cnt[(row0 + jl) * p.s_cap + s] = es.cnt_run[jl];
+    }
   }
 }
 
 // ============================================================================ split kernel
+constexpr int kSmemLimit = 232448;  // dynamic shared memory one CTA may use on sm_100
+
 template <int D, int NP, bool UMMA>
 struct SplitSmem {
   static constexpr int NATOM = D / 64;
   static constexpr int STAGE_BYTES = kTile * D * 2;
-  static constexpr int NSTAGE = split_stages<D, NP>();
   static constexpr int QBYTES = UMMA ? NATOM * NP * 128 : NP * D * 4;
+  static constexpr int QPAD = ((QBYTES + 1023) / 1024) * 1024;
+  static constexpr int EPI_BYTES = ((int)sizeof(EpiShared<NP>) + 127) / 128 * 128;
+  static constexpr int VST_BYTES = 4 * 2 * vstage_warp_bytes<NP>();
+  // key-tile ring: 4 tiles of 32 KB at d = 128 or 6 of 16 KB at d = 64 cover
+  // the load latency; fewer where the epilogue's buffers leave less room
+  static constexpr int FIXED = QPAD + EPI_BYTES + VST_BYTES + 2 * 8 * 8 + 5 * 8 + 16 + 1024;
+  static constexpr int NSTAGE_MAX = D == 128 ? 4 : 6;
+  static constexpr int NSTAGE_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
+  static constexpr int NSTAGE = NSTAGE_FIT < NSTAGE_MAX ? NSTAGE_FIT : NSTAGE_MAX;
+  static_assert(NSTAGE >= 3, "key-tile ring too shallow");
   static constexpr int Q_OFF = NSTAGE * STAGE_BYTES;
-  static constexpr int EPI_OFF = Q_OFF + ((QBYTES + 1023) / 1024) * 1024;
-  static constexpr int VST_OFF = EPI_OFF + ((int)sizeof(EpiShared<NP>) + 127) / 128 * 128;
-  static constexpr int BAR_OFF = VST_OFF + 4 * 2 * vstage_warp_bytes<NP>();
+  static constexpr int EPI_OFF = Q_OFF + QPAD;
+  static constexpr int VST_OFF = EPI_OFF + EPI_BYTES;
+  static constexpr int BAR_OFF = VST_OFF + VST_BYTES;
   static constexpr int NBARS = 2 * NSTAGE + 5;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
+  static_assert(ALLOC <= kSmemLimit, "shared memory over the per-CTA limit");
   static_assert(merge_floats<D, NP>() * 4 <= NSTAGE * STAGE_BYTES, "merge buffer must fit in the key stages");
   static_assert(NP * 256 * 4 <= (int)sizeof(WarpList<NP>) * 8, "dump histogram must fit in the warp lists");
 };
+
+// Fused append: row pos of key head h and of the group's value heads, from
+// k_new / v_new.  With h_v < h_k several key heads share a value head and
+// each of their splits writes the same bytes.
+template <int D>
+__device__ __forceinline__ void append_new_rows(const SplitParams& p, int b, int h, int j0, int pos) {
+  constexpr int C = D / 8;  // 16-byte chunks per row
+  const int v_base = (int)(((long long)j0 * p.h_v) / p.h_q);
+  const int n = (1 + p.nvh) * C;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int r = i / C, c = i % C;
+    if (r == 0) {
+      const size_t kh = (size_t)b * p.h_k + h;
+      const uint4 v = reinterpret_cast<const uint4*>(p.k_new + kh * D)[c];
+      reinterpret_cast<uint4*>(p.k_cache_w + (kh * p.l_cap + pos) * D)[c] = v;
+    } else {
+      const size_t vh = (size_t)b * p.h_v + v_base + r - 1;
+      const uint4 v = reinterpret_cast<const uint4*>(p.v_new + vh * D)[c];
+      reinterpret_cast<uint4*>(p.v_cache_w + (vh * p.l_cap + pos) * D)[c] = v;
+    }
+  }
+  fence_proxy_async_global();
+}
 
 // One key tile: 128 rows (or the rows left in the split, as 32-row boxes)
 // of every 64-column swizzle atom, into stage t % NSTAGE.
@@ -527,14 +674,13 @@ __global__ void __launch_bounds__(192, 1)
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j0 = h * p.G;
-  const int L = device_seq_len(p.seq_len_dev, p.seq_len, p.l_cap, (s == 0 && h == 0 && b == 0) ? p.status : nullptr);
-  int start, end;
-  split_range(L, p.nsplit, s, &start, &end);
-  const int ntiles = (end - start + kTile - 1) / kTile;
   const int row_base = (b * p.h_k + h) * p.l_cap;  // first cache row of this (batch, key head)
 
-  // ---------------------------------------------------------------- setup
-  int issued = 0;  // producer: tiles issued
+  // ---------------------------------------------------------------- setup before the dependency wait
+  // Nothing used here is written by a preceding kernel: barriers, TMEM, the
+  // tensor maps, and an L2 prefetch of the first key tiles this split can
+  // cover whatever the length (a prefetch moves no values, so it races with
+  // nothing).
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int i = 0; i < NSTAGE; ++i) {
@@ -549,36 +695,81 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init_fence();
     tma_prefetch_desc(&tmap_full);
     tma_prefetch_desc(&tmap_part);
-    // the first stages go out before the rest of the setup
-    for (; issued < ntiles && issued < NSTAGE; ++issued)
-      issue_key_tile<NATOM, NSTAGE, STAGE_BYTES>(issued, start, end, row_base, kst, full, &tmap_full, &tmap_part);
+    int pst, pcap;
+    split_cap_range(p.seq_len, p.nsplit, s, p.l_cap, &pst, &pcap);
+    const int pend = min(pcap, pst + NSTAGE * kTile);
+    const uint16_t* kb = p.k_cache + (size_t)row_base * D;
+    for (int r = pst; r < pend; r += kTile) prefetch_l2_bulk(kb + (size_t)r * D, (uint32_t)(min(kTile, pend - r) * D * 2));
   }
   if (UMMA && warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_trigger();
+  pdl_wait();
+
+  // ---------------------------------------------------------------- setup after it
+  // The global reads of this setup (q, the thresholds, the length) are issued
+  // back to back so that their latencies overlap.
+  constexpr int QCH = UMMA ? NATOM * NP * 8 : NP * D / 8;  // 16-byte chunks of the group's q (padded heads)
+  constexpr int QV = (QCH + kEpiThreads - 1) / kEpiThreads;
+  const int eth = threadIdx.x - 64;  // epilogue thread (warps 2..5)
+  uint4 qv[QV];
+  float tv = INFINITY;
   if (warp >= 2) {
-    const int et = threadIdx.x - 64;
-    epi_setup<NP>(es, et, p, b, j0, !DUMP);
-    if (UMMA) {
-      // q as the K-major B operand in the 128-byte swizzle layout; rows >= G are zero
-      for (int i = et; i < NATOM * NP * 8; i += kEpiThreads) {
-        const int a = i / (NP * 8), n = (i / 8) % NP, c = i % 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (n < p.G) v = *reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.h_q + j0 + n) * D + a * 64 + c * 8);
-        *reinterpret_cast<uint4*>(qsm + a * NP * 128 + n * 128 + ((c ^ (n & 7)) << 4)) = v;
+#pragma unroll
+    for (int k = 0; k < QV; ++k) {
+      const int i = eth + k * kEpiThreads;
+      int n, col;
+      if (UMMA) {
+        n = (i / 8) % NP;
+        col = (i / (NP * 8)) * 64 + (i % 8) * 8;
+      } else {
+        n = i / (D / 8);
+        col = (i % (D / 8)) * 8;
       }
-    } else {
-      float* qf = reinterpret_cast<float*>(qsm);
-      for (int i = et; i < NP * D; i += kEpiThreads) {
-        const int n = i / D, k = i % D;
-        float v = 0.f;
-        if (n < p.G) v = __uint_as_float((uint32_t)p.q[((size_t)b * p.h_q + j0 + n) * D + k] << 16);
-        qf[i] = v;
+      qv[k] = make_uint4(0, 0, 0, 0);
+      if (i < QCH && n < p.G)
+        qv[k] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.h_q + j0 + n) * D + col));
+    }
+    tv = load_tau<NP>(eth, p, b, j0, !DUMP);
+  }
+  const int L = device_seq_len(p.seq_len_dev, p.seq_len, p.l_cap, (s == 0 && h == 0 && b == 0) ? p.status : nullptr);
+  int start, end;
+  split_range(p.seq_len, p.nsplit, s, L, &start, &end);
+  const int ntiles = (end - start + kTile - 1) / kTile;
+  // fused append: the split holding row L - 1 writes the new key/value rows;
+  // its tile holding that row is loaded only after the barrier below
+  const bool owner = p.k_new != nullptr && start <= L - 1 && L - 1 < end;
+  if (owner) append_new_rows<D>(p, b, h, j0, L - 1);
+  int issued = 0;  // producer: tiles issued
+  if (threadIdx.x == 0) {
+    for (; issued < ntiles && issued < NSTAGE; ++issued) {
+      if (owner && L - 1 < start + (issued + 1) * kTile) break;
+      issue_key_tile<NATOM, NSTAGE, STAGE_BYTES>(issued, start, end, row_base, kst, full, &tmap_full, &tmap_part);
+    }
+  }
+  if (warp >= 2) {
+    epi_setup<NP>(es, eth, p, tv);
+#pragma unroll
+    for (int k = 0; k < QV; ++k) {
+      const int i = eth + k * kEpiThreads;
+      if (i < QCH) {
+        if (UMMA) {
+          // q as the K-major B operand in the 128-byte swizzle layout; rows >= G are zero
+          const int a = i / (NP * 8), n = (i / 8) % NP, c = i % 8;
+          *reinterpret_cast<uint4*>(qsm + a * NP * 128 + n * 128 + ((c ^ (n & 7)) << 4)) = qv[k];
+        } else {
+          float* qf = reinterpret_cast<float*>(qsm) + (i / (D / 8)) * D + (i % (D / 8)) * 8;
+          *reinterpret_cast<float4*>(qf) = make_float4(bf16_lo(qv[k].x), bf16_hi(qv[k].x), bf16_lo(qv[k].y),
+                                                       bf16_hi(qv[k].y));
+          *reinterpret_cast<float4*>(qf + 4) = make_float4(bf16_lo(qv[k].z), bf16_hi(qv[k].z), bf16_lo(qv[k].w),
+                                                           bf16_hi(qv[k].w));
+        }
       }
     }
     if (DUMP)
-      for (int i = et; i < NP * 256; i += kEpiThreads) hist[i] = 0u;
+      for (int i = eth; i < NP * 256; i += kEpiThreads) hist[i] = 0u;
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
@@ -589,6 +780,7 @@ __global__ void __launch_bounds__(192, 1)
   // ---------------------------------------------------------------- roles
   if (warp == 0) {
     if (lane == 0) {
+      if (owner) fence_proxy_async_global();  // the appended rows (written before the barrier) reach TMA
       for (int t = issued; t < ntiles; ++t) {
         const int stage = t % NSTAGE, round = t / NSTAGE;
         if (round > 0 && !mbar_wait(&empty[stage], (round - 1) & 1, abort_flag)) break;
@@ -705,10 +897,12 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     if (!DUMP) {
-      if (t == ntiles) flush_lists<D, NP>(es, acc, ea, ls, q, lane, vstage_w);
-      cp_async_wait_all();
-      named_bar_sync(1, kEpiThreads);  // every warp is done with the key stages (merge buffer below)
-      merge_and_store<D, NP>(es, reinterpret_cast<float*>(kst), acc, q, lane, et, p, b, j0, s);
+      // the warps' states go into the key ring: with tcgen05 it is free once a
+      // warp has seen the last tile's scores (every MMA and copy is done); on
+      // the CUDA-core path the other warps may still be reading it
+      if (!UMMA) named_bar_sync(1, kEpiThreads);
+      tail_merge<D, NP>(es, reinterpret_cast<float*>(kst), acc, ls, ea, vstage, q, lane, et, p, b, j0, s,
+                        t != ntiles);
     }
   }
 
@@ -763,13 +957,15 @@ __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const Spl
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int et = threadIdx.x, q = et >> 5, lane = et & 31;
   const int j0 = h * p.G;
+  pdl_trigger();
+  pdl_wait();
   const int L = device_seq_len(p.seq_len_dev, p.seq_len, p.l_cap, nullptr);
   int start, end;
-  split_range(L, p.nsplit, s, &start, &end);
+  split_range(p.seq_len, p.nsplit, s, L, &start, &end);
   const int ntiles = (end - start + kTile - 1) / kTile;
   const bool counting = p.want_counts != 0;
 
-  epi_setup<NP>(es, et, p, b, j0, true);
+  epi_setup<NP>(es, et, p, load_tau<NP>(et, p, b, j0, true));
   const EpiArgs ea = epi_args<D, NP>(p, b, j0);
   uint16_t* vstage_w = vstage + (size_t)q * 2 * (vstage_warp_bytes<NP>() / 2);
   WarpAcc<D, NP> acc;
@@ -788,84 +984,90 @@ __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const Spl
     const int tok = start + t * kTile + et;
     tile_epilogue<D, NP>(es, acc, ea, ls, q, lane, et, sc, tok, tok < end, counting, p, b, j0, start, vstage_w);
   }
-  flush_lists<D, NP>(es, acc, ea, ls, q, lane, vstage_w);
-  cp_async_wait_all();
-  named_bar_sync(1, kEpiThreads);
-  merge_and_store<D, NP>(es, mrg, acc, q, lane, et, p, b, j0, s);
+  tail_merge<D, NP>(es, mrg, acc, ls, ea, vstage, q, lane, et, p, b, j0, s, false);
 }
 
 // ============================================================================ combine kernel
 // O[b, j] = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s over the splits of
 // row (b, j); zero when nothing was kept.  Also the kept counts and the
 // ascending index list (concatenation of the per-split lists in split order).
-constexpr int kCombineThreads = 512;
+
+// Grid: (B*h_q rows, D/32 column chunks).  Warp w of a CTA takes splits
+// w, w+32, ... in blocks of eight (all loads of a block in flight at once)
+// with its own running maximum; lane c holds column 32*chunk + c, so every
+// load of a partial is one coalesced 128-byte segment.  The warps' states
+// are merged at the end in a fixed order (deterministic).
+constexpr int kCombineThreads = 1024;
 
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads) saga_combine_kernel(const CombineParams p) {
-  constexpr int DPL = D / 32;  // dims per lane
   constexpr int NW = kCombineThreads / 32;
-  __shared__ float red_m[NW];
-  __shared__ float wsum[NW];
-  __shared__ float wacc[NW][D];
+  constexpr int U = 8;
+  __shared__ float wm[NW], wden[NW];
+  __shared__ float wacc[NW][32];
   __shared__ int cnt_scan[kCombineThreads];
-  const int row = blockIdx.x;
+  const int row = blockIdx.x, chunk = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_trigger();
+  pdl_wait();
   const int S = p.nsplit;
   const float* pm = p.part_m + (size_t)row * p.s_cap;
   const float* pl = p.part_l + (size_t)row * p.s_cap;
-  const float* po = p.part_o + (size_t)row * p.s_cap * D;
+  const float* po = p.part_o + (size_t)row * p.s_cap * D + chunk * 32 + lane;
 
-  float m = -INFINITY;
-  for (int s = threadIdx.x; s < S; s += kCombineThreads) m = fmaxf(m, pm[s]);
-  m = warp_max(m);
-  if (lane == 0) red_m[warp] = m;
-  __syncthreads();
-  float M = red_m[0];
+  float m_run = -INFINITY, den = 0.f, acc = 0.f;
+  for (int s0 = warp; s0 < S; s0 += U * NW) {
+    float ms[U], ls[U], v[U];
 #pragma unroll
-  for (int w = 1; w < NW; ++w) M = fmaxf(M, red_m[w]);
-
-  float acc[DPL];
+    for (int u = 0; u < U; ++u) {
+      const int ss = s0 + u * NW;
+      const bool in = ss < S;
+      ms[u] = in ? pm[ss] : -INFINITY;
+      ls[u] = in ? pl[ss] : 0.f;
+      v[u] = in ? po[(size_t)ss * D] : 0.f;
+    }
+    float mb = ms[0];
 #pragma unroll
-  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  float den = 0.f;
-  if (M != -INFINITY) {
-    for (int s = warp; s < S; s += NW) {
-      const float ms = pm[s];
-      if (ms == -INFINITY) continue;
-      const float f = __expf(ms - M);
-      den = fmaf(f, pl[s], den);
-      const float* src = po + (size_t)s * D + lane * DPL;
-      if (DPL == 4) {
-        const float4 v = *reinterpret_cast<const float4*>(src);
-        acc[0] = fmaf(f, v.x, acc[0]);
-        acc[1] = fmaf(f, v.y, acc[1]);
-        acc[2] = fmaf(f, v.z, acc[2]);
-        acc[3] = fmaf(f, v.w, acc[3]);
-      } else {
-        const float2 v = *reinterpret_cast<const float2*>(src);
-        acc[0] = fmaf(f, v.x, acc[0]);
-        acc[1] = fmaf(f, v.y, acc[1]);
-      }
+    for (int u = 1; u < U; ++u) mb = fmaxf(mb, ms[u]);
+    if (mb > m_run) {  // warp-uniform
+      const float f = (m_run == -INFINITY) ? 0.f : __expf(m_run - mb);
+      den *= f;
+      acc *= f;
+      m_run = mb;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float f = (ms[u] == -INFINITY) ? 0.f : __expf(ms[u] - m_run);
+      den = fmaf(f, ls[u], den);
+      acc = fmaf(f, v[u], acc);
     }
   }
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) wacc[warp][lane * DPL + e] = acc[e];
-  if (lane == 0) wsum[warp] = den;
+  wacc[warp][lane] = acc;
+  if (lane == 0) {
+    wm[warp] = m_run;
+    wden[warp] = den;
+  }
   __syncthreads();
-  if (threadIdx.x < D) {
+  if (threadIdx.x < 32) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, wm[w]);
     float num = 0.f, dd = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-      num += wacc[w][threadIdx.x];
-      dd += wsum[w];
+      const float f = (wm[w] == -INFINITY) ? 0.f : __expf(wm[w] - M);
+      num = fmaf(f, wacc[w][threadIdx.x], num);
+      dd = fmaf(f, wden[w], dd);
     }
     const float o = (M == -INFINITY || dd <= 0.f) ? 0.f : num / dd;
+    const size_t oi = (size_t)row * D + chunk * 32 + threadIdx.x;
     if (p.out_bf16) {
-      reinterpret_cast<__nv_bfloat16*>(p.out)[(size_t)row * D + threadIdx.x] = __float2bfloat16_rn(o);
+      reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
     } else {
-      reinterpret_cast<float*>(p.out)[(size_t)row * D + threadIdx.x] = o;
+      reinterpret_cast<float*>(p.out)[oi] = o;
     }
   }
+  if (chunk != 0) return;
   if (p.sel_count == nullptr) return;
   // kept counts and index lists
   const int* pc = p.part_cnt + (size_t)row * p.s_cap;
@@ -892,7 +1094,7 @@ __global__ void __launch_bounds__(kCombineThreads) saga_combine_kernel(const Com
       for (int k = warp; k < nloc; k += NW) {
         const int ss = base + k;
         int st, en;
-        split_range(L, S, ss, &st, &en);
+        split_range(p.seq_len, S, ss, L, &st, &en);
         const int cnt = pc[ss];
         const int off = cnt_scan[k];
         const int* src = p.idxbuf + (size_t)row * p.l_cap + st;
@@ -976,6 +1178,8 @@ __global__ void __launch_bounds__(kSelectThreads) atopn_select_kernel(const Sele
   __shared__ uint32_t s_bin, s_rank, s_cnt;
   __shared__ int ncand;
   const int r = blockIdx.x;
+  pdl_trigger();
+  pdl_wait();
   int L = p.row_len;
   if (p.seq_len_dev != nullptr) L = device_seq_len(p.seq_len_dev, p.row_len, p.l_cap, nullptr);
   if (p.n_top >= L) {
@@ -1042,6 +1246,8 @@ __global__ void saga_append_kernel(const AppendParams p) {
   const int chunks_row = p.d / 8;  // 16-byte chunks per row
   const int nk = p.batch * p.h_k * chunks_row, nv = p.batch * p.h_v * chunks_row;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
   if (i >= nk + nv) return;
   int pos = p.pos;
   if (p.seq_len_dev != nullptr) pos = device_seq_len(p.seq_len_dev, p.pos + 1, p.l_cap, i == 0 ? p.status : nullptr) - 1;
@@ -1059,53 +1265,87 @@ __global__ void saga_append_kernel(const AppendParams p) {
 
 __global__ void saga_fill_kernel(float* dst, float v, int n) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
   if (i < n) dst[i] = v;
 }
 
 // ============================================================================ launchers
+// Every kernel is launched with programmatic stream serialization: it may
+// start while the previous kernel on the stream finishes, runs its
+// independent setup, and waits (pdl_wait) before touching shared data.
+// SAGA_PDL=0 in the environment turns this off (plain stream order).
+static bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("SAGA_PDL");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// cudaFuncSetAttribute holds per device: one bit per device ordinal.
+static cudaError_t ensure_smem(const void* fn, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
+
 template <int D, int NP, bool UMMA, bool DUMP>
 static cudaError_t run_split(const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p, dim3 grid,
                              cudaStream_t st, int* occ) {
   using K = SplitSmem<D, NP, UMMA>;
-  static bool prepared = false;
-  if (!prepared) {
-    cudaError_t e = cudaFuncSetAttribute(saga_split_kernel<D, NP, UMMA, DUMP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, K::ALLOC);
-    if (e != cudaSuccess) return e;
-    prepared = true;
-  }
+  static std::atomic<uint64_t> prepared{0};
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(saga_split_kernel<D, NP, UMMA, DUMP>), K::ALLOC, prepared);
+  if (e != cudaSuccess) return e;
   if (occ != nullptr)
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, saga_split_kernel<D, NP, UMMA, DUMP>, 192, K::ALLOC);
-  saga_split_kernel<D, NP, UMMA, DUMP><<<grid, 192, K::ALLOC, st>>>(tf, tp, p);
-  return cudaGetLastError();
+  return launch_k(saga_split_kernel<D, NP, UMMA, DUMP>, grid, dim3(192), K::ALLOC, st, tf, tp, p);
 }
 
 template <int D>
 static cudaError_t dispatch_np(int NP, bool dump, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p,
                                dim3 g, cudaStream_t st, int* occ) {
-#define SAGA_NP(NN, UM)                                                                \
-  case NN:                                                                            \
-    return dump ? run_split<D, NN, UM, true>(tf, tp, p, g, st, occ)                   \
-                : run_split<D, NN, UM, false>(tf, tp, p, g, st, occ);
   switch (NP) {
-    SAGA_NP(4, false)
-    SAGA_NP(16, true)
-    SAGA_NP(32, true)
+    case 4: return dump ? run_split<D, 4, false, true>(tf, tp, p, g, st, occ) : run_split<D, 4, false, false>(tf, tp, p, g, st, occ);
+    case 16: return dump ? run_split<D, 16, true, true>(tf, tp, p, g, st, occ) : run_split<D, 16, true, false>(tf, tp, p, g, st, occ);
+    case 32: return dump ? run_split<D, 32, true, true>(tf, tp, p, g, st, occ) : run_split<D, 32, true, false>(tf, tp, p, g, st, occ);
     case 64:
       if constexpr (D == 64) {
-        return dump ? run_split<D, 64, true, true>(tf, tp, p, g, st, occ)
-                    : run_split<D, 64, true, false>(tf, tp, p, g, st, occ);
+        return dump ? run_split<D, 64, true, true>(tf, tp, p, g, st, occ) : run_split<D, 64, true, false>(tf, tp, p, g, st, occ);
       } else {
         return cudaErrorInvalidValue;  // d = 128 supports at most 32 query heads per key head
       }
     default:
       return cudaErrorInvalidValue;
   }
-#undef SAGA_NP
 }
 
-cudaError_t launch_split(int D, int NP, bool dump, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p,
+// mode: kSplitDense / kSplitSparse attend (they differ only in p.tau, null
+// for dense), kSplitDump dumps scores for a refresh.
+cudaError_t launch_split(int D, int NP, int mode, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p,
                          dim3 grid, cudaStream_t st, int* occupancy_out) {
+  const bool dump = mode == kSplitDump;
   if (D == 64) return dispatch_np<64>(NP, dump, tf, tp, p, grid, st, occupancy_out);
   if (D == 128) return dispatch_np<128>(NP, dump, tf, tp, p, grid, st, occupancy_out);
   return cudaErrorInvalidValue;
@@ -1113,16 +1353,11 @@ cudaError_t launch_split(int D, int NP, bool dump, const CUtensorMap& tf, const 
 
 template <int D, int NP>
 static cudaError_t run_from_scores(const SplitParams& p, dim3 grid, cudaStream_t st) {
-  static bool prepared = false;
+  static std::atomic<uint64_t> prepared{0};
   const int bytes = FromScoresSmem<D, NP>::BYTES;
-  if (!prepared) {
-    cudaError_t e =
-        cudaFuncSetAttribute(saga_from_scores_kernel<D, NP>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    prepared = true;
-  }
-  saga_from_scores_kernel<D, NP><<<grid, kEpiThreads, bytes, st>>>(p);
-  return cudaGetLastError();
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(saga_from_scores_kernel<D, NP>), bytes, prepared);
+  if (e != cudaSuccess) return e;
+  return launch_k(saga_from_scores_kernel<D, NP>, grid, dim3(kEpiThreads), bytes, st, p);
 }
 
 cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, cudaStream_t st) {
@@ -1135,33 +1370,26 @@ cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, c
 }
 
 cudaError_t launch_combine(int D, const CombineParams& p, cudaStream_t st) {
-  if (D == 64) saga_combine_kernel<64><<<p.rows, kCombineThreads, 0, st>>>(p);
-  else if (D == 128) saga_combine_kernel<128><<<p.rows, kCombineThreads, 0, st>>>(p);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (D == 64) return launch_k(saga_combine_kernel<64>, dim3(p.rows, 2), dim3(kCombineThreads), 0, st, p);
+  if (D == 128) return launch_k(saga_combine_kernel<128>, dim3(p.rows, 4), dim3(kCombineThreads), 0, st, p);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_select(const SelectParams& p, int rows, cudaStream_t st) {
-  static bool done = false;
+  static std::atomic<uint64_t> prepared{0};
   const int bytes = kSelectCap * 4;
-  if (!done) {
-    cudaError_t e = cudaFuncSetAttribute(atopn_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    done = true;
-  }
-  atopn_select_kernel<<<rows, kSelectThreads, bytes, st>>>(p);
-  return cudaGetLastError();
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(atopn_select_kernel), bytes, prepared);
+  if (e != cudaSuccess) return e;
+  return launch_k(atopn_select_kernel, dim3(rows), dim3(kSelectThreads), bytes, st, p);
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st) {
   const int n = p.batch * (p.h_k + p.h_v) * (p.d / 8);
-  saga_append_kernel<<<(n + 255) / 256, 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_k(saga_append_kernel, dim3((n + 255) / 256), dim3(256), 0, st, p);
 }
 
 cudaError_t launch_fill(float* dst, float v, int n, cudaStream_t st) {
-  saga_fill_kernel<<<(n + 255) / 256, 256, 0, st>>>(dst, v, n);
-  return cudaGetLastError();
+  return launch_k(saga_fill_kernel, dim3((n + 255) / 256), dim3(256), 0, st, dst, v, n);
 }
 
 }  // namespace saga

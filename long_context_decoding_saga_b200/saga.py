@@ -29,7 +29,7 @@ SAGA_STATUS_TIMEOUT = 0x2
 
 EXPORTED = ("saga_workspace_bytes", "saga_kv_append", "atopn_refresh_threshold", "atopn_select_workspace_bytes",
             "atopn_select_threshold", "saga_decode_attn", "saga_trace_next_attention", "saga_get_status", "saga_last_error", "saga_abi_version",
-            "saga_noalloc_scratch_bytes", "saga_decode_attn_noalloc", "saga_noalloc_last_error")
+            "saga_noalloc_scratch_bytes", "saga_decode_attn_noalloc", "saga_noalloc_last_error", "saga_decode_step")
 
 
 class SagaError(RuntimeError):
@@ -78,6 +78,9 @@ def load(path: Optional[str] = None):
     lib.saga_decode_attn.argtypes = [sp, _P, _P, _P, _I, _P, _I, _I, ctypes.c_longlong, _P, _P, _I, _P, _P, _P,
                                      ctypes.c_size_t, _P]
     lib.saga_decode_attn.restype = _I
+    lib.saga_decode_step.argtypes = [sp, _P, _P, _P, _P, _P, _I, _P, _I, _I, ctypes.c_longlong, _P, _P, _I, _P, _P,
+                                     _P, ctypes.c_size_t, _P]
+    lib.saga_decode_step.restype = _I
     lib.saga_trace_next_attention.argtypes = [_P, _P]
     lib.saga_trace_next_attention.restype = _I
     lib.saga_get_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint)]
@@ -204,6 +207,37 @@ def saga_decode_attn(shape: SagaShape, q, k_cache, v_cache, seq_len: int, n_top:
                                    _ptr(seq_len_dev), int(n_top), int(refresh_interval), int(step), _ptr(tau),
                                    _ptr(out), out_dtype, _ptr(sel_count), _ptr(sel_idx), _ptr(workspace),
                                    workspace.numel(), _stream(stream)))
+
+
+def saga_decode_step(shape: SagaShape, q, k_new, v_new, k_cache, v_cache, seq_len: int, n_top: int,
+                     refresh_interval: int, step: int, tau, out, workspace, sel_count=None, sel_idx=None,
+                     seq_len_dev=None, stream=None):
+    """saga_kv_append at seq_len - 1 and saga_decode_attn, with the append done inside the attention kernels."""
+    B, hq, hk, hv, d, lc = shape.astuple()
+    _expect(q, "q", torch.bfloat16, (B, hq, d))
+    _expect(k_new, "k_new", torch.bfloat16, (B, hk, d))
+    _expect(v_new, "v_new", torch.bfloat16, (B, hv, d))
+    _expect(k_cache, "k_cache", torch.bfloat16, (B, hk, lc, d))
+    _expect(v_cache, "v_cache", torch.bfloat16, (B, hv, lc, d))
+    _expect(tau, "tau", torch.float32, (B, hq))
+    if out.dtype == torch.float32:
+        out_dtype = SAGA_OUT_F32
+    elif out.dtype == torch.bfloat16:
+        out_dtype = SAGA_OUT_BF16
+    else:
+        raise TypeError("out must be float32 or bfloat16")
+    _expect(out, "out", out.dtype, (B, hq, d))
+    _expect(workspace, "workspace", torch.uint8)
+    if sel_count is not None:
+        _expect(sel_count, "sel_count", torch.int32, (B, hq))
+    if sel_idx is not None:
+        _expect(sel_idx, "sel_idx", torch.int32, (B, hq, lc))
+    if seq_len_dev is not None:
+        _expect(seq_len_dev, "seq_len_dev", torch.int32)
+    _check(load().saga_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                   _ptr(v_cache), int(seq_len), _ptr(seq_len_dev), int(n_top), int(refresh_interval),
+                                   int(step), _ptr(tau), _ptr(out), out_dtype, _ptr(sel_count), _ptr(sel_idx),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def saga_trace_next_attention(ev_start: Optional[torch.cuda.Event], ev_end: Optional[torch.cuda.Event]):

@@ -3,8 +3,9 @@
 Holds one K and one V cache per layer (K and V stored separately, each with
 its own head count), the per-layer Atop-N thresholds, a workspace shared by
 the layers (their calls are sequential on one stream) and the output of every
-layer.  A decode step is, for every layer: append the new token's key/value
-rows, then the attention step (refresh on t % R == 0).
+layer.  A decode step is, for every layer, one saga_decode_step call: the
+new token's key/value rows are appended by the attention kernels, then the
+attention step runs (refresh on t % R == 0).
 
 `capture()` records one decode step of all layers into two CUDA graphs (a
 refresh step and a reuse step).  The graphs read the sequence length from a
@@ -57,10 +58,8 @@ class DecodeSession:
         self.length = l
 
     def _layer_step(self, i, q, k_new, v_new, seq_len, step, seq_len_dev=None):
-        s = self.shape
-        saga.saga_kv_append(s, self.k_cache[i], self.v_cache[i], k_new, v_new, seq_len - 1, seq_len_dev=seq_len_dev)
-        saga.saga_decode_attn(s, q, self.k_cache[i], self.v_cache[i], seq_len, self.n_top, self.refresh, step,
-                              self.tau[i], self.out[i], self.workspace,
+        saga.saga_decode_step(self.shape, q, k_new, v_new, self.k_cache[i], self.v_cache[i], seq_len, self.n_top,
+                              self.refresh, step, self.tau[i], self.out[i], self.workspace,
                               sel_count=None if self.sel_count is None else self.sel_count[i],
                               sel_idx=None if self.sel_idx is None else self.sel_idx[i], seq_len_dev=seq_len_dev)
 
@@ -109,12 +108,12 @@ class DecodeSession:
         return self.out
 
     def launches_per_step(self, refresh_step: bool) -> int:
-        """Kernels of this library launched per decode step (append, attention kernels)."""
+        """Kernels of this library launched per decode step (the append is fused into the first of them)."""
         dense = self.n_top >= self.shape.l_cap
         if refresh_step and not dense:
-            per_layer = 1 + 4  # append, score dump, radix select, from-scores, combine
+            per_layer = 4  # score dump (+append), radix select, from-scores, combine
         elif refresh_step and dense:
-            per_layer = 1 + 3  # append, threshold fill, split, combine
+            per_layer = 3  # threshold fill, split (+append), combine
         else:
-            per_layer = 1 + 2  # append, split, combine
+            per_layer = 2  # split (+append), combine
         return self.layers * per_layer

@@ -105,3 +105,123 @@ def run_parity(wl: workload.Workload, steps: int, layer: int = 0, gen_device: st
     status = saga.saga_get_status(sess.workspace)
     assert status & saga.SAGA_STATUS_TIMEOUT == 0
     return reports, sess
+
+
+# ---------------------------------------------------------------------------- full-size sampled parity
+def oracle_rows(inp, h_q, h_k, h_v, n_top, refresh, t, b, h):
+    """The oracle's result at decode step t for the query heads of key head h, batch b, one group at a time.
+
+    inp holds float32 numpy copies of the bf16 inputs: "K"[(b, h)] and "V"[(b, u)] the prefilled rows
+    [l_kv, d] of one head, "q" [steps, B, h_q, d], "k_new" [steps, B, h_k, d], "v_new" [steps, B, h_v, d].
+    Rebuilds the caches at steps r = t - t % R and t, takes the threshold from step r's own scores (the
+    refresh step) and applies it at step t.  Returns dict(out, tau, keep, scores).
+    """
+    G = h_q // h_k
+    js = list(range(h * G, (h + 1) * G))
+    l_kv = inp["K"][(b, h)].shape[0]
+    r = t - t % refresh
+
+    def cache(rows0, new, head):
+        return np.concatenate([rows0, new[:t + 1, b, head]], axis=0)[None, None]  # [1, 1, L, d]
+
+    Kh = cache(inp["K"][(b, h)], inp["k_new"], h)
+    L = Kh.shape[2]
+    # eq. 2 for the group's query heads against key head h (the group as the oracle's query heads)
+    A_t = saga_oracle.scores(inp["q"][t, b, js][None], Kh, L)[0]  # [G, L]
+    L_r = l_kv + r + 1
+    if n_top >= L_r:
+        tau = np.full(G, -np.inf, dtype=np.float32)
+    else:
+        A_r = A_t if r == t else saga_oracle.scores(inp["q"][r, b, js][None], Kh, L_r)[0]
+        tau = np.array([saga_oracle.nth_largest(A_r[g], n_top) for g in range(G)], dtype=np.float32)
+    keep = saga_oracle.select(A_t[None], tau[None])[0]
+    outs = np.zeros((G, inp["K"][(b, h)].shape[1]))
+    for g, j in enumerate(js):
+        u = saga_oracle.value_head(j, h_q, h_v)
+        Vh = cache(inp["V"][(b, u)], inp["v_new"], u)
+        outs[g] = saga_oracle.sparse_attention(A_t[None, g:g + 1], keep[None, g:g + 1], Vh, L)[0, 0]
+    return {"out": outs, "tau": tau, "keep": keep, "scores": A_t}
+
+
+def run_full_sampled(wl: workload.Workload, check_layers: Sequence[int], check_steps: Sequence[int],
+                     check_groups: Sequence[tuple], layers: Optional[int] = None, track: bool = False):
+    """All layers of `wl` per step through CUDA-graph replays with a device-side length (the benchmark's
+    launch configuration).  Returns the GPU rows of the checked (layer, step, batch, key head) groups, the
+    inputs those groups need (float32 numpy) and the N passed to the kernels."""
+    nl = wl.layers if layers is None else layers
+    steps = max(check_steps) + 1
+    l_cap = wl.l_kv + steps
+    n_top = wl.n_for_kernel(l_cap)
+    shape = saga.SagaShape.of(wl.batch, wl.h_q, wl.h_k, wl.h_v, wl.d, l_cap)
+    sess = DecodeSession(shape, nl, n_top, wl.refresh, device="cuda", track_selection=track)
+    G = wl.h_q // wl.h_k
+    qs, ks, vs, inputs = [], [], [], {}
+    for i in range(nl):
+        inp = workload.make_layer(wl, i, device="cuda", steps=steps)
+        sess.prefill(i, inp["K0"], inp["V0"])
+        qs.append(inp["q"])
+        ks.append(inp["k_new"])
+        vs.append(inp["v_new"])
+        if i in check_layers:
+            keep = {"K": {}, "V": {}}
+            for (b, h) in check_groups:
+                keep["K"][(b, h)] = inp["K0"][b, h].float().cpu().numpy()
+                for j in range(h * G, (h + 1) * G):
+                    u = saga_oracle.value_head(j, wl.h_q, wl.h_v)
+                    if (b, u) not in keep["V"]:
+                        keep["V"][(b, u)] = inp["V0"][b, u].float().cpu().numpy()
+            for k in ("q", "k_new", "v_new"):
+                keep[k] = inp[k].float().cpu().numpy()
+            inputs[i] = keep
+        del inp
+    q_all, k_all, v_all = torch.stack(qs, 1), torch.stack(ks, 1), torch.stack(vs, 1)
+    del qs, ks, vs
+    got = {}
+
+    def grab(t):
+        torch.cuda.synchronize()
+        for i in check_layers:
+            for (b, h) in check_groups:
+                js = slice(h * G, (h + 1) * G)
+                row = {"out": sess.out[i, b, js].cpu().numpy().astype(np.float64),
+                       "tau": sess.tau[i, b, js].cpu().numpy()}
+                if track:
+                    row["count"] = sess.sel_count[i, b, js].cpu().numpy()
+                    row["idx"] = sess.sel_idx[i, b, js].cpu().numpy()
+                got[(i, t, b, h)] = row
+
+    sess.step(q_all[0], k_all[0], v_all[0])  # step 0 eagerly, then the step graphs (as the benchmark does)
+    sess.capture()
+    if 0 in check_steps:
+        grab(0)
+    for t in range(1, steps):
+        sess.stage(q_all[t], k_all[t], v_all[t])
+        sess.replay()
+        if t in check_steps:
+            grab(t)
+    torch.cuda.synchronize()
+    status = saga.saga_get_status(sess.workspace)
+    assert status & saga.SAGA_STATUS_TIMEOUT == 0
+    del sess
+    return got, inputs, n_top
+
+
+def check_full_sampled(wl, got, inputs, n_top, track):
+    """Compares every grabbed group with the oracle; returns the largest output difference."""
+    worst = 0.0
+    for (i, t, b, h), row in got.items():
+        res = oracle_rows(inputs[i], wl.h_q, wl.h_k, wl.h_v, n_top, wl.refresh, t, b, h)
+        err = float(np.max(np.abs(row["out"] - res["out"])))
+        assert err <= OUT_TOL, f"layer {i} step {t} b {b} h {h}: max |out diff| {err}"
+        worst = max(worst, err)
+        with np.errstate(invalid="ignore"):
+            both = np.isneginf(res["tau"]) & np.isneginf(row["tau"])
+            terr = np.where(both, 0.0, np.abs(row["tau"].astype(np.float64) - res["tau"].astype(np.float64)))
+        assert float(np.max(terr)) <= BAND, f"layer {i} step {t}: threshold differs by {float(np.max(terr))}"
+        if track:
+            L = res["scores"].shape[1]
+            keep_g = keep_mask_from_lists(row["count"][None], row["idx"][None], L)[0]
+            far = np.abs(res["scores"].astype(np.float64) - res["tau"].astype(np.float64)[:, None]) > BAND
+            mism = (keep_g != res["keep"]) & far
+            assert not mism.any(), f"layer {i} step {t}: {int(mism.sum())} index mismatches outside the band"
+    return worst

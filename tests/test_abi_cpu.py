@@ -89,3 +89,19 @@ def test_binding_refuses_cpu_tensors(lib):
         saga.saga_kv_append(s, torch.zeros(1, 1, 1024, 64, dtype=torch.bfloat16),
                             torch.zeros(1, 8, 1024, 64, dtype=torch.bfloat16),
                             torch.zeros(1, 1, 64, dtype=torch.bfloat16), torch.zeros(1, 8, 64, dtype=torch.bfloat16), 0)
+
+
+def _step(lib, shape, k_new=FAKE, v_new=FAKE, seq_len=10):
+    p = FAKE
+    return lib.saga_decode_step(ctypes.byref(shape), p, k_new, v_new, p, p, seq_len, None, 4, 2, 0, p, p, 0, None,
+                                None, p, 1 << 30, None)
+
+
+def test_decode_step_validation(lib):
+    s = _shape()
+    assert _step(lib, s, k_new=None) == saga.SAGA_ERR_ARG
+    assert _step(lib, s, v_new=None) == saga.SAGA_ERR_ARG
+    assert _step(lib, s, k_new=ctypes.c_void_p(0x100008)) == saga.SAGA_ERR_ARG  # not 16-byte aligned
+    assert _step(lib, s, seq_len=0) == saga.SAGA_ERR_ARG
+    assert _step(lib, _shape(d=96)) == saga.SAGA_ERR_UNSUPPORTED
+    assert lib.saga_last_error()

@@ -189,3 +189,80 @@ def test_device_length_out_of_range_is_clamped_and_flagged():
     st = saga.saga_get_status(ws)
     assert st & saga.SAGA_STATUS_LEN_CLAMPED
     assert not st & saga.SAGA_STATUS_TIMEOUT
+
+
+@pytest.mark.parametrize("wl", [
+    small("fused_g12_d128", h_q=12, h_k=1, h_v=4, d=128, l_kv=2085, n_top=50, refresh=3, steps=5),
+    small("fused_hv_lt_hk", h_q=8, h_k=4, h_v=2, d=128, l_kv=903, n_top=25, refresh=2, steps=4, batch=2),
+    small("fused_dense", h_q=16, h_k=4, h_v=4, d=64, l_kv=700, n_top=workload.DENSE, refresh=1 << 30,
+          q_mode="gaussian", planted=0.0, steps=3),
+], ids=lambda w: w.name)
+def test_fused_append_equals_separate_append(wl):
+    """saga_decode_step (append inside the attention kernels) gives the same caches, thresholds, outputs
+    and index lists, bit for bit, as saga_kv_append followed by saga_decode_attn."""
+    inp = workload.make_layer(wl, 0, device="cuda", steps=wl.steps)
+    l_cap = wl.l_kv + wl.steps
+    n_top = wl.n_for_kernel(l_cap)
+    shape = saga.SagaShape.of(wl.batch, wl.h_q, wl.h_k, wl.h_v, wl.d, l_cap)
+    B, hq, hk, hv, d = wl.batch, wl.h_q, wl.h_k, wl.h_v, wl.d
+    runs = []
+    for fused in (False, True):
+        kc = torch.zeros((B, hk, l_cap, d), dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros((B, hv, l_cap, d), dtype=torch.bfloat16, device="cuda")
+        kc[:, :, :wl.l_kv] = inp["K0"]
+        vc[:, :, :wl.l_kv] = inp["V0"]
+        tau = torch.zeros((B, hq), dtype=torch.float32, device="cuda")
+        ws = saga.alloc_workspace(shape, "cuda")
+        outs, idxs = [], []
+        for t in range(wl.steps):
+            L = wl.l_kv + t + 1
+            out = torch.zeros((B, hq, d), dtype=torch.float32, device="cuda")
+            cnt = torch.zeros((B, hq), dtype=torch.int32, device="cuda")
+            idx = torch.zeros((B, hq, l_cap), dtype=torch.int32, device="cuda")
+            if fused:
+                saga.saga_decode_step(shape, inp["q"][t], inp["k_new"][t], inp["v_new"][t], kc, vc, L, n_top,
+                                      wl.refresh, t, tau, out, ws, sel_count=cnt, sel_idx=idx)
+            else:
+                saga.saga_kv_append(shape, kc, vc, inp["k_new"][t], inp["v_new"][t], L - 1)
+                saga.saga_decode_attn(shape, inp["q"][t], kc, vc, L, n_top, wl.refresh, t, tau, out, ws,
+                                      sel_count=cnt, sel_idx=idx)
+            outs.append((out, tau.clone(), cnt))
+            idxs.append(idx)
+        torch.cuda.synchronize()
+        runs.append((kc, vc, outs, idxs))
+    (k0, v0, o0, i0), (k1, v1, o1, i1) = runs
+    assert torch.equal(k0, k1) and torch.equal(v0, v1)
+    for t in range(wl.steps):
+        for a, b in zip(o0[t], o1[t]):
+            assert torch.equal(a, b), f"step {t}"
+        c = o0[t][2]
+        for bb in range(B):
+            for j in range(hq):
+                n = int(c[bb, j])
+                assert torch.equal(i0[t][bb, j, :n], i1[t][bb, j, :n])
+
+
+def test_plain_stream_order_matches():
+    """With programmatic dependent launch turned off (SAGA_PDL=0) the path still matches the oracle and
+    gives the same bits as with it on."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import sys, torch; sys.path.insert(0, %r)\n"
+        "from tests import gpu_harness; from tests.test_gpu_parity import small\n"
+        "wl = small('pdl', h_q=12, h_k=1, h_v=4, d=128, l_kv=3001, n_top=70, refresh=3, steps=6)\n"
+        "_, s = gpu_harness.run_parity(wl, wl.steps, graphs=True)\n"
+        "torch.save({'out': s.out.cpu(), 'tau': s.tau.cpu()}, sys.argv[1])\n" % root)
+    import tempfile
+    res = {}
+    with tempfile.TemporaryDirectory() as tmp:
+        for flag in ("0", "1"):
+            path = os.path.join(tmp, f"pdl_{flag}.pt")
+            env = dict(os.environ, SAGA_PDL=flag)
+            r = subprocess.run([sys.executable, "-c", code, path], env=env, cwd=root, capture_output=True,
+                               text=True, timeout=600)
+            assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+            res[flag] = torch.load(path)
+    assert torch.equal(res["0"]["out"], res["1"]["out"]) and torch.equal(res["0"]["tau"], res["1"]["tau"])
