@@ -86,52 +86,73 @@ def load_traffic(workload_name):
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle reasons sampled during the timed region."""
+    """SM clock and clock-event reasons sampled during the timed region.
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    Polls NVML from a thread every `period` seconds, plus one sample when it
+    starts and one when it stops, so even a timed region of a few ms is
+    covered.  Reads only; changes no setting.  Falls back to nvidia-smi when
+    the NVML binding is missing.
+    """
 
-    def __init__(self, index):
-        self.index = index
-        self.samples = []
-        self.proc = None
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20), ("hw_thermal_slowdown", 0x40),
+               ("sw_power_cap", 0x4))
+
+    def __init__(self, device_index, period=0.002):
+        self.device_index = device_index
+        self.period = period
+        self.samples = []  # (sm_mhz, max_mhz, reason_bits)
+        self._stop = threading.Event()
         self.thread = None
+        self.handle = None
+        self.nvml = None
+
+    def _open(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device_index)
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.nvml = pynvml
+
+    def _sample(self):
+        n = self.nvml
+        sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+        mx = n.nvmlDeviceGetMaxClockInfo(self.handle, n.NVML_CLOCK_SM)
+        get_reasons = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            n.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.samples.append((sm, mx, int(get_reasons(self.handle))))
+
+    def _loop(self):
+        while not self._stop.wait(self.period):
+            try:
+                self._sample()
+            except Exception:  # noqa: BLE001
+                return
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._open()
+            self._sample()
         except Exception:  # noqa: BLE001
-            self.proc = None
+            self.handle = None
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread = threading.Thread(target=self._loop, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) == 7:
-                self.samples.append(parts)
-
     def stop(self):
-        if self.proc is None:
+        if self.handle is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:  # noqa: BLE001
-            self.proc.kill()
+        self._stop.set()
         self.thread.join(timeout=2)
-        if not self.samples:
-            return None
-        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
-        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[3 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.samples)}
+        try:
+            self._sample()
+        except Exception:  # noqa: BLE001
+            pass
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({name for _, _, bits in self.samples for name, bit in self.REASONS if bits & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
 
 
 def oracle_threads():
@@ -285,7 +306,7 @@ def run_saga(args, wl, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    sampler = ClockSampler(local_rank)
+    sampler = ClockSampler(dev.index if dev.index is not None else local_rank)
     sampler.start()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     bytes_timed = 0

@@ -678,8 +678,8 @@ __global__ void __launch_bounds__(192, 1)
 
   // ---------------------------------------------------------------- setup before the dependency wait
   // Nothing used here is written by a preceding kernel: barriers, TMEM, the
-  // tensor maps, and an L2 prefetch of the first key tiles this split can
-  // cover whatever the length (a prefetch moves no values, so it races with
+  // tensor maps, and an L2 prefetch of the key rows this split can cover
+  // whatever the length (a prefetch moves no values, so it races with
   // nothing).
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -697,7 +697,11 @@ __global__ void __launch_bounds__(192, 1)
     tma_prefetch_desc(&tmap_part);
     int pst, pcap;
     split_cap_range(p.seq_len, p.nsplit, s, p.l_cap, &pst, &pcap);
-    const int pend = min(pcap, pst + NSTAGE * kTile);
+    // as much of the split as fits the grid's share of 48 MB of L2 (the
+    // previous kernel's tail leaves DRAM idle; more would evict itself)
+    const long long ncta = (long long)gridDim.x * gridDim.y * gridDim.z;
+    const int cap_rows = max(kTile, (int)(((48ll << 20) / ncta) / (D * 2)) / kTile * kTile);
+    const int pend = min(pcap, pst + cap_rows);
     const uint16_t* kb = p.k_cache + (size_t)row_base * D;
     for (int r = pst; r < pend; r += kTile) prefetch_l2_bulk(kb + (size_t)r * D, (uint32_t)(min(kTile, pend - r) * D * 2));
   }
