@@ -441,7 +441,7 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     args = ap.parse_args()
     from long_context_decoding_saga_b200 import workload
-    wl = workload.CONFIGS[args.workload]
+    wl = workload.by_name(args.workload)
     if args.layers > 0:
         wl = wl.with_(layers=args.layers)
 

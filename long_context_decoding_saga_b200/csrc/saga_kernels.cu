@@ -103,6 +103,11 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
 template <int NP>
 __host__ __device__ constexpr uint32_t tmem_cols() { return (2 * NP <= 32) ? 32u : (2 * NP <= 64) ? 64u : 128u; }
 
+// N of the scoring MMA: the group's query heads padded to the instruction's
+// minimum of 16 (padding rows of q are zero; their columns are not read).
+template <int NP>
+__host__ __device__ constexpr int mma_n() { return NP < 16 ? 16 : NP; }
+
 // ============================================================================ epilogue
 // Each of the four epilogue warps owns 32 token rows of every tile (its TMEM
 // lane quarter) and keeps its own online softmax, so no barrier couples the
@@ -573,7 +578,7 @@ template <int D, int NP, bool UMMA>
 struct SplitSmem {
   static constexpr int NATOM = D / 64;
   static constexpr int STAGE_BYTES = kTile * D * 2;
-  static constexpr int QBYTES = UMMA ? NATOM * NP * 128 : NP * D * 4;
+  static constexpr int QBYTES = UMMA ? NATOM * mma_n<NP>() * 128 : NP * D * 4;
   static constexpr int QPAD = ((QBYTES + 1023) / 1024) * 1024;
   static constexpr int EPI_BYTES = ((int)sizeof(EpiShared<NP>) + 127) / 128 * 128;
   static constexpr int VST_BYTES = 4 * 2 * vstage_warp_bytes<NP>();
@@ -653,8 +658,9 @@ __global__ void __launch_bounds__(192, 1)
   constexpr int NATOM = SM::NATOM;
   constexpr int NSTAGE = SM::NSTAGE;
   constexpr int STAGE_BYTES = SM::STAGE_BYTES;
-  constexpr uint32_t TMEM_COLS = tmem_cols<NP>();
-  constexpr uint32_t IDESC = umma_idesc_bf16(128, NP < 16 ? 16 : NP);
+  constexpr int NPM = mma_n<NP>();
+  constexpr uint32_t TMEM_COLS = tmem_cols<NPM>();
+  constexpr uint32_t IDESC = umma_idesc_bf16(128, NPM);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -715,7 +721,7 @@ __global__ void __launch_bounds__(192, 1)
   // ---------------------------------------------------------------- setup after it
   // The global reads of this setup (q, the thresholds, the length) are issued
   // back to back so that their latencies overlap.
-  constexpr int QCH = UMMA ? NATOM * NP * 8 : NP * D / 8;  // 16-byte chunks of the group's q (padded heads)
+  constexpr int QCH = UMMA ? NATOM * NPM * 8 : NP * D / 8;  // 16-byte chunks of the group's q (padded heads)
   constexpr int QV = (QCH + kEpiThreads - 1) / kEpiThreads;
   const int eth = threadIdx.x - 64;  // epilogue thread (warps 2..5)
   uint4 qv[QV];
@@ -726,8 +732,8 @@ __global__ void __launch_bounds__(192, 1)
       const int i = eth + k * kEpiThreads;
       int n, col;
       if (UMMA) {
-        n = (i / 8) % NP;
-        col = (i / (NP * 8)) * 64 + (i % 8) * 8;
+        n = (i / 8) % NPM;
+        col = (i / (NPM * 8)) * 64 + (i % 8) * 8;
       } else {
         n = i / (D / 8);
         col = (i % (D / 8)) * 8;
@@ -761,8 +767,8 @@ __global__ void __launch_bounds__(192, 1)
       if (i < QCH) {
         if (UMMA) {
           // q as the K-major B operand in the 128-byte swizzle layout; rows >= G are zero
-          const int a = i / (NP * 8), n = (i / 8) % NP, c = i % 8;
-          *reinterpret_cast<uint4*>(qsm + a * NP * 128 + n * 128 + ((c ^ (n & 7)) << 4)) = qv[k];
+          const int a = i / (NPM * 8), n = (i / 8) % NPM, c = i % 8;
+          *reinterpret_cast<uint4*>(qsm + a * NPM * 128 + n * 128 + ((c ^ (n & 7)) << 4)) = qv[k];
         } else {
           float* qf = reinterpret_cast<float*>(qsm) + (i / (D / 8)) * D + (i % (D / 8)) * 8;
           *reinterpret_cast<float4*>(qf) = make_float4(bf16_lo(qv[k].x), bf16_hi(qv[k].x), bf16_lo(qv[k].y),
@@ -803,11 +809,11 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const uint32_t a0 = smem_u32(kst + stage * STAGE_BYTES);
         const uint32_t b0 = smem_u32(qsm);
-        const uint32_t d_tmem = tmem_base + abuf * NP;
+        const uint32_t d_tmem = tmem_base + abuf * NPM;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t aa = a0 + (k >> 2) * 16384 + (k & 3) * 32;
-          const uint32_t bb = b0 + (k >> 2) * NP * 128 + (k & 3) * 32;
+          const uint32_t bb = b0 + (k >> 2) * NPM * 128 + (k & 3) * 32;
           umma_bf16(d_tmem, umma_sdesc_sw128(aa), umma_sdesc_sw128(bb), IDESC, k > 0 ? 1u : 0u);
         }
         umma_commit(&empty[stage]);
@@ -840,9 +846,16 @@ __global__ void __launch_bounds__(192, 1)
         if (counting) ok = named_bar_and(1, kEpiThreads, ok);  // warps leave together (barriers below)
         if (!ok) break;
         tc_fence_after();
-        const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * NP);
+        const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * NPM);
+        if constexpr (NP >= 16) {
 #pragma unroll
-        for (int i = 0; i < NP / 16; ++i) tmem_ld16(taddr + 16 * i, sc + 16 * i);
+          for (int i = 0; i < NP / 16; ++i) tmem_ld16(taddr + 16 * i, sc + 16 * i);
+        } else {
+          float all[16];
+          tmem_ld16(taddr, all);
+#pragma unroll
+          for (int i = 0; i < NP; ++i) sc[i] = all[i];
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acce[abuf]);
@@ -1331,7 +1344,7 @@ template <int D>
 static cudaError_t dispatch_np(int NP, bool dump, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p,
                                dim3 g, cudaStream_t st, int* occ) {
   switch (NP) {
-    case 4: return dump ? run_split<D, 4, false, true>(tf, tp, p, g, st, occ) : run_split<D, 4, false, false>(tf, tp, p, g, st, occ);
+    case 4: return dump ? run_split<D, 4, true, true>(tf, tp, p, g, st, occ) : run_split<D, 4, true, false>(tf, tp, p, g, st, occ);
     case 16: return dump ? run_split<D, 16, true, true>(tf, tp, p, g, st, occ) : run_split<D, 16, true, false>(tf, tp, p, g, st, occ);
     case 32: return dump ? run_split<D, 32, true, true>(tf, tp, p, g, st, occ) : run_split<D, 32, true, false>(tf, tp, p, g, st, occ);
     case 64:

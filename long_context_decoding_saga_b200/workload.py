@@ -108,6 +108,18 @@ def sweep_point(l_kv: int, batch: int, h_k: int, n_top: int, refresh: int) -> Wo
                     max(2 * refresh, 16), n_top, refresh, 0.01, "planted_mean", seed)
 
 
+def by_name(name: str) -> Workload:
+    """A configuration by name, or a sweep point by its name
+    (sweep_l<l_kv>_b<batch>_hk<h_k>_n<N>_r<R>)."""
+    if name in CONFIGS:
+        return CONFIGS[name]
+    import re
+    m = re.fullmatch(r"sweep_l(\d+)_b(\d+)_hk(\d+)_n(\d+)_r(\d+)", name)
+    if m is None:
+        raise KeyError(f"unknown workload {name!r}")
+    return sweep_point(*(int(x) for x in m.groups()))
+
+
 def sweep_points():
     for l_kv in SWEEP_L_KV:
         for b in SWEEP_BATCH:
