@@ -78,7 +78,7 @@ int device_sms(int* sms) {
   return SAGA_OK;
 }
 
-int np_for_group(int G) { return G <= 4 ? 4 : G <= 16 ? 16 : G <= 32 ? 32 : 64; }
+int np_for_group(int G) { return G <= 4 ? 4 : G <= 8 ? 8 : G <= 16 ? 16 : G <= 32 ? 32 : 64; }
 
 int validate_shape(const saga_shape* s) {
   if (s == nullptr) return fail(SAGA_ERR_ARG, "shape is NULL");

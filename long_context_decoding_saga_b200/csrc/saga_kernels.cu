@@ -573,6 +573,7 @@ __device__ __forceinline__ void tail_merge(EpiShared<NP>& es, float* mrg, const 
 
 // ============================================================================ split kernel
 constexpr int kSmemLimit = 232448;  // dynamic shared memory one CTA may use on sm_100
+constexpr int kSmemHalf = 115712;   // per CTA when two CTAs share an SM (233472 / 2 minus the 1 KB reserve)
 
 template <int D, int NP, bool UMMA>
 struct SplitSmem {
@@ -583,11 +584,16 @@ struct SplitSmem {
   static constexpr int EPI_BYTES = ((int)sizeof(EpiShared<NP>) + 127) / 128 * 128;
   static constexpr int VST_BYTES = 4 * 2 * vstage_warp_bytes<NP>();
   // key-tile ring: 4 tiles of 32 KB at d = 128 or 6 of 16 KB at d = 64 cover
-  // the load latency; fewer where the epilogue's buffers leave less room
+  // the load latency; fewer where the epilogue's buffers leave less room.
+  // When 4 tiles still fit in half of the SM's shared memory, the ring takes
+  // 4 so that two CTAs share an SM (twice the epilogue warps to hide latency,
+  // as many bytes in flight).
   static constexpr int FIXED = QPAD + EPI_BYTES + VST_BYTES + 2 * 8 * 8 + 5 * 8 + 16 + 1024;
   static constexpr int NSTAGE_MAX = D == 128 ? 4 : 6;
   static constexpr int NSTAGE_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
-  static constexpr int NSTAGE = NSTAGE_FIT < NSTAGE_MAX ? NSTAGE_FIT : NSTAGE_MAX;
+  static constexpr int NSTAGE_HALF = (kSmemHalf - FIXED) / STAGE_BYTES;
+  static constexpr int NSTAGE = NSTAGE_HALF >= 4 ? 4 : (NSTAGE_FIT < NSTAGE_MAX ? NSTAGE_FIT : NSTAGE_MAX);
+  static constexpr int CTAS_PER_SM = NSTAGE_HALF >= 4 ? 2 : 1;  // also bounds the registers (<= 170 for two)
   static_assert(NSTAGE >= 3, "key-tile ring too shallow");
   static constexpr int Q_OFF = NSTAGE * STAGE_BYTES;
   static constexpr int EPI_OFF = Q_OFF + QPAD;
@@ -651,7 +657,7 @@ __device__ __forceinline__ void issue_key_tile(int t, int start, int end, int ro
 // Warp roles: 0 = TMA producer, 1 = tcgen05 MMA issuer (idle on the
 // CUDA-core path), 2..5 = epilogue (one thread per token row of a tile).
 template <int D, int NP, bool UMMA, bool DUMP>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     saga_split_kernel(const __grid_constant__ CUtensorMap tmap_full, const __grid_constant__ CUtensorMap tmap_part,
                       const SplitParams p) {
   using SM = SplitSmem<D, NP, UMMA>;
@@ -1345,6 +1351,7 @@ static cudaError_t dispatch_np(int NP, bool dump, const CUtensorMap& tf, const C
                                dim3 g, cudaStream_t st, int* occ) {
   switch (NP) {
     case 4: return dump ? run_split<D, 4, true, true>(tf, tp, p, g, st, occ) : run_split<D, 4, true, false>(tf, tp, p, g, st, occ);
+    case 8: return dump ? run_split<D, 8, true, true>(tf, tp, p, g, st, occ) : run_split<D, 8, true, false>(tf, tp, p, g, st, occ);
     case 16: return dump ? run_split<D, 16, true, true>(tf, tp, p, g, st, occ) : run_split<D, 16, true, false>(tf, tp, p, g, st, occ);
     case 32: return dump ? run_split<D, 32, true, true>(tf, tp, p, g, st, occ) : run_split<D, 32, true, false>(tf, tp, p, g, st, occ);
     case 64:
@@ -1380,8 +1387,8 @@ static cudaError_t run_from_scores(const SplitParams& p, dim3 grid, cudaStream_t
 cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, cudaStream_t st) {
 #define SAGA_FS(DD, NN) \
   if (D == DD && NP == NN) return run_from_scores<DD, NN>(p, grid, st);
-  SAGA_FS(64, 4) SAGA_FS(64, 16) SAGA_FS(64, 32) SAGA_FS(64, 64)
-  SAGA_FS(128, 4) SAGA_FS(128, 16) SAGA_FS(128, 32)
+  SAGA_FS(64, 4) SAGA_FS(64, 8) SAGA_FS(64, 16) SAGA_FS(64, 32) SAGA_FS(64, 64)
+  SAGA_FS(128, 4) SAGA_FS(128, 8) SAGA_FS(128, 16) SAGA_FS(128, 32)
 #undef SAGA_FS
   return cudaErrorInvalidValue;
 }
