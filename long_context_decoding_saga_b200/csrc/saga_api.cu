@@ -244,7 +244,13 @@ int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, int
   cudaError_t e = launch_split(s->d, NP, mode, tf, tp, dummy, dim3(1), nullptr, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
   if (occ < 1) return fail(SAGA_ERR_UNSUPPORTED, "split kernel does not fit on an SM");
-  *S = choose_splits(s->batch * s->h_k, seq_len, occ * pr.sms, pr.ws.s_cap);
+  // A small step (at most 16 key tiles per SM) is latency-bound: one split
+  // per SM, which leaves a second CTA slot to the next call's kernel (it
+  // starts its setup and L2 prefetch early).  Larger steps fill every slot.
+  const int groups = s->batch * s->h_k;
+  const long long tiles = (long long)groups * ((seq_len + kTile - 1) / kTile);
+  const int slots = (occ > 1 && tiles <= 16ll * pr.sms) ? pr.sms : occ * pr.sms;
+  *S = choose_splits(groups, seq_len, slots, pr.ws.s_cap);
   return SAGA_OK;
 }
 

@@ -137,9 +137,10 @@ struct EpiShared {
   int tail_n[4][2];           // ... and their row counts
 };
 
-// Bytes of value rows each warp stages per list buffer.
-template <int NP>
-__host__ __device__ constexpr int vstage_warp_bytes() { return NP >= 64 ? 2048 : 4096; }
+// Bytes of value rows each warp stages per list buffer (2 KB at d = 64 with
+// 16 heads per group, which lets two CTAs share an SM).
+template <int D, int NP>
+__host__ __device__ constexpr int vstage_warp_bytes() { return (NP >= 64 || (D == 64 && NP == 16)) ? 2048 : 4096; }
 
 struct EpiArgs {
   const uint16_t* vgroup;  // V of the group's first value head, batch b
@@ -182,7 +183,7 @@ __device__ __forceinline__ EpiArgs epi_args(const SplitParams& p, int b, int j0)
   ea.G = p.G;
   ea.hpv = p.hpv;
   ea.nvh = p.nvh;
-  ea.rcapw = min(kBatch, vstage_warp_bytes<NP>() / (p.nvh * D * 2));
+  ea.rcapw = min(kBatch, vstage_warp_bytes<D, NP>() / (p.nvh * D * 2));
   ea.cpr = p.nvh * D / 8;
   ea.hmul = (65536 + p.hpv - 1) / p.hpv;
   return ea;
@@ -449,7 +450,7 @@ __device__ __forceinline__ void tail_merge(EpiShared<NP>& es, float* mrg, const 
                                            bool drop_lists) {
   constexpr int DPL = WarpAcc<D, NP>::DPL;
   constexpr int REG = NP * (D + 2);
-  constexpr int VWE = vstage_warp_bytes<NP>();  // elements of one warp's staging area (two buffers)
+  constexpr int VWE = vstage_warp_bytes<D, NP>();  // elements of one warp's staging area (two buffers)
   float* mine = mrg + q * REG;                  // m[NP], l[NP], o[NP][D]
   if (lane == 0) {
 #pragma unroll
@@ -582,19 +583,21 @@ struct SplitSmem {
   static constexpr int QBYTES = UMMA ? NATOM * mma_n<NP>() * 128 : NP * D * 4;
   static constexpr int QPAD = ((QBYTES + 1023) / 1024) * 1024;
   static constexpr int EPI_BYTES = ((int)sizeof(EpiShared<NP>) + 127) / 128 * 128;
-  static constexpr int VST_BYTES = 4 * 2 * vstage_warp_bytes<NP>();
+  static constexpr int VST_BYTES = 4 * 2 * vstage_warp_bytes<D, NP>();
   // key-tile ring: 4 tiles of 32 KB at d = 128 or 6 of 16 KB at d = 64 cover
   // the load latency; fewer where the epilogue's buffers leave less room.
-  // When 4 tiles still fit in half of the SM's shared memory, the ring takes
-  // 4 so that two CTAs share an SM (twice the epilogue warps to hide latency,
-  // as many bytes in flight).
+  // At d = 64, when 4 tiles of 16 KB fit in half of the SM's shared memory,
+  // the ring takes 4 so that two CTAs share an SM (twice the epilogue warps
+  // to hide latency, as many bytes in flight).
   static constexpr int FIXED = QPAD + EPI_BYTES + VST_BYTES + 2 * 8 * 8 + 5 * 8 + 16 + 1024;
   static constexpr int NSTAGE_MAX = D == 128 ? 4 : 6;
   static constexpr int NSTAGE_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
   static constexpr int NSTAGE_HALF = (kSmemHalf - FIXED) / STAGE_BYTES;
-  static constexpr int NSTAGE = NSTAGE_HALF >= 4 ? 4 : (NSTAGE_FIT < NSTAGE_MAX ? NSTAGE_FIT : NSTAGE_MAX);
-  static constexpr int CTAS_PER_SM = NSTAGE_HALF >= 4 ? 2 : 1;  // also bounds the registers (<= 170 for two)
-  static_assert(NSTAGE >= 3, "key-tile ring too shallow");
+  static constexpr bool TWO = D == 64 && NSTAGE_HALF >= 4;  // 2 x 32 KB at d = 128 measured slower
+  static constexpr int NSTAGE_TWO = NSTAGE_HALF < 4 ? NSTAGE_HALF : 4;
+  static constexpr int NSTAGE = TWO ? NSTAGE_TWO : (NSTAGE_FIT < NSTAGE_MAX ? NSTAGE_FIT : NSTAGE_MAX);
+  static constexpr int CTAS_PER_SM = TWO ? 2 : 1;  // also bounds the registers (<= 170 for two)
+  static_assert(NSTAGE >= 3 || (TWO && NSTAGE >= 2), "key-tile ring too shallow");
   static constexpr int Q_OFF = NSTAGE * STAGE_BYTES;
   static constexpr int EPI_OFF = Q_OFF + QPAD;
   static constexpr int VST_OFF = EPI_OFF + EPI_BYTES;
@@ -837,7 +840,7 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     const int erow = 32 * q + lane;
     const bool counting = p.want_counts != 0;
     const EpiArgs ea = epi_args<D, NP>(p, b, j0);
-    uint16_t* vstage_w = vstage + (size_t)q * 2 * (vstage_warp_bytes<NP>() / 2);
+    uint16_t* vstage_w = vstage + (size_t)q * 2 * (vstage_warp_bytes<D, NP>() / 2);
     WarpAcc<D, NP> acc;
     acc.init();
     ListState ls{0, 0, -1, 0};
@@ -966,7 +969,7 @@ __device__ __forceinline__ void load_scores(float (&dst)[NP], const float* srow,
 template <int D, int NP>
 struct FromScoresSmem {
   static constexpr int VST_OFF = ((int)sizeof(EpiShared<NP>) + 127) / 128 * 128;
-  static constexpr int MRG_OFF = VST_OFF + 4 * 2 * vstage_warp_bytes<NP>();
+  static constexpr int MRG_OFF = VST_OFF + 4 * 2 * vstage_warp_bytes<D, NP>();
   static constexpr int BYTES = MRG_OFF + merge_floats<D, NP>() * 4;
 };
 
@@ -990,7 +993,7 @@ __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const Spl
 
   epi_setup<NP>(es, et, p, load_tau<NP>(et, p, b, j0, true));
   const EpiArgs ea = epi_args<D, NP>(p, b, j0);
-  uint16_t* vstage_w = vstage + (size_t)q * 2 * (vstage_warp_bytes<NP>() / 2);
+  uint16_t* vstage_w = vstage + (size_t)q * 2 * (vstage_warp_bytes<D, NP>() / 2);
   WarpAcc<D, NP> acc;
   acc.init();
   ListState ls{0, 0, -1, 0};
