@@ -224,6 +224,35 @@ __device__ __forceinline__ uint64_t keep_mask(const EpiShared<NP>& es, const flo
   return valid ? keep : 0ull;
 }
 
+// One staged row of a list buffer into the warp's accumulators: every value
+// head of the group is in shared memory, so the loads need no branch (heads
+// that do not keep the row have weight 0).
+template <int D, int NP>
+__device__ __forceinline__ void staged_row(WarpAcc<D, NP>& acc, const EpiArgs& ea, const WarpList<NP>& li, int r,
+                                           const uint16_t* vbuf) {
+  constexpr int DPL = WarpAcc<D, NP>::DPL;
+  float w[NP];
+#pragma unroll
+  for (int j4 = 0; j4 < NP / 4; ++j4) {
+    const float4 v4 = *reinterpret_cast<const float4*>(&li.sc[r][4 * j4]);
+    w[4 * j4 + 0] = v4.x;
+    w[4 * j4 + 1] = v4.y;
+    w[4 * j4 + 2] = v4.z;
+    w[4 * j4 + 3] = v4.w;
+  }
+  const uint16_t* vrow = vbuf + (size_t)r * ea.nvh * D;
+#pragma unroll
+  for (int jl = 0; jl < NP; ++jl) {
+    if (jl < ea.G) {
+      float v[DPL];
+      load_bf16<DPL>(vrow + ((jl * ea.hmul) >> 16) * D, v);
+      acc.l[jl] += w[jl];
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc.o[jl][e] = fmaf(w[jl], v[e], acc.o[jl][e]);
+    }
+  }
+}
+
 // Softmax and value sum over list buffer bi (n rows) of this warp.
 template <int D, int NP>
 __device__ __forceinline__ void reduce_batch(EpiShared<NP>& es, WarpAcc<D, NP>& acc, const EpiArgs& ea, int q,
@@ -278,7 +307,18 @@ __device__ __forceinline__ void reduce_batch(EpiShared<NP>& es, WarpAcc<D, NP>& 
     }
   }
   __syncwarp();
-  for (int r = 0; r < n; ++r) {
+  // staged rows in groups (their loads are independent, so a group's are in
+  // flight together), then any rows that did not fit the staging buffer
+  const uint16_t* vbuf = vstage_w + (size_t)bi * ea.rcapw * ea.nvh * D + lane * DPL;
+  const int ns = min(n, ea.rcapw);
+  constexpr int RU = NP <= 8 ? 4 : (NP == 16 ? 2 : 1);
+  int r = 0;
+  for (; r + RU <= ns; r += RU) {
+#pragma unroll
+    for (int k = 0; k < RU; ++k) staged_row<D, NP>(acc, ea, li, r + k, vbuf);
+  }
+  for (; r < ns; ++r) staged_row<D, NP>(acc, ea, li, r, vbuf);
+  for (; r < n; ++r) {
     float w[NP];
 #pragma unroll
     for (int j4 = 0; j4 < NP / 4; ++j4) {
@@ -288,53 +328,15 @@ __device__ __forceinline__ void reduce_batch(EpiShared<NP>& es, WarpAcc<D, NP>& 
       w[4 * j4 + 2] = v4.z;
       w[4 * j4 + 3] = v4.w;
     }
-    if (r < ea.rcapw) {
-      // staged row: every value head of the group is in shared memory, so the
-      // loads need no branch (heads that do not keep the row have w = 0)
-      const uint16_t* vrow = vstage_w + ((size_t)bi * ea.rcapw + r) * ea.nvh * D + lane * DPL;
+    const uint16_t* vrow = ea.vgroup + (size_t)li.tok[r] * D + lane * DPL;
 #pragma unroll
-      for (int jl = 0; jl < NP; ++jl) {
-        if (jl < ea.G) {
-          const uint16_t* src = vrow + ((jl * ea.hmul) >> 16) * D;
-          float v[DPL];
-          if constexpr (DPL == 4) {
-            const uint2 raw = *reinterpret_cast<const uint2*>(src);
-            v[0] = bf16_lo(raw.x);
-            v[1] = bf16_hi(raw.x);
-            v[2] = bf16_lo(raw.y);
-            v[3] = bf16_hi(raw.y);
-          } else {
-            const uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
-            v[0] = bf16_lo(raw);
-            v[1] = bf16_hi(raw);
-          }
-          acc.l[jl] += w[jl];
+    for (int jl = 0; jl < NP; ++jl) {
+      if (w[jl] != 0.f) {  // same value in every lane
+        float v[DPL];
+        load_bf16_global<DPL>(vrow + (size_t)((jl * ea.hmul) >> 16) * ea.l_cap * D, v);
+        acc.l[jl] += w[jl];
 #pragma unroll
-          for (int e = 0; e < DPL; ++e) acc.o[jl][e] = fmaf(w[jl], v[e], acc.o[jl][e]);
-        }
-      }
-    } else {
-      const uint16_t* vrow = ea.vgroup + (size_t)li.tok[r] * D + lane * DPL;
-#pragma unroll
-      for (int jl = 0; jl < NP; ++jl) {
-        if (w[jl] != 0.f) {  // same value in every lane
-          const uint16_t* src = vrow + (size_t)((jl * ea.hmul) >> 16) * ea.l_cap * D;
-          float v[DPL];
-          if constexpr (DPL == 4) {
-            const uint2 raw = __ldg(reinterpret_cast<const uint2*>(src));
-            v[0] = bf16_lo(raw.x);
-            v[1] = bf16_hi(raw.x);
-            v[2] = bf16_lo(raw.y);
-            v[3] = bf16_hi(raw.y);
-          } else {
-            const uint32_t raw = __ldg(reinterpret_cast<const uint32_t*>(src));
-            v[0] = bf16_lo(raw);
-            v[1] = bf16_hi(raw);
-          }
-          acc.l[jl] += w[jl];
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) acc.o[jl][e] = fmaf(w[jl], v[e], acc.o[jl][e]);
-        }
+        for (int e = 0; e < DPL; ++e) acc.o[jl][e] = fmaf(w[jl], v[e], acc.o[jl][e]);
       }
     }
   }
@@ -385,6 +387,21 @@ __device__ __forceinline__ void append_rows(EpiShared<NP>& es, WarpAcc<D, NP>& a
   }
   cp_async_commit();
   ls.n = r1;
+}
+
+// Before the tail: a warp left with many unreduced rows reduces them with
+// the batch reduction (columns across lanes), which beats the tail's
+// row-pool pass once there are more than a few rows.
+template <int D, int NP>
+__device__ __forceinline__ void flush_large_lists(EpiShared<NP>& es, WarpAcc<D, NP>& acc, const EpiArgs& ea,
+                                                  ListState& ls, int q, int lane, const uint16_t* vstage_w) {
+  const int rows = ls.n + (ls.pend >= 0 ? ls.npend : 0);
+  if (rows <= 8) return;  // warp-uniform
+  // the newest cp.async group belongs to the current buffer only if it holds rows
+  if (ls.pend >= 0) reduce_batch<D, NP>(es, acc, ea, q, lane, ls.pend, ls.npend, vstage_w, ls.n > 0);
+  if (ls.n > 0) reduce_batch<D, NP>(es, acc, ea, q, lane, ls.cur, ls.n, vstage_w, false);
+  ls.pend = -1;
+  ls.n = 0;
 }
 
 // Counting mode (kept counts and ascending index lists requested): the four
@@ -923,6 +940,7 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
       }
     }
     if (!DUMP) {
+      if (t == ntiles) flush_large_lists<D, NP>(es, acc, ea, ls, q, lane, vstage_w);
       // the warps' states go into the key ring: with tcgen05 it is free once a
       // warp has seen the last tile's scores (every MMA and copy is done); on
       // the CUDA-core path the other warps may still be reading it
@@ -1010,6 +1028,7 @@ __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const Spl
     const int tok = start + t * kTile + et;
     tile_epilogue<D, NP>(es, acc, ea, ls, q, lane, et, sc, tok, tok < end, counting, p, b, j0, start, vstage_w);
   }
+  flush_large_lists<D, NP>(es, acc, ea, ls, q, lane, vstage_w);
   tail_merge<D, NP>(es, mrg, acc, ls, ea, vstage, q, lane, et, p, b, j0, s, false);
 }
 
