@@ -108,6 +108,11 @@ __host__ __device__ constexpr uint32_t tmem_cols() { return (2 * NP <= 32) ? 32u
 template <int NP>
 __host__ __device__ constexpr int mma_n() { return NP < 16 ? 16 : NP; }
 
+// TMEM accumulator buffers: the MMA may run this many tiles ahead of the
+// epilogue (4 while they fit in 128 columns).
+template <int NP>
+__host__ __device__ constexpr int acc_bufs() { return mma_n<NP>() <= 32 ? 4 : 2; }
+
 // ============================================================================ epilogue
 // Each of the four epilogue warps owns 32 token rows of every tile (its TMEM
 // lane quarter) and keeps its own online softmax, so no barrier couples the
@@ -606,8 +611,8 @@ struct SplitSmem {
   // At d = 64, when 4 tiles of 16 KB fit in half of the SM's shared memory,
   // the ring takes 4 so that two CTAs share an SM (twice the epilogue warps
   // to hide latency, as many bytes in flight).
-  static constexpr int FIXED = QPAD + EPI_BYTES + VST_BYTES + 2 * 8 * 8 + 5 * 8 + 16 + 1024;
   static constexpr int NSTAGE_MAX = D == 128 ? 4 : 6;
+  static constexpr int FIXED = QPAD + EPI_BYTES + VST_BYTES + (2 * NSTAGE_MAX + 2 * acc_bufs<NP>() + 1) * 8 + 16 + 1024;
   static constexpr int NSTAGE_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
   static constexpr int NSTAGE_HALF = (kSmemHalf - FIXED) / STAGE_BYTES;
   static constexpr bool TWO = D == 64 && NSTAGE_HALF >= 4;  // 2 x 32 KB at d = 128 measured slower
@@ -619,11 +624,12 @@ struct SplitSmem {
   static constexpr int EPI_OFF = Q_OFF + QPAD;
   static constexpr int VST_OFF = EPI_OFF + EPI_BYTES;
   static constexpr int BAR_OFF = VST_OFF + VST_BYTES;
-  static constexpr int NBARS = 2 * NSTAGE + 5;
+  static constexpr int NBARS = 2 * NSTAGE + 2 * acc_bufs<NP>() + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
   static_assert(ALLOC <= kSmemLimit, "shared memory over the per-CTA limit");
+  static_assert(!TWO || ALLOC <= kSmemHalf, "two CTAs per SM must fit in half the shared memory");
   static_assert(merge_floats<D, NP>() * 4 <= NSTAGE * STAGE_BYTES, "merge buffer must fit in the key stages");
   static_assert(NP * 256 * 4 <= (int)sizeof(WarpList<NP>) * 8, "dump histogram must fit in the warp lists");
 };
@@ -685,7 +691,8 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
   constexpr int NSTAGE = SM::NSTAGE;
   constexpr int STAGE_BYTES = SM::STAGE_BYTES;
   constexpr int NPM = mma_n<NP>();
-  constexpr uint32_t TMEM_COLS = tmem_cols<NPM>();
+  constexpr int NACC = acc_bufs<NP>();
+  constexpr uint32_t TMEM_COLS = NACC * NPM <= 32 ? 32u : NACC * NPM <= 64 ? 64u : NACC * NPM <= 128 ? 128u : 256u;
   constexpr uint32_t IDESC = umma_idesc_bf16(128, NPM);
 
   extern __shared__ uint8_t smem_raw[];
@@ -698,8 +705,8 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFF);
   uint64_t* empty = full + NSTAGE;
   uint64_t* accf = empty + NSTAGE;
-  uint64_t* acce = accf + 2;
-  uint64_t* fin = acce + 2;
+  uint64_t* acce = accf + NACC;
+  uint64_t* fin = acce + NACC;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::MISC_OFF + 4);
 
@@ -719,7 +726,7 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], UMMA ? 1 : 4);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NACC; ++i) {
       mbar_init(&accf[i], 1);
       mbar_init(&acce[i], 4);
     }
@@ -830,8 +837,8 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
       for (int t = 0; t < ntiles; ++t) {
         const int stage = t % NSTAGE, round = t / NSTAGE;
         if (!mbar_wait(&full[stage], round & 1, abort_flag)) break;
-        const int abuf = t & 1;
-        if (t >= 2 && !mbar_wait(&acce[abuf], ((t >> 1) - 1) & 1, abort_flag)) break;
+        const int abuf = t % NACC;
+        if (t >= NACC && !mbar_wait(&acce[abuf], ((t / NACC) - 1) & 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t a0 = smem_u32(kst + stage * STAGE_BYTES);
         const uint32_t b0 = smem_u32(qsm);
@@ -867,8 +874,8 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
       float sc[NP];
       bool ok;
       if (UMMA) {
-        const int abuf = t & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&accf[abuf], (t >> 1) & 1, abort_flag));
+        const int abuf = t % NACC;
+        ok = __all_sync(0xffffffffu, mbar_wait(&accf[abuf], (t / NACC) & 1, abort_flag));
         if (counting) ok = named_bar_and(1, kEpiThreads, ok);  // warps leave together (barriers below)
         if (!ok) break;
         tc_fence_after();
