@@ -458,9 +458,10 @@ __device__ __forceinline__ void tile_epilogue(EpiShared<NP>& es, WarpAcc<D, NP>&
 // still waiting, unreduced, in their lists, and writes the split's partial.
 // Each warp publishes its state (in mrg: 4 * NP * (D + 2) floats, 16-byte
 // aligned) and its list descriptors.  After one barrier the unreduced rows
-// of all warps form one pool; each warp takes whole heads: its lanes first
-// hold one pool row each (weight, one max reduction per head), then the
-// columns while the rows are accumulated from shuffled weights.
+// of all warps form one pool; each warp takes a block of contiguous heads
+// and works on them together: its lanes first hold one pool row each
+// (weights, one max reduction per head), then the columns while the rows
+// are accumulated from shuffled weights.
 // Deterministic (fixed order in every sum).
 template <int D, int NP>
 __host__ __device__ constexpr int merge_floats() { return 4 * NP * (D + 2); }
@@ -506,89 +507,129 @@ __device__ __forceinline__ void tail_merge(EpiShared<NP>& es, float* mrg, const 
   for (int wk = 0; wk < 8; ++wk) off[wk + 1] = off[wk] + es.tail_n[wk >> 1][wk & 1];
   const int npool = off[8];
   const size_t row0 = (size_t)b * p.h_q + j0;
-  // warp q takes heads q, q+4, ...; lanes hold columns [lane*DPL, lane*DPL+DPL)
-  for (int jl = q; jl < p.G; jl += 4) {
-    const int u = (jl * ea.hmul) >> 16;  // the head's value head within the group
-    float mw[4], M = -INFINITY;
+  // warp q takes the contiguous heads [q*HB, q*HB + HB) (with h_q/h_v query
+  // heads per value head these usually share one value head) and works on
+  // them together: one pass over the pool serves all of them
+  constexpr int NH = (NP + 3) / 4;
+  const int HB = (p.G + 3) / 4;
+  const int h0 = q * HB;
+  float M[NH], mwv[NH][4];
+  int u[NH];
+  bool hv[NH];
+#pragma unroll
+  for (int hh = 0; hh < NH; ++hh) {
+    const int jl = h0 + hh;
+    hv[hh] = hh < HB && jl < p.G;
+    u[hh] = hv[hh] ? (jl * ea.hmul) >> 16 : 0;
+    M[hh] = -INFINITY;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      mw[w] = mrg[w * REG + jl];
-      M = fmaxf(M, mw[w]);
+      mwv[hh][w] = hv[hh] ? mrg[w * REG + jl] : -INFINITY;
+      M[hh] = fmaxf(M[hh], mwv[hh][w]);
     }
-    for (int base = 0; base < npool; base += 32) {  // pool maximum, one row per lane
-      const int k = base + lane;
-      float sc = -INFINITY;
+  }
+  // lane k of a chunk holds pool row base + k: its list, row, keep mask, scores
+  for (int base = 0; base < npool; base += 32) {
+    const int k = base + lane;
+    uint64_t keep = 0ull;
+    int wk = 0, r = k;
+    if (k < npool) {
+#pragma unroll
+      for (int i = 1; i < 8; ++i)
+        if (k >= off[i]) {
+          wk = i;
+          r = k - off[i];
+        }
+      keep = es.list[wk >> 1][es.tail_buf[wk >> 1][wk & 1]].keep[r];
+    }
+    const WarpList<NP>& li = es.list[wk >> 1][es.tail_buf[wk >> 1][wk & 1]];
+#pragma unroll
+    for (int hh = 0; hh < NH; ++hh) {
+      const int jl = h0 + hh;
+      const float sc = (hv[hh] && ((keep >> jl) & 1ull)) ? li.sc[r][jl] : -INFINITY;
+      M[hh] = fmaxf(M[hh], warp_max(sc));
+    }
+  }
+  float o[NH][DPL], lsum[NH];
+#pragma unroll
+  for (int hh = 0; hh < NH; ++hh) {
+    const int jl = h0 + hh;
+    lsum[hh] = 0.f;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) o[hh][e] = 0.f;
+    if (hv[hh] && M[hh] != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float f = (mwv[hh][w] == -INFINITY) ? 0.f : __expf(mwv[hh][w] - M[hh]);
+        lsum[hh] = fmaf(f, mrg[w * REG + NP + jl], lsum[hh]);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) o[hh][e] = fmaf(f, mrg[w * REG + 2 * NP + jl * D + lane * DPL + e], o[hh][e]);
+      }
+    }
+  }
+  for (int base = 0; base < npool; base += 32) {
+    // lane k: its pool row's weights and where its value rows are (shared
+    // memory offset of value head 0 of the group, or -(token + 1) for a row
+    // that was not staged)
+    const int k = base + lane;
+    float wgt[NH];
+    int loc = 0;
+    {
+      uint64_t keep = 0ull;
+      int wk = 0, r = k, bi = 0;
       if (k < npool) {
-        int wk = 0, r = k;
 #pragma unroll
         for (int i = 1; i < 8; ++i)
           if (k >= off[i]) {
             wk = i;
             r = k - off[i];
           }
-        const WarpList<NP>& li = es.list[wk >> 1][es.tail_buf[wk >> 1][wk & 1]];
-        if ((li.keep[r] >> jl) & 1ull) sc = li.sc[r][jl];
+        bi = es.tail_buf[wk >> 1][wk & 1];
+        keep = es.list[wk >> 1][bi].keep[r];
       }
-      M = fmaxf(M, warp_max(sc));
+      const WarpList<NP>& li = es.list[wk >> 1][bi];
+#pragma unroll
+      for (int hh = 0; hh < NH; ++hh) {
+        const int jl = h0 + hh;
+        const bool kept = hv[hh] && ((keep >> jl) & 1ull);
+        wgt[hh] = kept ? __expf(li.sc[r][jl] - M[hh]) : 0.f;
+        lsum[hh] += warp_sum(wgt[hh]);
+      }
+      if (k < npool) loc = r < ea.rcapw ? (wk >> 1) * VWE + (bi * ea.rcapw + r) * ea.nvh * D : -(li.tok[r] + 1);
     }
-    float o[DPL];
-    float lsum = 0.f;
+    const int nrow = min(32, npool - base);
+#pragma unroll 2
+    for (int i = 0; i < nrow; ++i) {
+      const int li_loc = __shfl_sync(0xffffffffu, loc, i);
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) o[e] = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float f = (mw[w] == -INFINITY) ? 0.f : __expf(mw[w] - M);
-        lsum = fmaf(f, mrg[w * REG + NP + jl], lsum);
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) o[e] = fmaf(f, mrg[w * REG + 2 * NP + jl * D + lane * DPL + e], o[e]);
-      }
-      for (int base = 0; base < npool; base += 32) {
-        // lane k: its pool row's weight and where its value row is (shared
-        // memory offset, or -(token + 1) for a row that was not staged)
-        const int k = base + lane;
-        float wgt = 0.f;
-        int loc = 0;
-        if (k < npool) {
-          int wk = 0, r = k;
-#pragma unroll
-          for (int i = 1; i < 8; ++i)
-            if (k >= off[i]) {
-              wk = i;
-              r = k - off[i];
-            }
-          const int bi = es.tail_buf[wk >> 1][wk & 1];
-          const WarpList<NP>& li = es.list[wk >> 1][bi];
-          if ((li.keep[r] >> jl) & 1ull) wgt = __expf(li.sc[r][jl] - M);
-          loc = r < ea.rcapw ? (wk >> 1) * VWE + ((bi * ea.rcapw + r) * ea.nvh + u) * D : -(li.tok[r] + 1);
-        }
-        lsum += warp_sum(wgt);
-        const int nrow = min(32, npool - base);
-#pragma unroll 4
-        for (int i = 0; i < nrow; ++i) {
-          const float w = __shfl_sync(0xffffffffu, wgt, i);
-          const int li_loc = __shfl_sync(0xffffffffu, loc, i);
-          if (w == 0.f) continue;  // warp-uniform
+      for (int hh = 0; hh < NH; ++hh) {
+        const float w = __shfl_sync(0xffffffffu, wgt[hh], i);
+        if (w != 0.f) {  // warp-uniform
           float v[DPL];
           if (li_loc >= 0) {
-            load_bf16<DPL>(vstage + li_loc + lane * DPL, v);
+            load_bf16<DPL>(vstage + li_loc + u[hh] * D + lane * DPL, v);
           } else {
-            load_bf16_global<DPL>(ea.vgroup + ((size_t)u * ea.l_cap + (size_t)(-li_loc - 1)) * D + lane * DPL, v);
+            load_bf16_global<DPL>(ea.vgroup + ((size_t)u[hh] * ea.l_cap + (size_t)(-li_loc - 1)) * D + lane * DPL, v);
           }
 #pragma unroll
-          for (int e = 0; e < DPL; ++e) o[e] = fmaf(w, v[e], o[e]);
+          for (int e = 0; e < DPL; ++e) o[hh][e] = fmaf(w, v[e], o[hh][e]);
         }
       }
     }
+  }
+#pragma unroll
+  for (int hh = 0; hh < NH; ++hh) {
+    if (!hv[hh]) continue;
+    const int jl = h0 + hh;
     float* dst = &p.part_o[((row0 + jl) * p.s_cap + s) * D + lane * DPL];
     if constexpr (DPL == 4) {
-      *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<float4*>(dst) = make_float4(o[hh][0], o[hh][1], o[hh][2], o[hh][3]);
     } else {
-      *reinterpret_cast<float2*>(dst) = make_float2(o[0], o[1]);
+      *reinterpret_cast<float2*>(dst) = make_float2(o[hh][0], o[hh][1]);
     }
     if (lane == 0) {
-      p.part_m[(row0 + jl) * p.s_cap + s] = M;
-      p.part_l[(row0 + jl) * p.s_cap + s] = lsum;
+      p.part_m[(row0 + jl) * p.s_cap + s] = M[hh];
+      p.part_l[(row0 + jl) * p.s_cap + s] = lsum[hh];
       p.part_cnt[(row0 + jl) * p.s_cap + s] = es.cnt_run[jl];
     }
   }
