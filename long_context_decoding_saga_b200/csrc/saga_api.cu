@@ -17,6 +17,8 @@ namespace saga {
 cudaError_t launch_split(int D, int NP, int mode, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p,
                          dim3 grid, cudaStream_t st, int* occupancy_out);
 cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, cudaStream_t st);
+cudaError_t launch_dense(int D, int NP, const CUtensorMap& kf, const CUtensorMap& kp, const CUtensorMap& vf,
+                         const CUtensorMap& vp, const SplitParams& p, dim3 grid, cudaStream_t st, int* occ);
 cudaError_t launch_combine(int D, const CombineParams& p, cudaStream_t st);
 cudaError_t launch_select(const SelectParams& p, int rows, cudaStream_t st);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
@@ -170,6 +172,22 @@ EncodeTiledFn get_encode() {
 
 // 2-D view of the key cache: rows = B*h_k*l_cap tokens, d bf16 columns;
 // boxes of 64 columns (one 128-byte swizzle atom) by `box_rows` rows.
+// 2-D view of the value cache: rows = B*h_v*l_cap tokens, d bf16 columns;
+// boxes of 64 columns by `box_rows` rows, stored row-major (no swizzle).
+int make_value_map(CUtensorMap* m, const void* v_cache, const saga_shape* s, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (enc == nullptr) return fail(SAGA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
+  cuuint64_t dims[2] = {(cuuint64_t)s->d, (cuuint64_t)s->batch * s->h_v * s->l_cap};
+  cuuint64_t strides[1] = {(cuuint64_t)s->d * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(v_cache), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SAGA_ERR_CUDA, "cuTensorMapEncodeTiled (values) failed (%d)", (int)r);
+  return SAGA_OK;
+}
+
 int make_key_map(CUtensorMap* m, const void* k_cache, const saga_shape* s, int box_rows) {
   EncodeTiledFn enc = get_encode();
   if (enc == nullptr) return fail(SAGA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
@@ -238,10 +256,11 @@ void fill_split_common(SplitParams& p, const saga_shape* s, const Prepared& pr, 
 }
 
 int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, int mode, const CUtensorMap& tf,
-               const CUtensorMap& tp, int* S) {
+               const CUtensorMap& tp, int* S, bool dense = false) {
   int occ = 0;
   SplitParams dummy{};
-  cudaError_t e = launch_split(s->d, NP, mode, tf, tp, dummy, dim3(1), nullptr, &occ);
+  cudaError_t e = dense ? launch_dense(s->d, NP, tf, tp, tf, tp, dummy, dim3(1), nullptr, &occ)
+                        : launch_split(s->d, NP, mode, tf, tp, dummy, dim3(1), nullptr, &occ);
   if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
   if (occ < 1) return fail(SAGA_ERR_UNSUPPORTED, "split kernel does not fit on an SM");
   // A small step (at most 16 key tiles per SM) is latency-bound: one split
@@ -447,7 +466,17 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
     if (e != cudaSuccess) return cuda_fail(e, "from-scores launch");
   } else {
     const int mode = no_threshold ? kSplitDense : kSplitSparse;
-    rc = splits_for(s, pr, seq_len, NP, mode, tf, tp, &S);
+    // every token kept and one value head per group: the dense kernel (value
+    // tiles by TMA, no lists)
+    const bool dense = no_threshold && p.nvh == 1 && s->h_v <= s->h_k && NP <= 16;
+    CUtensorMap vf, vp;
+    if (dense) {
+      rc = make_value_map(&vf, v_cache, s, kTile);
+      if (rc) return rc;
+      rc = make_value_map(&vp, v_cache, s, kUnit);
+      if (rc) return rc;
+    }
+    rc = splits_for(s, pr, seq_len, NP, mode, tf, tp, &S, dense);
     if (rc) return rc;
     p.nsplit = S;
     if (ev0 != nullptr) {
@@ -463,8 +492,9 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
     p.v_cache_w = nr.v_cache;
     p.k_new = nr.k_new;
     p.v_new = nr.v_new;
-    e = launch_split(s->d, NP, mode, tf, tp, p, dim3(S, s->h_k, s->batch), st, nullptr);
-    if (e != cudaSuccess) return cuda_fail(e, "split launch");
+    e = dense ? launch_dense(s->d, NP, tf, tp, vf, vp, p, dim3(S, s->h_k, s->batch), st, nullptr)
+              : launch_split(s->d, NP, mode, tf, tp, p, dim3(S, s->h_k, s->batch), st, nullptr);
+    if (e != cudaSuccess) return cuda_fail(e, dense ? "dense launch" : "split launch");
   }
   if (ev1 != nullptr) {
     e = trace_record(ev1, st);

@@ -1080,6 +1080,384 @@ __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const Spl
   tail_merge<D, NP>(es, mrg, acc, ls, ea, vstage, q, lane, et, p, b, j0, s, false);
 }
 
+// ============================================================================ dense kernel
+// Attention with every token kept (N covers the context) and one value head
+// per key-head group (h_v <= h_k): a tile's value rows are contiguous, so
+// they come in by TMA with its key rows, and each epilogue warp runs the
+// softmax and the value sum of its 32 rows per tile (online, no lists).
+// Warp roles as in the split kernel; the partials feed the same combine.
+template <int D, int NP>
+struct DenseSmem {
+  static constexpr int NATOM = D / 64;
+  static constexpr int KBYTES = kTile * D * 2;
+  static constexpr int STAGE_BYTES = 2 * KBYTES;  // key tile (128-byte swizzle) + value tile (no swizzle)
+  static constexpr int NPM = mma_n<NP>();
+  static constexpr int NACC = acc_bufs<NP>();
+  static constexpr int QPAD = ((NATOM * NPM * 128 + 1023) / 1024) * 1024;
+  static constexpr int PBUF_BYTES = 4 * 32 * NP * 4;  // each warp's weights of a tile, [32][NP]
+  static constexpr int FIXED = QPAD + PBUF_BYTES + (2 * 4 + 2 * NACC + 1) * 8 + 16 + 1024;
+  static constexpr int NSTAGE_HALF = (kSmemHalf - FIXED) / STAGE_BYTES;
+  static constexpr bool TWO = NSTAGE_HALF >= 3;  // two CTAs per SM with 3 stages each
+  static constexpr int NSTAGE_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
+  static constexpr int NSTAGE = TWO ? 3 : (NSTAGE_FIT < 4 ? NSTAGE_FIT : 4);
+  static constexpr int CTAS_PER_SM = TWO ? 2 : 1;
+  static constexpr int Q_OFF = NSTAGE * STAGE_BYTES;
+  static constexpr int P_OFF = Q_OFF + QPAD;
+  static constexpr int BAR_OFF = P_OFF + PBUF_BYTES;
+  static constexpr int NBARS = 2 * NSTAGE + 2 * NACC + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int BYTES = MISC_OFF + 16;
+  static constexpr int ALLOC = BYTES + 1024;
+  static_assert(NSTAGE >= 2, "ring too shallow");
+  static_assert(ALLOC <= kSmemLimit, "shared memory over the per-CTA limit");
+  static_assert(!TWO || ALLOC <= kSmemHalf, "two CTAs per SM must fit in half the shared memory");
+  static_assert(4 * NP * (D + 2) * 4 <= NSTAGE * STAGE_BYTES, "merge buffer must fit in the ring");
+};
+
+// Key and value rows of tile t into its stage (128-row boxes, or 32-row
+// boxes for the rows left in the split).
+template <int NATOM, int NSTAGE, int STAGE_BYTES, int KBYTES>
+__device__ __forceinline__ void issue_kv_tile(int t, int start, int end, int krow, int vrow, uint8_t* ring,
+                                              uint64_t* full, const CUtensorMap* tkf, const CUtensorMap* tkp,
+                                              const CUtensorMap* tvf, const CUtensorMap* tvp) {
+  const int stage = t % NSTAGE;
+  const int r0 = start + t * kTile;
+  const int rows = min(kTile, end - r0);
+  uint8_t* dst = ring + stage * STAGE_BYTES;
+  if (rows == kTile) {
+    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+#pragma unroll
+    for (int a = 0; a < NATOM; ++a) {
+      tma_load_2d(dst + a * 16384, tkf, &full[stage], a * 64, krow + r0);
+      tma_load_2d(dst + KBYTES + a * 16384, tvf, &full[stage], a * 64, vrow + r0);
+    }
+  } else {
+    const int nsub = (rows + kUnit - 1) / kUnit;
+    mbar_arrive_expect_tx(&full[stage], 2 * nsub * kUnit * 128 * NATOM);
+    for (int i = 0; i < nsub; ++i)
+#pragma unroll
+      for (int a = 0; a < NATOM; ++a) {
+        tma_load_2d(dst + a * 16384 + i * kUnit * 128, tkp, &full[stage], a * 64, krow + r0 + i * kUnit);
+        tma_load_2d(dst + KBYTES + a * 16384 + i * kUnit * 128, tvp, &full[stage], a * 64, vrow + r0 + i * kUnit);
+      }
+  }
+}
+
+template <int D, int NP>
+__global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
+    saga_dense_kernel(const __grid_constant__ CUtensorMap tk_full, const __grid_constant__ CUtensorMap tk_part,
+                      const __grid_constant__ CUtensorMap tv_full, const __grid_constant__ CUtensorMap tv_part,
+                      const SplitParams p) {
+  using SM = DenseSmem<D, NP>;
+  constexpr int NATOM = SM::NATOM;
+  constexpr int NSTAGE = SM::NSTAGE;
+  constexpr int STAGE_BYTES = SM::STAGE_BYTES;
+  constexpr int KBYTES = SM::KBYTES;
+  constexpr int NPM = SM::NPM;
+  constexpr int NACC = SM::NACC;
+  constexpr int DPL = D / 32;
+  constexpr uint32_t TMEM_COLS = NACC * NPM <= 32 ? 32u : NACC * NPM <= 64 ? 64u : NACC * NPM <= 128 ? 128u : 256u;
+  constexpr uint32_t IDESC = umma_idesc_bf16(128, NPM);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint8_t* qsm = smem + SM::Q_OFF;
+  float* pbuf = reinterpret_cast<float*>(smem + SM::P_OFF);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFF);
+  uint64_t* empty = full + NSTAGE;
+  uint64_t* accf = empty + NSTAGE;
+  uint64_t* acce = accf + NACC;
+  uint64_t* fin = acce + NACC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::MISC_OFF + 4);
+
+  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j0 = h * p.G;
+  const int v_base = (int)(((long long)j0 * p.h_v) / p.h_q);
+  const int krow = (b * p.h_k + h) * p.l_cap;       // first cache row of this (batch, key head)
+  const int vrow = (b * p.h_v + v_base) * p.l_cap;  // ... and of its value head
+
+  // ---------------------------------------------------------------- setup before the dependency wait
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < NSTAGE; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1 + 4);  // the MMA's commit and the four epilogue warps
+    }
+    for (int i = 0; i < NACC; ++i) {
+      mbar_init(&accf[i], 1);
+      mbar_init(&acce[i], 4);
+    }
+    mbar_init(fin, 1);
+    mbar_init_fence();
+    tma_prefetch_desc(&tk_full);
+    tma_prefetch_desc(&tk_part);
+    tma_prefetch_desc(&tv_full);
+    tma_prefetch_desc(&tv_part);
+    int pst, pcap;
+    split_cap_range(p.seq_len, p.nsplit, s, p.l_cap, &pst, &pcap);
+    const long long ncta = (long long)gridDim.x * gridDim.y * gridDim.z;
+    const int cap_rows = max(kTile, (int)(((48ll << 20) / ncta) / (2 * D * 2)) / kTile * kTile);
+    const int pend = min(pcap, pst + cap_rows);
+    for (int r = pst; r < pend; r += kTile) {
+      const uint32_t bytes = (uint32_t)(min(kTile, pend - r) * D * 2);
+      prefetch_l2_bulk(p.k_cache + ((size_t)krow + r) * D, bytes);
+      prefetch_l2_bulk(p.v_cache + ((size_t)vrow + r) * D, bytes);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  pdl_trigger();
+  pdl_wait();
+
+  // ---------------------------------------------------------------- setup after it
+  constexpr int QCH = NATOM * NPM * 8;
+  constexpr int QV = (QCH + kEpiThreads - 1) / kEpiThreads;
+  const int eth = threadIdx.x - 64;
+  uint4 qv[QV];
+  if (warp >= 2) {
+#pragma unroll
+    for (int k = 0; k < QV; ++k) {
+      const int i = eth + k * kEpiThreads;
+      const int n = (i / 8) % NPM, col = (i / (NPM * 8)) * 64 + (i % 8) * 8;
+      qv[k] = make_uint4(0, 0, 0, 0);
+      if (i < QCH && n < p.G) qv[k] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.h_q + j0 + n) * D + col));
+    }
+  }
+  const int L = device_seq_len(p.seq_len_dev, p.seq_len, p.l_cap, (s == 0 && h == 0 && b == 0) ? p.status : nullptr);
+  int start, end;
+  split_range(p.seq_len, p.nsplit, s, L, &start, &end);
+  const int ntiles = (end - start + kTile - 1) / kTile;
+  const bool owner = p.k_new != nullptr && start <= L - 1 && L - 1 < end;
+  if (owner) append_new_rows<D>(p, b, h, j0, L - 1);
+  int issued = 0;
+  if (threadIdx.x == 0) {
+    for (; issued < ntiles && issued < NSTAGE; ++issued) {
+      if (owner && L - 1 < start + (issued + 1) * kTile) break;
+      issue_kv_tile<NATOM, NSTAGE, STAGE_BYTES, KBYTES>(issued, start, end, krow, vrow, ring, full, &tk_full, &tk_part,
+                                                        &tv_full, &tv_part);
+    }
+  }
+  if (warp >= 2) {
+#pragma unroll
+    for (int k = 0; k < QV; ++k) {
+      const int i = eth + k * kEpiThreads;
+      if (i < QCH) {
+        const int a = i / (NPM * 8), n = (i / 8) % NPM, c = i % 8;
+        *reinterpret_cast<uint4*>(qsm + a * NPM * 128 + n * 128 + ((c ^ (n & 7)) << 4)) = qv[k];
+      }
+    }
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // ---------------------------------------------------------------- roles
+  if (warp == 0) {
+    if (lane == 0) {
+      if (owner) fence_proxy_async_global();
+      for (int t = issued; t < ntiles; ++t) {
+        const int stage = t % NSTAGE, round = t / NSTAGE;
+        if (round > 0 && !mbar_wait(&empty[stage], (round - 1) & 1, abort_flag)) break;
+        issue_kv_tile<NATOM, NSTAGE, STAGE_BYTES, KBYTES>(t, start, end, krow, vrow, ring, full, &tk_full, &tk_part,
+                                                          &tv_full, &tv_part);
+        issued = t + 1;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int t = 0; t < ntiles; ++t) {
+        const int stage = t % NSTAGE, round = t / NSTAGE;
+        if (!mbar_wait(&full[stage], round & 1, abort_flag)) break;
+        const int abuf = t % NACC;
+        if (t >= NACC && !mbar_wait(&acce[abuf], ((t / NACC) - 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(ring + stage * STAGE_BYTES);
+        const uint32_t b0 = smem_u32(qsm);
+        const uint32_t d_tmem = tmem_base + abuf * NPM;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t aa = a0 + (k >> 2) * 16384 + (k & 3) * 32;
+          const uint32_t bb = b0 + (k >> 2) * NPM * 128 + (k & 3) * 32;
+          umma_bf16(d_tmem, umma_sdesc_sw128(aa), umma_sdesc_sw128(bb), IDESC, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&empty[stage]);
+        umma_commit(&accf[abuf]);
+      }
+      umma_commit(fin);
+      if (!mbar_wait_drain(fin, 0)) *abort_flag = 1;
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int et = threadIdx.x - 64;
+    const int q = warp & 3;  // TMEM lane quarter: rows 32q .. 32q+31 of every tile
+    const int erow = 32 * q + lane;
+    const bool counting = p.want_counts != 0;
+    float m[NP], lp[NP], o[NP][DPL];  // running max (warp-uniform), per-lane weight sums, columns of the lane
+#pragma unroll
+    for (int jl = 0; jl < NP; ++jl) {
+      m[jl] = -INFINITY;
+      lp[jl] = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) o[jl][e] = 0.f;
+    }
+    float* pw = pbuf + q * 32 * NP;
+    // the lane's columns of a value row: atom (lane*DPL)/64, byte offset within the 128-byte row
+    const int vcol = ((lane * DPL) / 64) * 16384 + ((lane * DPL) % 64) * 2;
+    int t = 0;
+    for (; t < ntiles; ++t) {
+      const int stage = t % NSTAGE;
+      const int abuf = t % NACC;
+      if (!__all_sync(0xffffffffu, mbar_wait(&accf[abuf], (t / NACC) & 1, abort_flag))) break;
+      tc_fence_after();
+      float sc[NP];
+      {
+        const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(abuf * NPM);
+        if constexpr (NP >= 16) {
+#pragma unroll
+          for (int i = 0; i < NP / 16; ++i) tmem_ld16(taddr + 16 * i, sc + 16 * i);
+        } else {
+          float all[16];
+          tmem_ld16(taddr, all);
+#pragma unroll
+          for (int i = 0; i < NP; ++i) sc[i] = all[i];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[abuf]);
+      const int tok = start + t * kTile + erow;
+      const bool valid = tok < end;
+      // online softmax of the warp's 32 rows, per head
+#pragma unroll
+      for (int jl = 0; jl < NP; ++jl) {
+        float pj = 0.f;
+        if (jl < p.G) {
+          const float x = sc[jl] * p.scale;
+          const uint32_t kmax = __reduce_max_sync(0xffffffffu, valid ? float_key(x) : 0u);
+          if (kmax != 0u) {  // warp-uniform
+            const float tm = key_float(kmax);
+            if (tm > m[jl]) {
+              const float f = (m[jl] == -INFINITY) ? 0.f : __expf(m[jl] - tm);
+              lp[jl] *= f;
+#pragma unroll
+              for (int e = 0; e < DPL; ++e) o[jl][e] *= f;
+              m[jl] = tm;
+            }
+          }
+          pj = valid ? __expf(x - m[jl]) : 0.f;
+          if (counting && valid) p.idxbuf[((size_t)b * p.h_q + j0 + jl) * p.l_cap + tok] = tok;
+        }
+        lp[jl] += pj;
+        sc[jl] = pj;
+      }
+#pragma unroll
+      for (int j4 = 0; j4 < NP / 4; ++j4)
+        *reinterpret_cast<float4*>(&pw[lane * NP + 4 * j4]) =
+            make_float4(sc[4 * j4], sc[4 * j4 + 1], sc[4 * j4 + 2], sc[4 * j4 + 3]);
+      // the value tile landed with the key tile (same stage barrier)
+      mbar_wait(&full[stage], (t / NSTAGE) & 1, abort_flag);
+      __syncwarp();
+      const uint8_t* vt = ring + stage * STAGE_BYTES + KBYTES + (32 * q) * 128 + vcol;
+      // rows past the split's end hold no loaded values (stale or outside
+      // data): never read them, even with weight 0 (0 * NaN is NaN)
+      const int nrows = min(32, max(0, end - (start + t * kTile + 32 * q)));
+#pragma unroll 4
+      for (int r = 0; r < nrows; ++r) {
+        float w[NP];
+#pragma unroll
+        for (int j4 = 0; j4 < NP / 4; ++j4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(&pw[r * NP + 4 * j4]);
+          w[4 * j4] = w4.x;
+          w[4 * j4 + 1] = w4.y;
+          w[4 * j4 + 2] = w4.z;
+          w[4 * j4 + 3] = w4.w;
+        }
+        float v[DPL];
+        load_bf16<DPL>(reinterpret_cast<const uint16_t*>(vt + r * 128), v);
+#pragma unroll
+        for (int jl = 0; jl < NP; ++jl)
+          if (jl < p.G) {
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) o[jl][e] = fmaf(w[jl], v[e], o[jl][e]);
+          }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+    }
+    // ---- merge the four warps' states and write the split's partial
+    constexpr int REG = NP * (D + 2);
+    float lw[NP];
+#pragma unroll
+    for (int jl = 0; jl < NP; ++jl) lw[jl] = warp_sum(lp[jl]);
+    named_bar_sync(1, kEpiThreads);  // every warp is done with the ring (value rows)
+    float* mrg = reinterpret_cast<float*>(ring);
+    float* mine = mrg + q * REG;
+    if (lane == 0) {
+#pragma unroll
+      for (int jl = 0; jl < NP; ++jl) {
+        mine[jl] = m[jl];
+        mine[NP + jl] = lw[jl];
+      }
+    }
+#pragma unroll
+    for (int jl = 0; jl < NP; ++jl)
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) mine[2 * NP + jl * D + lane * DPL + e] = o[jl][e];
+    named_bar_sync(1, kEpiThreads);
+    const size_t row0 = (size_t)b * p.h_q + j0;
+    for (int idx = et; idx < p.G * (D / 4); idx += kEpiThreads) {
+      const int jl = idx / (D / 4), c4 = idx % (D / 4);
+      float m4[4], M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        m4[w] = mrg[w * REG + jl];
+        M = fmaxf(M, m4[w]);
+      }
+      float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      float lsum = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float f = (m4[w] == -INFINITY) ? 0.f : __expf(m4[w] - M);
+        const float4 v = *reinterpret_cast<const float4*>(&mrg[w * REG + 2 * NP + jl * D + c4 * 4]);
+        acc4.x = fmaf(f, v.x, acc4.x);
+        acc4.y = fmaf(f, v.y, acc4.y);
+        acc4.z = fmaf(f, v.z, acc4.z);
+        acc4.w = fmaf(f, v.w, acc4.w);
+        lsum = fmaf(f, mrg[w * REG + NP + jl], lsum);
+      }
+      *reinterpret_cast<float4*>(&p.part_o[((row0 + jl) * p.s_cap + s) * D + c4 * 4]) = acc4;
+      if (c4 == 0) {
+        p.part_m[(row0 + jl) * p.s_cap + s] = M;
+        p.part_l[(row0 + jl) * p.s_cap + s] = lsum;
+        p.part_cnt[(row0 + jl) * p.s_cap + s] = end - start;
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag != 0) {
+    if (threadIdx.x == 0) flag_status(p.status, SAGA_STATUS_TIMEOUT);
+    if (warp == 0 && lane == 0)
+      for (int t = max(0, issued - NSTAGE); t < issued; ++t) mbar_wait_drain(&full[t % NSTAGE], (t / NSTAGE) & 1);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
 // ============================================================================ combine kernel
 // O[b, j] = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s over the splits of
 // row (b, j); zero when nothing was kept.  Also the kept counts and the
@@ -1452,6 +1830,29 @@ static cudaError_t run_from_scores(const SplitParams& p, dim3 grid, cudaStream_t
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(saga_from_scores_kernel<D, NP>), bytes, prepared);
   if (e != cudaSuccess) return e;
   return launch_k(saga_from_scores_kernel<D, NP>, grid, dim3(kEpiThreads), bytes, st, p);
+}
+
+template <int D, int NP>
+static cudaError_t run_dense(const CUtensorMap& kf, const CUtensorMap& kp, const CUtensorMap& vf, const CUtensorMap& vp,
+                             const SplitParams& p, dim3 grid, cudaStream_t st, int* occ) {
+  using K = DenseSmem<D, NP>;
+  static std::atomic<uint64_t> prepared{0};
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(saga_dense_kernel<D, NP>), K::ALLOC, prepared);
+  if (e != cudaSuccess) return e;
+  if (occ != nullptr)
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, saga_dense_kernel<D, NP>, 192, K::ALLOC);
+  return launch_k(saga_dense_kernel<D, NP>, grid, dim3(192), K::ALLOC, st, kf, kp, vf, vp, p);
+}
+
+// Dense attention (every token kept) for groups whose query heads share one
+// value head; NP in {4, 8, 16}.
+cudaError_t launch_dense(int D, int NP, const CUtensorMap& kf, const CUtensorMap& kp, const CUtensorMap& vf,
+                         const CUtensorMap& vp, const SplitParams& p, dim3 grid, cudaStream_t st, int* occ) {
+#define SAGA_DN(DD, NN) \
+  if (D == DD && NP == NN) return run_dense<DD, NN>(kf, kp, vf, vp, p, grid, st, occ);
+  SAGA_DN(64, 4) SAGA_DN(64, 8) SAGA_DN(64, 16) SAGA_DN(128, 4) SAGA_DN(128, 8) SAGA_DN(128, 16)
+#undef SAGA_DN
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, cudaStream_t st) {

@@ -47,6 +47,11 @@ CASES = [
           q_mode="gaussian", planted=0.0, steps=4),
     small("dense_g12_d128", h_q=12, h_k=1, h_v=4, d=128, l_kv=700, n_top=workload.DENSE, refresh=1 << 30,
           q_mode="gaussian", planted=0.0, steps=3),
+    # dense kernel (value tiles by TMA): d = 128 with value heads shared by key heads, batch 2, ragged length
+    small("dense_hv_lt_hk_d128", batch=2, h_q=8, h_k=4, h_v=2, d=128, l_kv=1333, n_top=workload.DENSE,
+          refresh=1 << 30, q_mode="gaussian", planted=0.0, steps=3),
+    small("dense_g16_d64", h_q=32, h_k=2, h_v=2, d=64, l_kv=2500, n_top=workload.DENSE, refresh=1 << 30,
+          q_mode="gaussian", planted=0.0, steps=3),
 ]
 
 
