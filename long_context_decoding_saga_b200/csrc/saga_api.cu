@@ -80,6 +80,16 @@ int device_sms(int* sms) {
   return SAGA_OK;
 }
 
+// Sub-groups per key head: at d = 64 a group of 16 or more query heads runs
+// as CTAs of 8 heads each (the 8-head kernel keeps two CTAs per SM and a
+// light epilogue; the sub-groups' repeated key tiles come from L2), when the
+// sub-groups split along value-head boundaries.
+int head_split(const saga_shape* s) {
+  const int G = s->h_q / s->h_k, hpv = s->h_q / s->h_v;
+  if (s->d == 64 && G >= 16 && G % 8 == 0 && (8 % hpv == 0 || hpv % 8 == 0)) return G / 8;
+  return 1;
+}
+
 int np_for_group(int G) { return G <= 4 ? 4 : G <= 8 ? 8 : G <= 16 ? 16 : G <= 32 ? 32 : 64; }
 
 int validate_shape(const saga_shape* s) {
@@ -245,8 +255,10 @@ void fill_split_common(SplitParams& p, const saga_shape* s, const Prepared& pr, 
   p.l_cap = s->l_cap;
   p.s_cap = pr.ws.s_cap;
   p.ld_scores = pr.ws.ld_scores;
-  p.G = s->h_q / s->h_k;
-  p.nvh = s->h_v >= s->h_k ? s->h_v / s->h_k : 1;
+  p.hsplit = head_split(s);
+  p.G = s->h_q / s->h_k / p.hsplit;
+  const int hpv = s->h_q / s->h_v;  // query heads per value head
+  p.nvh = p.G >= hpv ? p.G / hpv : 1;
   p.hpv = p.G / p.nvh;
   p.scale = (float)(1.0 / sqrt((double)s->d));
   p.part_o = reinterpret_cast<float*>(pr.base + pr.ws.part_o);
@@ -266,7 +278,7 @@ int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, int
   // A small step (at most 16 key tiles per SM) is latency-bound: one split
   // per SM, which leaves a second CTA slot to the next call's kernel (it
   // starts its setup and L2 prefetch early).  Larger steps fill every slot.
-  const int groups = s->batch * s->h_k;
+  const int groups = s->batch * s->h_k * head_split(s);
   const long long tiles = (long long)groups * ((seq_len + kTile - 1) / kTile);
   const int slots = (occ > 1 && tiles <= 16ll * pr.sms) ? pr.sms : occ * pr.sms;
   *S = choose_splits(groups, seq_len, slots, pr.ws.s_cap);
@@ -278,7 +290,8 @@ int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, int
 int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const void* k_cache, int seq_len,
                 const int* seq_len_dev, int n_top, float* tau, cudaStream_t st, cudaEvent_t ev_start = nullptr,
                 const NewRows& nr = NewRows()) {
-  const int G = s->h_q / s->h_k, NP = np_for_group(G);
+  const int hsplit = head_split(s);
+  const int G = s->h_q / s->h_k / hsplit, NP = np_for_group(G);
   CUtensorMap tf, tp;
   int rc = make_key_map(&tf, k_cache, s, kTile);
   if (rc) return rc;
@@ -304,7 +317,7 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   p.scores_out = reinterpret_cast<float*>(pr.base + pr.ws.scores);
   p.hist_out = hist;
   p.nsplit = S;
-  e = launch_split(s->d, NP, kSplitDump, tf, tp, p, dim3(S, s->h_k, s->batch), st, nullptr);
+  e = launch_split(s->d, NP, kSplitDump, tf, tp, p, dim3(S * hsplit, s->h_k, s->batch), st, nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "score dump launch");
   SelectParams sp{};
   sp.scores = p.scores_out;
@@ -433,7 +446,8 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
   rc = prepare_ws(s, workspace, ws_bytes, &pr);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int G = s->h_q / s->h_k, NP = np_for_group(G);
+  const int hsplit = head_split(s);
+  const int G = s->h_q / s->h_k / hsplit, NP = np_for_group(G);
   const bool refresh = (step % refresh_interval) == 0;
   const bool no_threshold = n_top >= s->l_cap;  // every possible length is covered by N
   const int rows = s->batch * s->h_q;
@@ -462,7 +476,7 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
     if (rc) return rc;
     p.scores_in = reinterpret_cast<const float*>(pr.base + pr.ws.scores);
     p.nsplit = S;
-    e = launch_from_scores(s->d, NP, p, dim3(S, s->h_k, s->batch), st);
+    e = launch_from_scores(s->d, NP, p, dim3(S * hsplit, s->h_k, s->batch), st);
     if (e != cudaSuccess) return cuda_fail(e, "from-scores launch");
   } else {
     const int mode = no_threshold ? kSplitDense : kSplitSparse;
@@ -492,8 +506,8 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
     p.v_cache_w = nr.v_cache;
     p.k_new = nr.k_new;
     p.v_new = nr.v_new;
-    e = dense ? launch_dense(s->d, NP, tf, tp, vf, vp, p, dim3(S, s->h_k, s->batch), st, nullptr)
-              : launch_split(s->d, NP, mode, tf, tp, p, dim3(S, s->h_k, s->batch), st, nullptr);
+    e = dense ? launch_dense(s->d, NP, tf, tp, vf, vp, p, dim3(S * hsplit, s->h_k, s->batch), st, nullptr)
+              : launch_split(s->d, NP, mode, tf, tp, p, dim3(S * hsplit, s->h_k, s->batch), st, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, dense ? "dense launch" : "split launch");
   }
   if (ev1 != nullptr) {

@@ -86,9 +86,10 @@ struct SplitParams {
   int batch, h_q, h_k, h_v, l_cap;
   int nsplit;    // splits per (batch, key head)
   int s_cap;     // partials stride
-  int G;         // h_q / h_k
-  int nvh;       // value heads per key-head group
-  int hpv;       // query heads of the group per value head
+  int G;         // query heads per CTA: h_q / h_k / hsplit
+  int hsplit;    // CTAs sharing a key head's query heads (sub-groups of G heads)
+  int nvh;       // value heads of a CTA's query heads
+  int hpv;       // query heads of the CTA per value head
   float scale;   // fp32(1/sqrt(d))
   int want_counts;
 };
@@ -134,6 +135,22 @@ struct AppendParams {
   int pos;
   int batch, h_k, h_v, d, l_cap;
 };
+
+// A CTA's coordinates: split s, key head h, batch b, first query head j0.
+// The sub-groups of one split are adjacent in blockIdx.x, so they run in the
+// same wave and the repeated key tiles come from L2.
+struct CtaCoord {
+  int s, h, b, j0;
+};
+__device__ inline CtaCoord cta_coord(const SplitParams& p) {
+  CtaCoord c;
+  c.s = blockIdx.x / p.hsplit;
+  const int part = blockIdx.x - c.s * p.hsplit;
+  c.h = blockIdx.y;
+  c.b = blockIdx.z;
+  c.j0 = (c.h * p.hsplit + part) * p.G;
+  return c;
+}
 
 // Reads the effective sequence length on the device, clamped to [1, l_cap].
 __device__ inline int device_seq_len(const int* dev, int host_len, int l_cap, unsigned* status) {

@@ -751,9 +751,10 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::MISC_OFF + 4);
 
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const CtaCoord cc = cta_coord(p);
+  const int s = cc.s, h = cc.h, b = cc.b;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j0 = h * p.G;
+  const int j0 = cc.j0;
   const int row_base = (b * p.h_k + h) * p.l_cap;  // first cache row of this (batch, key head)
 
   // ---------------------------------------------------------------- setup before the dependency wait
@@ -1046,9 +1047,10 @@ __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const Spl
   EpiShared<NP>& es = *reinterpret_cast<EpiShared<NP>*>(smem_raw);
   uint16_t* vstage = reinterpret_cast<uint16_t*>(smem_raw + SM::VST_OFF);
   float* mrg = reinterpret_cast<float*>(smem_raw + SM::MRG_OFF);
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const CtaCoord cc = cta_coord(p);
+  const int s = cc.s, h = cc.h, b = cc.b;
   const int et = threadIdx.x, q = et >> 5, lane = et & 31;
-  const int j0 = h * p.G;
+  const int j0 = cc.j0;
   pdl_trigger();
   pdl_wait();
   const int L = device_seq_len(p.seq_len_dev, p.seq_len, p.l_cap, nullptr);
@@ -1172,9 +1174,10 @@ __global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::MISC_OFF + 4);
 
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const CtaCoord cc = cta_coord(p);
+  const int s = cc.s, h = cc.h, b = cc.b;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j0 = h * p.G;
+  const int j0 = cc.j0;
   const int v_base = (int)(((long long)j0 * p.h_v) / p.h_q);
   const int krow = (b * p.h_k + h) * p.l_cap;       // first cache row of this (batch, key head)
   const int vrow = (b * p.h_v + v_base) * p.l_cap;  // ... and of its value head
