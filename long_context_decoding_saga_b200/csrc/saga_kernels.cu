@@ -1467,16 +1467,17 @@ __global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
 // ascending index list (concatenation of the per-split lists in split order).
 
 // Grid: (B*h_q rows, D/32 column chunks).  Warp w of a CTA takes splits
-// w, w+32, ... in blocks of eight (all loads of a block in flight at once)
-// with its own running maximum; lane c holds column 32*chunk + c, so every
-// load of a partial is one coalesced 128-byte segment.  The warps' states
-// are merged at the end in a fixed order (deterministic).
-constexpr int kCombineThreads = 1024;
+// w, w+8, ... in blocks of 24 (all loads of a block in flight at once, one
+// round for up to 192 splits) with its own running maximum; lane c holds
+// column 32*chunk + c, so every load of a partial is one coalesced 128-byte
+// segment.  The eight warps' states are merged at the end in a fixed order
+// (deterministic).
+constexpr int kCombineThreads = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads) saga_combine_kernel(const CombineParams p) {
   constexpr int NW = kCombineThreads / 32;
-  constexpr int U = 8;
+  constexpr int U = 24;
   __shared__ float wm[NW], wden[NW];
   __shared__ float wacc[NW][32];
   __shared__ int cnt_scan[kCombineThreads];
