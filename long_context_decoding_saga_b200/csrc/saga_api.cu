@@ -21,6 +21,7 @@ cudaError_t launch_dense(int D, int NP, const CUtensorMap& kf, const CUtensorMap
                          const CUtensorMap& vp, const SplitParams& p, dim3 grid, cudaStream_t st, int* occ);
 cudaError_t launch_combine(int D, const CombineParams& p, cudaStream_t st);
 cudaError_t launch_select(const SelectParams& p, int rows, cudaStream_t st);
+cudaError_t launch_select_parallel(const SelectParams& p, int rows, cudaStream_t st);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
 cudaError_t launch_fill(float* dst, float v, int n, cudaStream_t st);
 }  // namespace saga
@@ -137,7 +138,9 @@ WsLayout ws_layout(const saga_shape* s, int sms) {
   w.scores = off;
   off = align256(off + (size_t)rows * w.ld_scores * 4);
   w.hist = off;
-  off = align256(off + (size_t)rows * 256 * 4);
+  off = align256(off + (size_t)rows * (2 * 256 + 1) * 4);
+  w.cand = off;
+  off = align256(off + (size_t)rows * kCandCap * 4);
   w.idx = off;
   off = align256(off + (size_t)rows * s->l_cap * 4);
   w.total = off;
@@ -306,7 +309,7 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
     cudaError_t et = trace_record(ev_start, st);
     if (et != cudaSuccess) return cuda_fail(et, "trace event record");
   }
-  cudaError_t e = cudaMemsetAsync(hist, 0, rows * 256 * 4, st);
+  cudaError_t e = cudaMemsetAsync(hist, 0, rows * (2 * 256 + 1) * 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(hist)");
   SplitParams p;
   fill_split_common(p, s, pr, q, k_cache, seq_len, seq_len_dev);
@@ -329,7 +332,11 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   sp.row_len = seq_len;
   sp.l_cap = s->l_cap;
   sp.n_top = n_top;
-  e = launch_select(sp, (int)rows, st);
+  sp.hist2 = hist + rows * 256;
+  sp.cand_cnt = reinterpret_cast<int*>(hist + rows * 512);
+  sp.cand = reinterpret_cast<uint32_t*>(pr.base + pr.ws.cand);
+  sp.cand_cap = kCandCap;
+  e = launch_select_parallel(sp, (int)rows, st);
   if (e != cudaSuccess) return cuda_fail(e, "radix select launch");
   return SAGA_OK;
 }

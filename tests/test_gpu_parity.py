@@ -271,3 +271,39 @@ def test_plain_stream_order_matches():
             assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
             res[flag] = torch.load(path)
     assert torch.equal(res["0"]["out"], res["1"]["out"]) and torch.equal(res["0"]["tau"], res["1"]["tau"])
+
+
+def test_refresh_select_heavy_bin_falls_back():
+    """The refresh's parallel select when the N-th largest lies in a tie of more than 16384 scores (the
+    candidate buffer's size): the single-CTA digit scans take over and the threshold is still that score,
+    with every tied token kept."""
+    L0, N = 20000, 300
+    B, hq, hk, hv, d = 1, 4, 1, 4, 64
+    g = torch.Generator().manual_seed(5)
+    K = torch.ones((B, hk, L0, d)).to(torch.bfloat16)
+    bump = torch.randperm(L0, generator=g)[:50]
+    K[0, 0, bump] = 2.0  # 50 larger scores, then a 19950-way tie
+    V = torch.randn((B, hv, L0, d), generator=g).to(torch.bfloat16)
+    q = torch.full((B, hq, d), 0.25).to(torch.bfloat16)
+    kn = torch.ones((B, hk, d)).to(torch.bfloat16)
+    vn = torch.randn((B, hv, d), generator=g).to(torch.bfloat16)
+    l_cap = L0 + 1
+    shape = saga.SagaShape.of(B, hq, hk, hv, d, l_cap)
+    kc = torch.zeros((B, hk, l_cap, d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros((B, hv, l_cap, d), dtype=torch.bfloat16, device="cuda")
+    kc[:, :, :L0] = K.cuda()
+    vc[:, :, :L0] = V.cuda()
+    tau = torch.zeros((B, hq), device="cuda")
+    out = torch.zeros((B, hq, d), device="cuda")
+    cnt = torch.zeros((B, hq), dtype=torch.int32, device="cuda")
+    idx = torch.zeros((B, hq, l_cap), dtype=torch.int32, device="cuda")
+    ws = saga.alloc_workspace(shape, "cuda")
+    saga.saga_decode_step(shape, q.cuda(), kn.cuda(), vn.cuda(), kc, vc, l_cap, N, 4, 0, tau, out, ws,
+                          sel_count=cnt, sel_idx=idx)
+    torch.cuda.synchronize()
+    orc = saga_oracle.OracleLayer(K.float().numpy(), V.float().numpy(), hq, N, 4, l_cap=l_cap)
+    res = orc.step(q.float().numpy(), kn.float().numpy(), vn.float().numpy())
+    assert np.array_equal(tau.cpu().numpy(), res["tau"])  # the tied score, exactly
+    assert (cnt.cpu().numpy() == res["keep"].sum(-1)).all()  # every tied token kept (more than N)
+    assert int(cnt[0, 0]) > 16384
+    assert np.max(np.abs(out.cpu().numpy() - res["out"])) <= gpu_harness.OUT_TOL
