@@ -6,19 +6,22 @@
 //                    streams 128-token key tiles into a 128-byte-swizzled
 //                    shared-memory ring; scores A = q K^T / sqrt(d) (eq. 2)
 //                    for all query heads of the key head come from one
-//                    tcgen05.mma per 16 dims (keys = M 128, queries = N) into
-//                    TMEM, or from CUDA-core FMAs for groups of <= 4 query
-//                    heads; four epilogue warps compare against the Atop-N
-//                    threshold (Atop-N step 1), compact the kept tokens with
-//                    ballots and prefix sums, and accumulate the sparse
-//                    softmax and value sum of eq. 7 online over the h_v value
-//                    heads, writing one (max, sum, o) partial per split.
+//                    tcgen05.mma per 16 dims (keys = M 128, queries = N,
+//                    padded to 16) into TMEM; four epilogue warps compare
+//                    against the Atop-N threshold (Atop-N step 1), compact
+//                    the kept tokens with ballots, and accumulate the sparse
+//                    softmax and value sum of eq. 7 online over the h_v
+//                    value heads, writing one (max, sum, o) partial per split.
 //   dump variant   : refresh steps (Atop-N step 2) - the same scores are
 //                    written out with a per-head histogram of their top byte.
-//   select kernel  : exact N-th largest score per row by radix selection.
+//   select kernels : exact N-th largest score per row by radix selection
+//                    (many CTAs per row on refresh steps).
 //   from-scores    : refresh steps - compare/gather from the dumped scores.
+//   dense kernel   : every token kept, one value head per group - value
+//                    tiles by TMA, online softmax per tile, no lists.
 //   combine kernel : merges the split partials (log-sum-exp) into O.
-//   append kernel  : writes the new token's key/value rows into the cache.
+//   append kernel  : writes the new token's key/value rows into the cache
+//                    (when not fused into the attention kernels).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -153,6 +156,7 @@ struct EpiArgs {
   int rcapw;  // rows per list buffer whose value rows are staged in shared memory
   int cpr;    // 16-byte chunks of one row over the group's value heads
   int hmul;   // ceil(65536 / hpv): (j * hmul) >> 16 == j / hpv for j < 64
+  float scale;  // applied to a kept row's scores when it is listed (1 when they are scaled already)
 };
 
 // Per-lane online-softmax state: lane owns dims [lane*DPL, lane*DPL+DPL) of every head.
@@ -191,6 +195,7 @@ __device__ __forceinline__ EpiArgs epi_args(const SplitParams& p, int b, int j0)
   ea.rcapw = min(kBatch, vstage_warp_bytes<D, NP>() / (p.nvh * D * 2));
   ea.cpr = p.nvh * D / 8;
   ea.hmul = (65536 + p.hpv - 1) / p.hpv;
+  ea.scale = p.scale;
   return ea;
 }
 
@@ -198,6 +203,33 @@ __device__ __forceinline__ EpiArgs epi_args(const SplitParams& p, int b, int j0)
 // (N covers every length); nothing compared in dump mode.  Padding heads keep
 // nothing (+inf).  The load is separate from the shared-memory setup so that
 // a kernel can issue all of its setup loads back to back.
+// The smallest float x0 with fl(x0 * s) >= tv (s > 0): since x -> fl(x * s)
+// is monotone, `x >= x0` decides exactly what `fl(x * s) >= tv` decides for
+// every finite x, so a tile's raw dot products are compared without scaling
+// them.  -inf / +inf map to themselves.
+__device__ __forceinline__ bool scaled_ge(uint32_t k, float s, float tv) { return key_float(k) * s >= tv; }
+
+__device__ float raw_threshold(float tv, float s) {
+  if (tv == -INFINITY || tv == INFINITY) return tv;
+  const float y = tv / s;
+  if (y == INFINITY) return INFINITY;
+  if (y == -INFINITY) return -INFINITY;
+  const uint32_t kmin = float_key(-INFINITY), kmax = float_key(INFINITY);
+  uint32_t k = float_key(y);
+  for (int i = 0; i < 8 && k > kmin && scaled_ge(k - 1, s, tv); ++i) --k;
+  for (int i = 0; i < 8 && k < kmax && !scaled_ge(k, s, tv); ++i) ++k;
+  if (!(scaled_ge(k, s, tv) && (k == kmin || !scaled_ge(k - 1, s, tv)))) {
+    // not found near tv / s: binary search over every float (predicate monotone in the key)
+    uint32_t lo = kmin, hi = kmax;  // scaled_ge(kmax) holds: +inf * s = +inf
+    while (lo < hi) {
+      const uint32_t mid = lo + (hi - lo) / 2;
+      if (scaled_ge(mid, s, tv)) hi = mid; else lo = mid + 1;
+    }
+    k = lo;
+  }
+  return key_float(k);
+}
+
 template <int NP>
 __device__ __forceinline__ float load_tau(int et, const SplitParams& p, int b, int j0, bool compare) {
   float tv = INFINITY;
@@ -217,6 +249,18 @@ __device__ __forceinline__ void epi_setup(EpiShared<NP>& es, int et, const Split
 // Atop-N step 1 for the lane's token: bit j set when query head j keeps it.
 template <int NP>
 __device__ __forceinline__ uint64_t keep_mask(const EpiShared<NP>& es, const float (&sc)[NP], bool valid) {
+  if constexpr (NP <= 32) {
+    uint32_t k32 = 0;
+#pragma unroll
+    for (int j4 = 0; j4 < NP / 4; ++j4) {
+      const float4 tv = *reinterpret_cast<const float4*>(&es.tau[4 * j4]);
+      k32 |= (uint32_t)(sc[4 * j4 + 0] >= tv.x) << (4 * j4 + 0);
+      k32 |= (uint32_t)(sc[4 * j4 + 1] >= tv.y) << (4 * j4 + 1);
+      k32 |= (uint32_t)(sc[4 * j4 + 2] >= tv.z) << (4 * j4 + 2);
+      k32 |= (uint32_t)(sc[4 * j4 + 3] >= tv.w) << (4 * j4 + 3);
+    }
+    return valid ? (uint64_t)k32 : 0ull;
+  }
   uint64_t keep = 0;
 #pragma unroll
   for (int j4 = 0; j4 < NP / 4; ++j4) {
@@ -370,7 +414,8 @@ __device__ __forceinline__ void append_rows(EpiShared<NP>& es, WarpAcc<D, NP>& a
 #pragma unroll
     for (int j4 = 0; j4 < NP / 4; ++j4)
       *reinterpret_cast<float4*>(&li.sc[pos][4 * j4]) =
-          make_float4(sc[4 * j4 + 0], sc[4 * j4 + 1], sc[4 * j4 + 2], sc[4 * j4 + 3]);
+          make_float4(sc[4 * j4 + 0] * ea.scale, sc[4 * j4 + 1] * ea.scale, sc[4 * j4 + 2] * ea.scale,
+                      sc[4 * j4 + 3] * ea.scale);
   }
   __syncwarp();
   // value rows (every value head of the group) of the new list entries:
@@ -721,12 +766,13 @@ __device__ __forceinline__ void issue_key_tile(int t, int start, int end, int ro
   }
 }
 
-// Warp roles: 0 = TMA producer, 1 = tcgen05 MMA issuer (idle on the
-// CUDA-core path), 2..5 = epilogue (one thread per token row of a tile).
+// Warp roles: 0 = TMA producer, 1 = tcgen05 MMA issuer, 2..5 = epilogue
+// (one thread per token row of a tile).
 template <int D, int NP, bool UMMA, bool DUMP>
 __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     saga_split_kernel(const __grid_constant__ CUtensorMap tmap_full, const __grid_constant__ CUtensorMap tmap_part,
                       const SplitParams p) {
+  static_assert(UMMA, "scores come from tcgen05 for every group size");
   using SM = SplitSmem<D, NP, UMMA>;
   constexpr int NATOM = SM::NATOM;
   constexpr int NSTAGE = SM::NSTAGE;
@@ -819,6 +865,8 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     }
     tv = load_tau<NP>(eth, p, b, j0, !DUMP);
   }
+  // the epilogue compares raw dot products (scaled only once listed)
+  if (warp >= 2 && eth < NP) tv = raw_threshold(tv, p.scale);
   const int L = device_seq_len(p.seq_len_dev, p.seq_len, p.l_cap, (s == 0 && h == 0 && b == 0) ? p.status : nullptr);
   int start, end;
   split_range(p.seq_len, p.nsplit, s, L, &start, &end);
@@ -915,7 +963,7 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     for (; t < ntiles; ++t) {
       float sc[NP];
       bool ok;
-      if (UMMA) {
+      {
         const int abuf = t % NACC;
         ok = __all_sync(0xffffffffu, mbar_wait(&accf[abuf], (t / NACC) & 1, abort_flag));
         if (counting) ok = named_bar_and(1, kEpiThreads, ok);  // warps leave together (barriers below)
@@ -934,44 +982,11 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acce[abuf]);
-      } else {
-        const int stage = t % NSTAGE;
-        ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], (t / NSTAGE) & 1, abort_flag));
-        if (counting) ok = named_bar_and(1, kEpiThreads, ok);
-        if (!ok) break;
-        const uint8_t* rowp = kst + stage * STAGE_BYTES + erow * 128;
-        const float* qf = reinterpret_cast<const float*>(qsm);
-#pragma unroll
-        for (int n = 0; n < NP; ++n) sc[n] = 0.f;
-#pragma unroll
-        for (int a = 0; a < NATOM; ++a) {
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(rowp + a * 16384 + ((c ^ (erow & 7)) << 4));
-            const float kv[8] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y),
-                                 bf16_lo(raw.z), bf16_hi(raw.z), bf16_lo(raw.w), bf16_hi(raw.w)};
-#pragma unroll
-            for (int n = 0; n < NP; ++n) {
-              const float4 qa = *reinterpret_cast<const float4*>(qf + n * D + a * 64 + c * 8);
-              const float4 qb = *reinterpret_cast<const float4*>(qf + n * D + a * 64 + c * 8 + 4);
-              float x = sc[n];
-              x = fmaf(kv[0], qa.x, x);
-              x = fmaf(kv[1], qa.y, x);
-              x = fmaf(kv[2], qa.z, x);
-              x = fmaf(kv[3], qa.w, x);
-              x = fmaf(kv[4], qb.x, x);
-              x = fmaf(kv[5], qb.y, x);
-              x = fmaf(kv[6], qb.z, x);
-              x = fmaf(kv[7], qb.w, x);
-              sc[n] = x;
-            }
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
       }
+      if (DUMP) {
 #pragma unroll
-      for (int n = 0; n < NP; ++n) sc[n] *= p.scale;
+        for (int n = 0; n < NP; ++n) sc[n] *= p.scale;
+      }
       const int tok = start + t * kTile + erow;
       const bool valid = tok < end;
       if (DUMP) {
@@ -1059,8 +1074,9 @@ __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const Spl
   const int ntiles = (end - start + kTile - 1) / kTile;
   const bool counting = p.want_counts != 0;
 
-  epi_setup<NP>(es, et, p, load_tau<NP>(et, p, b, j0, true));
-  const EpiArgs ea = epi_args<D, NP>(p, b, j0);
+  epi_setup<NP>(es, et, p, load_tau<NP>(et, p, b, j0, true));  // dumped scores are scaled: compare as they are
+  EpiArgs ea = epi_args<D, NP>(p, b, j0);
+  ea.scale = 1.f;  // the dumped scores are scaled already
   uint16_t* vstage_w = vstage + (size_t)q * 2 * (vstage_warp_bytes<D, NP>() / 2);
   WarpAcc<D, NP> acc;
   acc.init();
