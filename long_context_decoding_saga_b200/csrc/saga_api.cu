@@ -283,7 +283,14 @@ int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, int
   // starts its setup and L2 prefetch early).  Larger steps fill every slot.
   const int groups = s->batch * s->h_k * head_split(s);
   const long long tiles = (long long)groups * ((seq_len + kTile - 1) / kTile);
-  const int slots = (occ > 1 && tiles <= 16ll * pr.sms) ? pr.sms : occ * pr.sms;
+  int slots = (occ > 1 && tiles <= 16ll * pr.sms) ? pr.sms : occ * pr.sms;
+  // With one split CTA per SM, the combine CTAs of the previous call (up to
+  // four share an SM once its split CTA has left) would hold back as many
+  // split CTAs of this call until the combine ends: a small step leaves
+  // them their SMs.
+  const int combine_ctas = s->batch * s->h_q * (s->d / 32);
+  const int reserve = (combine_ctas + 3) / 4;
+  if (occ == 1 && tiles <= 16ll * pr.sms && reserve <= pr.sms / 8) slots = pr.sms - reserve;
   *S = choose_splits(groups, seq_len, slots, pr.ws.s_cap);
   return SAGA_OK;
 }

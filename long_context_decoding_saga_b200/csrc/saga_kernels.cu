@@ -80,6 +80,30 @@ __device__ __forceinline__ void load_bf16_global(const uint16_t* src, float (&v)
   }
 }
 
+// DPL bf16 values as one packed word (generic address: shared or global).
+template <int N>
+struct Bf16Pack;
+template <>
+struct Bf16Pack<4> {
+  using T = uint2;
+  static __device__ __forceinline__ T zero() { return make_uint2(0u, 0u); }
+  static __device__ __forceinline__ void unpack(T r, float (&v)[4]) {
+    v[0] = bf16_lo(r.x);
+    v[1] = bf16_hi(r.x);
+    v[2] = bf16_lo(r.y);
+    v[3] = bf16_hi(r.y);
+  }
+};
+template <>
+struct Bf16Pack<2> {
+  using T = uint32_t;
+  static __device__ __forceinline__ T zero() { return 0u; }
+  static __device__ __forceinline__ void unpack(T r, float (&v)[2]) {
+    v[0] = bf16_lo(r);
+    v[1] = bf16_hi(r);
+  }
+};
+
 __device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
   uint32_t out;
   asm volatile(
@@ -591,8 +615,9 @@ __device__ __forceinline__ void tail_merge(EpiShared<NP>& es, float* mrg, const 
 #pragma unroll
     for (int hh = 0; hh < NH; ++hh) {
       const int jl = h0 + hh;
-      const float sc = (hv[hh] && ((keep >> jl) & 1ull)) ? li.sc[r][jl] : -INFINITY;
-      M[hh] = fmaxf(M[hh], warp_max(sc));
+      const uint32_t kk = (hv[hh] && ((keep >> jl) & 1ull)) ? float_key(li.sc[r][jl]) : 0u;
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, kk);
+      if (kmax != 0u) M[hh] = fmaxf(M[hh], key_float(kmax));
     }
   }
   float o[NH][DPL], lsum[NH];
@@ -642,22 +667,40 @@ __device__ __forceinline__ void tail_merge(EpiShared<NP>& es, float* mrg, const 
       }
       if (k < npool) loc = r < ea.rcapw ? (wk >> 1) * VWE + (bi * ea.rcapw + r) * ea.nvh * D : -(li.tok[r] + 1);
     }
+    // rows in groups of RG: every value load of a group (shared memory for
+    // staged rows, L2 for the others) is issued before the group's sums, so
+    // their latencies overlap; the sums keep the row order
+    using PK = Bf16Pack<DPL>;
+    constexpr int RG = NH <= 4 ? 4 : 2;
     const int nrow = min(32, npool - base);
-#pragma unroll 2
-    for (int i = 0; i < nrow; ++i) {
-      const int li_loc = __shfl_sync(0xffffffffu, loc, i);
+    for (int i0 = 0; i0 < nrow; i0 += RG) {
+      typename PK::T raw[RG][NH];
+      float wv[RG][NH];
 #pragma unroll
-      for (int hh = 0; hh < NH; ++hh) {
-        const float w = __shfl_sync(0xffffffffu, wgt[hh], i);
-        if (w != 0.f) {  // warp-uniform
-          float v[DPL];
-          if (li_loc >= 0) {
-            load_bf16<DPL>(vstage + li_loc + u[hh] * D + lane * DPL, v);
-          } else {
-            load_bf16_global<DPL>(ea.vgroup + ((size_t)u[hh] * ea.l_cap + (size_t)(-li_loc - 1)) * D + lane * DPL, v);
+      for (int k = 0; k < RG; ++k) {
+        const int i = i0 + k;
+        const int li_loc = __shfl_sync(0xffffffffu, loc, i & 31);
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+          const float w = __shfl_sync(0xffffffffu, wgt[hh], i & 31);
+          wv[k][hh] = i < nrow ? w : 0.f;
+          const uint16_t* src = li_loc >= 0
+                                    ? vstage + li_loc + u[hh] * D + lane * DPL
+                                    : ea.vgroup + ((size_t)u[hh] * ea.l_cap + (size_t)(-li_loc - 1)) * D + lane * DPL;
+          raw[k][hh] = PK::zero();
+          if (wv[k][hh] != 0.f) raw[k][hh] = *reinterpret_cast<const typename PK::T*>(src);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < RG; ++k) {
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) {
+          if (wv[k][hh] != 0.f) {  // warp-uniform
+            float v[DPL];
+            PK::unpack(raw[k][hh], v);
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) o[hh][e] = fmaf(wv[k][hh], v[e], o[hh][e]);
           }
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) o[hh][e] = fmaf(w, v[e], o[hh][e]);
         }
       }
     }
@@ -1482,16 +1525,21 @@ __global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
 // row (b, j); zero when nothing was kept.  Also the kept counts and the
 // ascending index list (concatenation of the per-split lists in split order).
 
-// Grid: (B*h_q rows, D/32 column chunks).  Warp w of a CTA takes splits
-// w, w+8, ... in blocks of 24 (all loads of a block in flight at once, one
-// round for up to 192 splits) with its own running maximum; lane c holds
-// column 32*chunk + c, so every load of a partial is one coalesced 128-byte
-// segment.  The eight warps' states are merged at the end in a fixed order
-// (deterministic).
+// Grid: (B*h_q rows, D/32 column chunks).  Warp w of a CTA takes the splits
+// [w*U, w*U + U) of each round of NW*U (one round for up to 192 splits):
+// lane u loads the (m, l) of split u, the warp reduces them, and every lane
+// loads the partial o of all U splits in its column (32*chunk + lane, so
+// each load is one coalesced 128-byte segment), all in flight at once,
+// weighting them with the shuffled factors.  The eight warps' states are
+// merged at the end in a fixed order (deterministic).
+// At most 64 registers a thread (16K for the CTA): with the 48K of a d = 128
+// split CTA that fills the SM's register file, so a combine CTA and a split
+// CTA of the next call share an SM - the split CTAs are resident before
+// their dependency wait ends.
 constexpr int kCombineThreads = 256;
 
 template <int D>
-__global__ void __launch_bounds__(kCombineThreads) saga_combine_kernel(const CombineParams p) {
+__global__ void __launch_bounds__(kCombineThreads, 4) saga_combine_kernel(const CombineParams p) {
   constexpr int NW = kCombineThreads / 32;
   constexpr int U = 24;
   __shared__ float wm[NW], wden[NW];
@@ -1507,31 +1555,25 @@ __global__ void __launch_bounds__(kCombineThreads) saga_combine_kernel(const Com
   const float* po = p.part_o + (size_t)row * p.s_cap * D + chunk * 32 + lane;
 
   float m_run = -INFINITY, den = 0.f, acc = 0.f;
-  for (int s0 = warp; s0 < S; s0 += U * NW) {
-    float ms[U], ls[U], v[U];
+  for (int s0 = warp * U; s0 < S; s0 += U * NW) {
+    const int su = s0 + lane;
+    const bool own = lane < U && su < S;
+    const float mu = own ? pm[su] : -INFINITY;
+    const float lu = own ? pl[su] : 0.f;
+    float v[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int ss = s0 + u * NW;
-      const bool in = ss < S;
-      ms[u] = in ? pm[ss] : -INFINITY;
-      ls[u] = in ? pl[ss] : 0.f;
-      v[u] = in ? po[(size_t)ss * D] : 0.f;
-    }
-    float mb = ms[0];
-#pragma unroll
-    for (int u = 1; u < U; ++u) mb = fmaxf(mb, ms[u]);
+    for (int u = 0; u < U; ++u) v[u] = s0 + u < S ? po[(size_t)(s0 + u) * D] : 0.f;
+    const float mb = warp_max(mu);
     if (mb > m_run) {  // warp-uniform
       const float f = (m_run == -INFINITY) ? 0.f : __expf(m_run - mb);
       den *= f;
       acc *= f;
       m_run = mb;
     }
+    const float fu = (mu == -INFINITY) ? 0.f : __expf(mu - m_run);
+    den += warp_sum(fu * lu);
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const float f = (ms[u] == -INFINITY) ? 0.f : __expf(ms[u] - m_run);
-      den = fmaf(f, ls[u], den);
-      acc = fmaf(f, v[u], acc);
-    }
+    for (int u = 0; u < U; ++u) acc = fmaf(__shfl_sync(0xffffffffu, fu, u), v[u], acc);
   }
   wacc[warp][lane] = acc;
   if (lane == 0) {
@@ -1981,13 +2023,19 @@ static cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 // cudaFuncSetAttribute holds per device: one bit per device ordinal.
+// Per kernel and device, once: the dynamic shared memory it may take, and
+// the largest shared-memory carveout.  Every kernel of the library asks for
+// the same carveout, so an SM running a small kernel (a combine) never has
+// to drain and reconfigure before a split CTA of the next call can join it.
 static cudaError_t ensure_smem(const void* fn, int bytes, std::atomic<uint64_t>& done) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
   if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (bytes > 0) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
   return e;
 }
@@ -2075,8 +2123,18 @@ cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, c
 }
 
 cudaError_t launch_combine(int D, const CombineParams& p, cudaStream_t st) {
-  if (D == 64) return launch_k(saga_combine_kernel<64>, dim3(p.rows, 2), dim3(kCombineThreads), 0, st, p);
-  if (D == 128) return launch_k(saga_combine_kernel<128>, dim3(p.rows, 4), dim3(kCombineThreads), 0, st, p);
+  static std::atomic<uint64_t> prepared64{0}, prepared128{0};
+  cudaError_t e;
+  if (D == 64) {
+    e = ensure_smem(reinterpret_cast<const void*>(saga_combine_kernel<64>), 0, prepared64);
+    if (e != cudaSuccess) return e;
+    return launch_k(saga_combine_kernel<64>, dim3(p.rows, 2), dim3(kCombineThreads), 0, st, p);
+  }
+  if (D == 128) {
+    e = ensure_smem(reinterpret_cast<const void*>(saga_combine_kernel<128>), 0, prepared128);
+    if (e != cudaSuccess) return e;
+    return launch_k(saga_combine_kernel<128>, dim3(p.rows, 4), dim3(kCombineThreads), 0, st, p);
+  }
   return cudaErrorInvalidValue;
 }
 
@@ -2096,6 +2154,11 @@ cudaError_t launch_select_parallel(const SelectParams& p, int rows, cudaStream_t
   if (e != cudaSuccess) return e;
   // parts per row: about 8K scores each, at most 32
   const int parts = max(1, min(32, (p.row_len + 8191) / 8192));
+  static std::atomic<uint64_t> prep_h{0}, prep_c{0};
+  e = ensure_smem(reinterpret_cast<const void*>(atopn_hist2_kernel), 0, prep_h);
+  if (e != cudaSuccess) return e;
+  e = ensure_smem(reinterpret_cast<const void*>(atopn_collect_kernel), 0, prep_c);
+  if (e != cudaSuccess) return e;
   e = launch_k(atopn_hist2_kernel, dim3(rows, parts), dim3(kSelPartThreads), 0, st, p);
   if (e != cudaSuccess) return e;
   e = launch_k(atopn_collect_kernel, dim3(rows, parts), dim3(kSelPartThreads), 0, st, p);
@@ -2104,11 +2167,17 @@ cudaError_t launch_select_parallel(const SelectParams& p, int rows, cudaStream_t
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st) {
+  static std::atomic<uint64_t> prepared{0};
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(saga_append_kernel), 0, prepared);
+  if (e != cudaSuccess) return e;
   const int n = p.batch * (p.h_k + p.h_v) * (p.d / 8);
   return launch_k(saga_append_kernel, dim3((n + 255) / 256), dim3(256), 0, st, p);
 }
 
 cudaError_t launch_fill(float* dst, float v, int n, cudaStream_t st) {
+  static std::atomic<uint64_t> prepared{0};
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(saga_fill_kernel), 0, prepared);
+  if (e != cudaSuccess) return e;
   return launch_k(saga_fill_kernel, dim3((n + 255) / 256), dim3(256), 0, st, dst, v, n);
 }
 
