@@ -463,21 +463,6 @@ __device__ __forceinline__ void append_rows(EpiShared<NP>& es, WarpAcc<D, NP>& a
   ls.n = r1;
 }
 
-// Before the tail: a warp left with many unreduced rows reduces them with
-// the batch reduction (columns across lanes), which beats the tail's
-// row-pool pass once there are more than a few rows.
-template <int D, int NP>
-__device__ __forceinline__ void flush_large_lists(EpiShared<NP>& es, WarpAcc<D, NP>& acc, const EpiArgs& ea,
-                                                  ListState& ls, int q, int lane, const uint16_t* vstage_w) {
-  const int rows = ls.n + (ls.pend >= 0 ? ls.npend : 0);
-  if (rows <= 8) return;  // warp-uniform
-  // the newest cp.async group belongs to the current buffer only if it holds rows
-  if (ls.pend >= 0) reduce_batch<D, NP>(es, acc, ea, q, lane, ls.pend, ls.npend, vstage_w, ls.n > 0);
-  if (ls.n > 0) reduce_batch<D, NP>(es, acc, ea, q, lane, ls.cur, ls.n, vstage_w, false);
-  ls.pend = -1;
-  ls.n = 0;
-}
-
 // Counting mode (kept counts and ascending index lists requested): the four
 // warps go through each tile together; per-head ballots give each kept
 // token its position in the split's list.
@@ -1047,11 +1032,8 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
       }
     }
     if (!DUMP) {
-      if (t == ntiles) flush_large_lists<D, NP>(es, acc, ea, ls, q, lane, vstage_w);
-      // the warps' states go into the key ring: with tcgen05 it is free once a
-      // warp has seen the last tile's scores (every MMA and copy is done); on
-      // the CUDA-core path the other warps may still be reading it
-      if (!UMMA) named_bar_sync(1, kEpiThreads);
+      // the warps' states go into the key ring: it is free once a warp has
+      // seen the last tile's scores (every MMA and copy is done)
       tail_merge<D, NP>(es, reinterpret_cast<float*>(kst), acc, ls, ea, vstage, q, lane, et, p, b, j0, s,
                         t != ntiles);
     }
@@ -1137,7 +1119,6 @@ __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const Spl
     const int tok = start + t * kTile + et;
     tile_epilogue<D, NP>(es, acc, ea, ls, q, lane, et, sc, tok, tok < end, counting, p, b, j0, start, vstage_w);
   }
-  flush_large_lists<D, NP>(es, acc, ea, ls, q, lane, vstage_w);
   tail_merge<D, NP>(es, mrg, acc, ls, ea, vstage, q, lane, et, p, b, j0, s, false);
 }
 
