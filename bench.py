@@ -267,9 +267,14 @@ def run_saga(args, wl, rank, world, local_rank):
     torch.cuda.set_device(dev)
 
     W, K = args.warmup, args.steps
+    # untimed steps after the warm-up so that the timed window starts on a
+    # refresh step (t % R == 0): K a multiple of R then times refresh and
+    # reuse steps in their true proportion, and a shorter window never leaves
+    # the refresh out
+    A = (wl.refresh - (1 + W) % wl.refresh) % wl.refresh if wl.refresh <= 1024 else 0
     E = 0 if args.no_e2e else max(4, min(K, 16))
     T = max(2, min(K, 8))  # kernel-timing replays
-    total_steps = 1 + W + K + E + T
+    total_steps = 1 + W + A + K + E + T
     l_cap = wl.l_kv + total_steps
     n_top = wl.n_for_kernel(l_cap)
     shape = saga.SagaShape.of(wl.batch, wl.h_q, wl.h_k, wl.h_v, wl.d, l_cap)
@@ -301,7 +306,7 @@ def run_saga(args, wl, rank, world, local_rank):
             sess.replay()
             cur += 1
 
-    replay_range(W)
+    replay_range(W + A)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -414,7 +419,7 @@ def run_saga(args, wl, rank, world, local_rank):
                    "h_v": wl.h_v, "d": wl.d, "n_top": wl.n_top if not wl.dense else "dense", "refresh": wl.refresh,
                    "layers": wl.layers, "parallelism": f"replicas{world}",
                    "l2": "inputs exceed L2 (all layers' caches cycle through L2 each step)",
-                   "refresh_steps_timed": refresh_steps},
+                   "refresh_steps_timed": refresh_steps, "alignment_steps": A},
         "roofline": roofline,
         "e2e": ({"value": job["e2e_value"], "unit": "GB/s",
                  "h2d_bytes_per_step": e2e["h2d_bytes_per_step"] * world,
