@@ -311,25 +311,51 @@ def run_saga(args, wl, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    # L2: a step whose streamed bytes are under twice the L2 would find part of
+    # its inputs still in L2 from the step before, so such steps are timed one
+    # by one with a 2 x L2 write between them, outside their events
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    step_bytes = wl.layers * layer_bytes(wl, wl.l_kv)
+    flush = args.flush_l2 == "on" or (args.flush_l2 == "auto" and step_bytes < 2 * l2_bytes)
+    scratch = torch.empty(2 * l2_bytes // 4, dtype=torch.float32, device=dev) if flush else None
     sampler = ClockSampler(dev.index if dev.index is not None else local_rank)
     sampler.start()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    marks = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     bytes_timed = 0
     refresh_steps = 0
+    kinds = []
     torch.cuda.nvtx.range_push("bench_timed")
-    ev0.record()
-    for _ in range(K):
+    for s_i in range(K):
         L = sess.length + 1
         bytes_timed += wl.layers * layer_bytes(wl, L)
-        refresh_steps += int(sess.t % wl.refresh == 0)
+        kinds.append(sess.t % wl.refresh == 0)
+        refresh_steps += int(kinds[-1])
+        if flush or s_i == 0:
+            marks[s_i][0].record()
         sess.stage(q_all[cur], k_all[cur], v_all[cur])
         sess.replay()
+        marks[s_i][1].record()
+        if flush:
+            scratch.fill_(float(s_i))
         cur += 1
-    ev1.record()
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     clocks = sampler.stop()
-    ms = ev0.elapsed_time(ev1)
+    # per-step durations: each step's own events when flushing, else from the
+    # previous step's end mark (back-to-back steps)
+    step_ms = []
+    for s_i in range(K):
+        start_ev = marks[s_i][0] if (flush or s_i == 0) else marks[s_i - 1][1]
+        step_ms.append(start_ev.elapsed_time(marks[s_i][1]))
+    ms = sum(step_ms)
+    ref_ms = [t for t, k in zip(step_ms, kinds) if k]
+    reuse_ms = [t for t, k in zip(step_ms, kinds) if not k]
+    step_stats = {"refresh_mean_us": statistics.mean(ref_ms) * 1e3 if ref_ms else None,
+                  "reuse_mean_us": statistics.mean(reuse_ms) * 1e3 if reuse_ms else None}
+    if ref_ms and reuse_ms and wl.refresh <= 1024:
+        step_stats["amortized_us"] = (step_stats["refresh_mean_us"] + (wl.refresh - 1) * step_stats["reuse_mean_us"]) / wl.refresh
+    if flush:
+        del scratch
     launches = refresh_steps * sess.launches_per_step(True) + (K - refresh_steps) * sess.launches_per_step(False)
     if world > 1:
         dist.barrier()
@@ -418,8 +444,11 @@ def run_saga(args, wl, rank, world, local_rank):
         "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "l_kv": wl.l_kv, "h_q": wl.h_q, "h_k": wl.h_k,
                    "h_v": wl.h_v, "d": wl.d, "n_top": wl.n_top if not wl.dense else "dense", "refresh": wl.refresh,
                    "layers": wl.layers, "parallelism": f"replicas{world}",
-                   "l2": "inputs exceed L2 (all layers' caches cycle through L2 each step)",
+                   "l2": ("flushed between timed steps (a 2 x L2 write outside each step's events)" if flush
+                          else "inputs exceed twice the L2 (all layers' caches cycle through L2 each step)"
+                          if step_bytes >= 2 * l2_bytes else "inputs fit in twice the L2; not flushed (--flush-l2 off)"),
                    "refresh_steps_timed": refresh_steps, "alignment_steps": A},
+        "step_us": step_stats,
         "roofline": roofline,
         "e2e": ({"value": job["e2e_value"], "unit": "GB/s",
                  "h2d_bytes_per_step": e2e["h2d_bytes_per_step"] * world,
@@ -444,6 +473,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
+    ap.add_argument("--flush-l2", default="auto", choices=["auto", "on", "off"],
+                    help="write 2 x L2 between timed steps (auto: when a step streams less than 2 x L2)")
     args = ap.parse_args()
     from long_context_decoding_saga_b200 import workload
     wl = workload.by_name(args.workload)

@@ -16,7 +16,7 @@
 namespace saga {
 cudaError_t launch_split(int D, int NP, int mode, const CUtensorMap& tf, const CUtensorMap& tp, const SplitParams& p,
                          dim3 grid, cudaStream_t st, int* occupancy_out);
-cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, cudaStream_t st);
+cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, cudaStream_t st, int* occ = nullptr);
 cudaError_t launch_dense(int D, int NP, const CUtensorMap& kf, const CUtensorMap& kp, const CUtensorMap& vf,
                          const CUtensorMap& vp, const SplitParams& p, dim3 grid, cudaStream_t st, int* occ);
 cudaError_t launch_combine(int D, const CombineParams& p, cudaStream_t st);
@@ -486,8 +486,16 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
   if (refresh && !no_threshold) {
     rc = run_refresh(s, pr, q, k_cache, seq_len, seq_len_dev, n_top, tau, st, ev0, nr);
     if (rc) return rc;
-    rc = splits_for(s, pr, seq_len, NP, kSplitDump, tf, tp, &S);
-    if (rc) return rc;
+    // the compare/gather pass reads scores, not keys: it runs with every
+    // CTA slot filled (it is latency-bound on its score loads per tile)
+    {
+      int occ = 0;
+      SplitParams dummy{};
+      e = launch_from_scores(s->d, NP, dummy, dim3(1), nullptr, &occ);
+      if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+      if (occ < 1) return fail(SAGA_ERR_UNSUPPORTED, "from-scores kernel does not fit on an SM");
+      S = choose_splits(s->batch * s->h_k * hsplit, seq_len, occ * pr.sms, pr.ws.s_cap);
+    }
     p.scores_in = reinterpret_cast<const float*>(pr.base + pr.ws.scores);
     p.nsplit = S;
     e = launch_from_scores(s->d, NP, p, dim3(S * hsplit, s->h_k, s->batch), st);

@@ -2063,11 +2063,13 @@ cudaError_t launch_split(int D, int NP, int mode, const CUtensorMap& tf, const C
 }
 
 template <int D, int NP>
-static cudaError_t run_from_scores(const SplitParams& p, dim3 grid, cudaStream_t st) {
+static cudaError_t run_from_scores(const SplitParams& p, dim3 grid, cudaStream_t st, int* occ) {
   static std::atomic<uint64_t> prepared{0};
   const int bytes = FromScoresSmem<D, NP>::BYTES;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(saga_from_scores_kernel<D, NP>), bytes, prepared);
   if (e != cudaSuccess) return e;
+  if (occ != nullptr)
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, saga_from_scores_kernel<D, NP>, kEpiThreads, bytes);
   return launch_k(saga_from_scores_kernel<D, NP>, grid, dim3(kEpiThreads), bytes, st, p);
 }
 
@@ -2094,9 +2096,9 @@ cudaError_t launch_dense(int D, int NP, const CUtensorMap& kf, const CUtensorMap
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, cudaStream_t st) {
+cudaError_t launch_from_scores(int D, int NP, const SplitParams& p, dim3 grid, cudaStream_t st, int* occ) {
 #define SAGA_FS(DD, NN) \
-  if (D == DD && NP == NN) return run_from_scores<DD, NN>(p, grid, st);
+  if (D == DD && NP == NN) return run_from_scores<DD, NN>(p, grid, st, occ);
   SAGA_FS(64, 4) SAGA_FS(64, 8) SAGA_FS(64, 16) SAGA_FS(64, 32) SAGA_FS(64, 64)
   SAGA_FS(128, 4) SAGA_FS(128, 8) SAGA_FS(128, 16) SAGA_FS(128, 32)
 #undef SAGA_FS
