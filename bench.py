@@ -197,6 +197,26 @@ def cpu_baseline(wl, seconds_budget=20.0):
             "us_per_layer_step": dt / done * 1e6, "us_per_step_scaled": dt / done * 1e6 * wl.layers}
 
 
+def alignment_steps(warmup, refresh):
+    """Untimed steps after the first (eager) step and the warm-up so that the timed window starts on a
+    refresh step (t % refresh == 0); none for a schedule that never refreshes again."""
+    if refresh > 1024:
+        return 0
+    return (refresh - (1 + warmup) % refresh) % refresh
+
+
+def step_means(step_ms, kinds, refresh):
+    """Mean refresh-step and reuse-step times (µs) of the timed steps and, when both kinds were timed,
+    their amortized mean over one refresh period."""
+    ref = [t for t, k in zip(step_ms, kinds) if k]
+    reuse = [t for t, k in zip(step_ms, kinds) if not k]
+    out = {"refresh_mean_us": statistics.mean(ref) * 1e3 if ref else None,
+           "reuse_mean_us": statistics.mean(reuse) * 1e3 if reuse else None}
+    if ref and reuse and refresh <= 1024:
+        out["amortized_us"] = (out["refresh_mean_us"] + (refresh - 1) * out["reuse_mean_us"]) / refresh
+    return out
+
+
 def gather_rank_stats(local, world):
     """Every rank's timing record, in rank order (one all_gather over the process group: NCCL or gloo)."""
     if world == 1:
@@ -271,7 +291,7 @@ def run_saga(args, wl, rank, world, local_rank):
     # refresh step (t % R == 0): K a multiple of R then times refresh and
     # reuse steps in their true proportion, and a shorter window never leaves
     # the refresh out
-    A = (wl.refresh - (1 + W) % wl.refresh) % wl.refresh if wl.refresh <= 1024 else 0
+    A = alignment_steps(W, wl.refresh)
     E = 0 if args.no_e2e else max(4, min(K, 16))
     T = max(2, min(K, 8))  # kernel-timing replays
     total_steps = 1 + W + A + K + E + T
@@ -348,12 +368,7 @@ def run_saga(args, wl, rank, world, local_rank):
         start_ev = marks[s_i][0] if (flush or s_i == 0) else marks[s_i - 1][1]
         step_ms.append(start_ev.elapsed_time(marks[s_i][1]))
     ms = sum(step_ms)
-    ref_ms = [t for t, k in zip(step_ms, kinds) if k]
-    reuse_ms = [t for t, k in zip(step_ms, kinds) if not k]
-    step_stats = {"refresh_mean_us": statistics.mean(ref_ms) * 1e3 if ref_ms else None,
-                  "reuse_mean_us": statistics.mean(reuse_ms) * 1e3 if reuse_ms else None}
-    if ref_ms and reuse_ms and wl.refresh <= 1024:
-        step_stats["amortized_us"] = (step_stats["refresh_mean_us"] + (wl.refresh - 1) * step_stats["reuse_mean_us"]) / wl.refresh
+    step_stats = step_means(step_ms, kinds, wl.refresh)
     if flush:
         del scratch
     launches = refresh_steps * sess.launches_per_step(True) + (K - refresh_steps) * sess.launches_per_step(False)
