@@ -433,6 +433,22 @@ def run_saga(args, wl, rank, world, local_rank):
             torch.cuda.synchronize()
             kernel_ms.extend(a.elapsed_time(b) for a, b in evs)
         del g
+    # kept-count statistics of the last step (layer 0), from one untimed call with index lists; it
+    # rewrites that layer's output and threshold with the same values and leaves the caches alone
+    kept = None
+    try:
+        B_, hq_ = wl.batch, wl.h_q
+        cnt = torch.zeros((B_, hq_), dtype=torch.int32, device=dev)
+        idx = torch.zeros((B_, hq_, l_cap), dtype=torch.int32, device=dev)
+        saga.saga_decode_attn(shape, sess.q_buf[0], sess.k_cache[0], sess.v_cache[0], sess.length, n_top,
+                              wl.refresh, sess.t - 1, sess.tau[0], sess.out[0], sess.workspace, sel_count=cnt,
+                              sel_idx=idx)
+        c = cnt.float().cpu()
+        kept = {"layer": 0, "L": sess.length, "n_top": n_top, "min": int(c.min()), "mean": float(c.mean()),
+                "max": int(c.max())}
+        del idx
+    except Exception as exc:  # noqa: BLE001  (reported, never fatal to the benchmark line)
+        kept = {"error": str(exc)[:200]}
     status = saga.saga_get_status(sess.workspace)
 
     # ---- gather over ranks (every rank takes part, whatever it measured)
@@ -464,6 +480,7 @@ def run_saga(args, wl, rank, world, local_rank):
                           if step_bytes >= 2 * l2_bytes else "inputs fit in twice the L2; not flushed (--flush-l2 off)"),
                    "refresh_steps_timed": refresh_steps, "alignment_steps": A},
         "step_us": step_stats,
+        "kept": kept,
         "roofline": roofline,
         "e2e": ({"value": job["e2e_value"], "unit": "GB/s",
                  "h2d_bytes_per_step": e2e["h2d_bytes_per_step"] * world,
