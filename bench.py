@@ -197,12 +197,23 @@ def cpu_baseline(wl, seconds_budget=20.0):
             "us_per_layer_step": dt / done * 1e6, "us_per_step_scaled": dt / done * 1e6 * wl.layers}
 
 
-def alignment_steps(warmup, refresh):
-    """Untimed steps after the first (eager) step and the warm-up so that the timed window starts on a
-    refresh step (t % refresh == 0); none for a schedule that never refreshes again."""
+def refresh_count(first, steps, refresh):
+    """Refresh steps (t % refresh == 0) among t = first .. first + steps - 1."""
+    return sum(1 for t in range(first, first + steps) if t % refresh == 0)
+
+
+def alignment_steps(warmup, refresh, steps):
+    """Untimed steps after the first (eager) step and the warm-up that place the K = `steps` timed steps
+    so that they hold the nearest whole number to K / R of refresh steps (halves rounded up): exactly
+    K / R when K is a multiple of R, else the nearer of floor and ceil.  None for a schedule that never
+    refreshes again."""
     if refresh > 1024:
         return 0
-    return (refresh - (1 + warmup) % refresh) % refresh
+    target = int(steps / refresh + 0.5)
+    for a in range(refresh):
+        if refresh_count(1 + warmup + a, steps, refresh) == target:
+            return a
+    return 0
 
 
 def step_means(step_ms, kinds, refresh):
@@ -287,11 +298,10 @@ def run_saga(args, wl, rank, world, local_rank):
     torch.cuda.set_device(dev)
 
     W, K = args.warmup, args.steps
-    # untimed steps after the warm-up so that the timed window starts on a
-    # refresh step (t % R == 0): K a multiple of R then times refresh and
-    # reuse steps in their true proportion, and a shorter window never leaves
-    # the refresh out
-    A = alignment_steps(W, wl.refresh)
+    # untimed steps after the warm-up that place the timed window so that it
+    # holds refresh and reuse steps in the proportion of the schedule (exact
+    # when K is a multiple of R)
+    A = alignment_steps(W, wl.refresh, K)
     E = 0 if args.no_e2e else max(4, min(K, 16))
     T = max(2, min(K, 8))  # kernel-timing replays
     total_steps = 1 + W + A + K + E + T

@@ -1,6 +1,7 @@
-"""The benchmark's timed window (CPU only): it starts on a refresh step, so a
-window of K = R steps holds exactly one refresh step, and the per-kind means
-amortize over one refresh period."""
+"""The benchmark's timed window (CPU only): it holds refresh and reuse steps
+in the proportion of the refresh schedule (the nearest whole number of
+refresh steps to K / R; exactly K / R when R divides K), and the per-kind
+means amortize over one refresh period."""
 import os
 import sys
 
@@ -12,17 +13,19 @@ import bench  # noqa: E402
 
 @pytest.mark.parametrize("warmup", [3, 4, 7, 31, 40])
 @pytest.mark.parametrize("refresh", [1, 2, 16, 32, 64])
-def test_window_starts_on_refresh(warmup, refresh):
-    a = bench.alignment_steps(warmup, refresh)
-    assert 0 <= a < refresh or (refresh == 1 and a == 0)
-    first_timed = 1 + warmup + a  # step 0 runs eagerly before the warm-up
-    assert first_timed % refresh == 0
-    kinds = [(first_timed + i) % refresh == 0 for i in range(refresh)]
-    assert sum(kinds) == 1 and kinds[0]
+@pytest.mark.parametrize("steps", [1, 5, 8, 16, 20, 32, 40, 64, 100])
+def test_window_holds_proportional_refreshes(warmup, refresh, steps):
+    a = bench.alignment_steps(warmup, refresh, steps)
+    assert 0 <= a < max(refresh, 1)
+    first = 1 + warmup + a  # step 0 runs eagerly before the warm-up
+    n = sum(1 for t in range(first, first + steps) if t % refresh == 0)
+    assert n == int(steps / refresh + 0.5)
+    if steps % refresh == 0:
+        assert n == steps // refresh
 
 
 def test_no_alignment_without_refresh():
-    assert bench.alignment_steps(3, 1 << 30) == 0
+    assert bench.alignment_steps(3, 1 << 30, 32) == 0
 
 
 def test_step_means_amortize():
