@@ -202,18 +202,23 @@ def refresh_count(first, steps, refresh):
     return sum(1 for t in range(first, first + steps) if t % refresh == 0)
 
 
-def alignment_steps(warmup, refresh, steps):
-    """Untimed steps after the first (eager) step and the warm-up that place the K = `steps` timed steps
-    so that they hold the nearest whole number to K / R of refresh steps (halves rounded up): exactly
-    K / R when K is a multiple of R, else the nearer of floor and ceil.  None for a schedule that never
-    refreshes again."""
+def alignment_from(first, refresh, steps):
+    """Untimed steps to run before a window of `steps` steps that would start at step `first`, so that
+    the window holds the nearest whole number to steps / R of refresh steps (halves rounded up):
+    exactly steps / R when R divides it, else the nearer of floor and ceil.  None for a schedule that
+    never refreshes again."""
     if refresh > 1024:
         return 0
     target = int(steps / refresh + 0.5)
     for a in range(refresh):
-        if refresh_count(1 + warmup + a, steps, refresh) == target:
+        if refresh_count(first + a, steps, refresh) == target:
             return a
     return 0
+
+
+def alignment_steps(warmup, refresh, steps):
+    """alignment_from for the timed window, which follows the first (eager) step and the warm-up."""
+    return alignment_from(1 + warmup, refresh, steps)
 
 
 def step_means(step_ms, kinds, refresh):
@@ -302,9 +307,10 @@ def run_saga(args, wl, rank, world, local_rank):
     # holds refresh and reuse steps in the proportion of the schedule (exact
     # when K is a multiple of R)
     A = alignment_steps(W, wl.refresh, K)
-    E = 0 if args.no_e2e else max(4, min(K, 16))
+    E = 0 if args.no_e2e else max(4, min(K, 64))
+    A2 = alignment_from(1 + W + A + K, wl.refresh, E) if E else 0  # the e2e window likewise
     T = max(2, min(K, 8))  # kernel-timing replays
-    total_steps = 1 + W + A + K + E + T
+    total_steps = 1 + W + A + K + A2 + E + T
     l_cap = wl.l_kv + total_steps
     n_top = wl.n_for_kernel(l_cap)
     shape = saga.SagaShape.of(wl.batch, wl.h_q, wl.h_k, wl.h_v, wl.d, l_cap)
@@ -388,6 +394,7 @@ def run_saga(args, wl, rank, world, local_rank):
     # end to end: pinned host inputs in, every layer's output out, inside the timed region
     e2e = None
     if E > 0:
+        replay_range(A2)
         hq = [q_all[cur + s].cpu().pin_memory() for s in range(E)]
         hk = [k_all[cur + s].cpu().pin_memory() for s in range(E)]
         hv = [v_all[cur + s].cpu().pin_memory() for s in range(E)]
@@ -396,10 +403,12 @@ def run_saga(args, wl, rank, world, local_rank):
         if world > 1:
             dist.barrier()
         e_bytes = 0
+        e_refresh = 0
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record()
         for s in range(E):
             e_bytes += wl.layers * layer_bytes(wl, sess.length + 1)
+            e_refresh += int(sess.t % wl.refresh == 0)
             sess.stage(hq[s], hk[s], hv[s])
             sess.replay()
             hout.copy_(sess.out, non_blocking=True)
@@ -410,7 +419,7 @@ def run_saga(args, wl, rank, world, local_rank):
         h2d = (hq[0].numel() * 2 + hk[0].numel() * 2 + hv[0].numel() * 2)
         d2h = hout.numel() * hout.element_size()
         e2e = {"value": e_bytes / (e_ms / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / E}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / E, "steps": E, "refresh_steps": e_refresh}
 
     # dominant kernel: the split-context attention kernel of reuse steps (with the fused append),
     # bracketed by CUDA events on its stream inside a freshly recorded graph (one event pair per layer;
@@ -494,7 +503,8 @@ def run_saga(args, wl, rank, world, local_rank):
         "roofline": roofline,
         "e2e": ({"value": job["e2e_value"], "unit": "GB/s",
                  "h2d_bytes_per_step": e2e["h2d_bytes_per_step"] * world,
-                 "d2h_bytes_per_step": e2e["d2h_bytes_per_step"] * world} if e2e else None),
+                 "d2h_bytes_per_step": e2e["d2h_bytes_per_step"] * world, "steps": e2e["steps"],
+                 "refresh_steps": e2e["refresh_steps"]} if e2e else None),
         "gpu_launches": launches,
         "clocks": clocks,
         "status_word": status,

@@ -36,3 +36,10 @@ def test_step_means_amortize():
     assert st["amortized_us"] == pytest.approx(4000.0)  # equals the window mean when K = R
     only = bench.step_means([3.0, 5.0], [True, True], 1)
     assert only["reuse_mean_us"] is None and "amortized_us" not in only
+
+
+@pytest.mark.parametrize("first", [0, 1, 5, 36, 77])
+@pytest.mark.parametrize("refresh,steps", [(32, 32), (32, 16), (16, 64), (64, 32), (1, 7)])
+def test_any_window_start(first, refresh, steps):
+    a = bench.alignment_from(first, refresh, steps)
+    assert bench.refresh_count(first + a, steps, refresh) == int(steps / refresh + 0.5)
