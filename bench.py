@@ -221,6 +221,18 @@ def alignment_steps(warmup, refresh, steps):
     return alignment_from(1 + warmup, refresh, steps)
 
 
+def step_plan(warmup, steps, refresh, e2e=True):
+    """The decode steps a run makes, in order: 1 eager step, `warmup` untimed steps, A untimed steps that
+    place the timed window, K = `steps` timed steps, A2 untimed steps that place the end-to-end window,
+    E end-to-end steps, T kernel-timing replays; `total` sizes the caches (l_kv + total)."""
+    A = alignment_steps(warmup, refresh, steps)
+    E = max(4, min(steps, 64)) if e2e else 0
+    A2 = alignment_from(1 + warmup + A + steps, refresh, E) if E else 0
+    T = max(2, min(steps, 8))
+    return {"A": A, "E": E, "A2": A2, "T": T, "total": 1 + warmup + A + steps + A2 + E + T,
+            "timed_first": 1 + warmup + A, "e2e_first": 1 + warmup + A + steps + A2}
+
+
 def step_means(step_ms, kinds, refresh):
     """Mean refresh-step and reuse-step times (µs) of the timed steps and, when both kinds were timed,
     their amortized mean over one refresh period."""
@@ -303,14 +315,8 @@ def run_saga(args, wl, rank, world, local_rank):
     torch.cuda.set_device(dev)
 
     W, K = args.warmup, args.steps
-    # untimed steps after the warm-up that place the timed window so that it
-    # holds refresh and reuse steps in the proportion of the schedule (exact
-    # when K is a multiple of R)
-    A = alignment_steps(W, wl.refresh, K)
-    E = 0 if args.no_e2e else max(4, min(K, 64))
-    A2 = alignment_from(1 + W + A + K, wl.refresh, E) if E else 0  # the e2e window likewise
-    T = max(2, min(K, 8))  # kernel-timing replays
-    total_steps = 1 + W + A + K + A2 + E + T
+    plan = step_plan(W, K, wl.refresh, not args.no_e2e)
+    A, E, A2, T, total_steps = plan["A"], plan["E"], plan["A2"], plan["T"], plan["total"]
     l_cap = wl.l_kv + total_steps
     n_top = wl.n_for_kernel(l_cap)
     shape = saga.SagaShape.of(wl.batch, wl.h_q, wl.h_k, wl.h_v, wl.d, l_cap)

@@ -43,3 +43,18 @@ def test_step_means_amortize():
 def test_any_window_start(first, refresh, steps):
     a = bench.alignment_from(first, refresh, steps)
     assert bench.refresh_count(first + a, steps, refresh) == int(steps / refresh + 0.5)
+
+
+@pytest.mark.parametrize("warmup,steps,refresh,e2e", [(3, 32, 32, True), (3, 16, 16, True), (3, 16, 64, True),
+                                                      (5, 100, 64, True), (3, 10, 1, False), (3, 32, 1 << 30, True)])
+def test_step_plan(warmup, steps, refresh, e2e):
+    p = bench.step_plan(warmup, steps, refresh, e2e)
+    assert p["total"] == 1 + warmup + p["A"] + steps + p["A2"] + p["E"] + p["T"]
+    assert p["timed_first"] == 1 + warmup + p["A"]
+    assert p["e2e_first"] == p["timed_first"] + steps + p["A2"]
+    if refresh <= 1024:
+        want = int(steps / refresh + 0.5)
+        assert bench.refresh_count(p["timed_first"], steps, refresh) == want
+        if e2e:
+            assert bench.refresh_count(p["e2e_first"], p["E"], refresh) == int(p["E"] / refresh + 0.5)
+    assert (p["E"] == 0) == (not e2e)
