@@ -168,32 +168,32 @@ def oracle_threads():
     return n
 
 
-def cpu_baseline(wl, seconds_budget=20.0):
-    """The oracle as it stands, on a bounded sample: whole decode steps of single layers at full size."""
-    import numpy as np
-    import torch
-
+def cpu_baseline(wl, seconds_budget=10.0, max_steps=512):
+    """The oracle as it stands, on a bounded sample: consecutive decode steps of layer 0 at full size,
+    from a refresh step on, until `seconds_budget` has passed and the steps cover whole refresh periods
+    (or three times the budget has passed, or `max_steps` steps were made)."""
     from long_context_decoding_saga_b200 import workload
     from oracle import saga_oracle
 
     cores = oracle_threads()
-    inp = workload.make_layer(wl, 0, device="cpu", steps=2)
+    inp = workload.make_layer(wl, 0, device="cpu", steps=max_steps)
     orc = saga_oracle.OracleLayer(inp["K0"].float().numpy(), inp["V0"].float().numpy(), wl.h_q,
-                                  wl.n_for_kernel(wl.l_kv + 2), wl.refresh, l_cap=wl.l_kv + 2)
+                                  wl.n_for_kernel(wl.l_kv + max_steps), wl.refresh, l_cap=wl.l_kv + max_steps)
     t0 = time.perf_counter()
-    done, nbytes = 0, 0
-    kinds = []
-    for t in range(2):
+    done, nbytes, refreshes = 0, 0, 0
+    for t in range(max_steps):
         orc.step(inp["q"][t].float().numpy(), inp["k_new"][t].float().numpy(), inp["v_new"][t].float().numpy())
         done += 1
         nbytes += layer_bytes(wl, wl.l_kv + t + 1)
-        kinds.append("refresh" if t % wl.refresh == 0 else "reuse")
-        if time.perf_counter() - t0 > seconds_budget:
+        refreshes += int(t % wl.refresh == 0)
+        el = time.perf_counter() - t0
+        whole = wl.refresh > 1024 or (t + 1) % wl.refresh == 0
+        if (el > seconds_budget and whole) or el > 3 * seconds_budget:
             break
     dt = time.perf_counter() - t0
-    del torch, np
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{done} layer-steps of layer 0 ({'+'.join(kinds)}) at full size, numpy oracle",
+            "sample": f"{done} consecutive decode steps of layer 0 at full size ({refreshes} of them refresh "
+                      f"steps), numpy oracle, {dt:.1f} s",
             "us_per_layer_step": dt / done * 1e6, "us_per_step_scaled": dt / done * 1e6 * wl.layers}
 
 
