@@ -174,13 +174,6 @@ class OracleLayer:
         return {"out": out, "tau": self.tau.copy(), "keep": keep, "scores": A, "L": L, "refreshed": refreshed}
 
 
-def decode_attention(q, k_cache, v_cache, L, tau):
-    """One step's attention given the threshold to compare against (no state)."""
-    A = scores(q, k_cache, L)
-    keep = select(A, tau)
-    return sparse_attention(A, keep, v_cache, L), keep, A
-
-
 def refresh_threshold(q, k_cache, L, n_top):
     """The exact threshold a refresh step computes from the current scores."""
     return threshold(scores(q, k_cache, L), n_top)

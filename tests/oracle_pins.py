@@ -14,6 +14,9 @@ What pins what:
   on tie-free data;
 * tie rule: every score equal to the threshold is kept;
 * stale-threshold reuse: a two-step example worked out by hand (closed form);
+* the stand-alone refresh threshold: brute-force exact scores (math.fsum) and a Python sort, with
+  ties; it also equals what a refresh step stores;
+* capacity growth: a layer that outgrows its initial capacity matches one created large enough;
 * softmax / value sum: constant value rows give that constant; each output
   coordinate lies between the kept rows' extremes; a single kept token gives
   its value row; an empty selection gives zero;
@@ -196,6 +199,55 @@ def pin_single_and_empty(o):
     assert (res["out"] == 0).all()
 
 
+def pin_refresh_threshold_bruteforce(o):
+    """The stand-alone refresh threshold is the N-th largest (with multiplicity) of the row's scores.
+
+    Scores by brute force on a hand-made cache: K heads expanded to the query heads with
+    repeat_interleave (the contiguous grouping), every dot product summed exactly with math.fsum
+    (bf16 products are exact in float64; d = 16 makes the 1/sqrt(d) scale 0.25, exact too), rounded
+    once to fp32, then sorted with Python's sort.  Integer-valued keys make ties at the threshold.
+    The same threshold must also be what a refresh step of OracleLayer stores for the same inputs.
+    """
+    rng = np.random.default_rng(14)
+    B, h_q, h_k, h_v, d, l_kv = 2, 6, 2, 3, 16, 23
+    for trial in range(6):
+        k0 = _bf16(np.round(rng.standard_normal((B, h_k, l_kv, d)) * 2) if trial % 2 else rng.standard_normal((B, h_k, l_kv, d)))
+        v0 = _rand(rng, (B, h_v, l_kv, d))
+        q = _bf16(np.round(rng.standard_normal((B, h_q, d)) * 2) if trial % 2 else rng.standard_normal((B, h_q, d)))
+        kn, vn = _rand(rng, (B, h_k, d)), _rand(rng, (B, h_v, d))
+        K = np.concatenate([k0, kn[:, :, None]], axis=2)
+        L = l_kv + 1
+        Kq = torch.as_tensor(K, dtype=torch.float64).repeat_interleave(h_q // h_k, dim=1).numpy()
+        for n in (1, 3, 7, L - 1, L, L + 4):
+            got = o.refresh_threshold(q, K, L, n)
+            for b in range(B):
+                for j in range(h_q):
+                    row = [float(np.float32(math.fsum(float(q[b, j, c]) * float(Kq[b, j, i, c]) for c in range(d)) * 0.25))
+                           for i in range(L)]
+                    expect = sorted(row, reverse=True)[n - 1] if n < L else -math.inf
+                    assert float(got[b, j]) == expect, (trial, n, b, j, float(got[b, j]), expect)
+            layer = o.OracleLayer(k0, v0, h_q, n, 5)
+            res = layer.step(q, kn, vn)
+            assert res["refreshed"]
+            np.testing.assert_array_equal(res["tau"], got)
+
+
+def pin_capacity_growth(o):
+    """A layer created with the default capacity grows past it and gives, step for step, the same
+    thresholds, selections and outputs as one created large enough from the start."""
+    rng = np.random.default_rng(15)
+    B, h_q, h_k, h_v, d, l_kv, steps = 1, 4, 1, 2, 8, 12, 150
+    k0, v0 = _rand(rng, (B, h_k, l_kv, d)), _rand(rng, (B, h_v, l_kv, d))
+    grown = o.OracleLayer(k0, v0, h_q, 5, 7)
+    big = o.OracleLayer(k0, v0, h_q, 5, 7, l_cap=l_kv + steps)
+    for _ in range(steps):
+        q, kn, vn = _rand(rng, (B, h_q, d)), _rand(rng, (B, h_k, d)), _rand(rng, (B, h_v, d))
+        a, b = grown.step(q, kn, vn), big.step(q, kn, vn)
+        for key in ("tau", "keep", "scores", "out"):
+            np.testing.assert_array_equal(a[key], b[key])
+    assert grown.length == l_kv + steps
+
+
 def pin_vector_reads(o):
     with open(os.path.join(GOLDEN, "vector_reads_llama_128k.json")) as f:
         g = json.load(f)
@@ -207,4 +259,5 @@ def pin_vector_reads(o):
 
 
 ALL_PINS = [pin_dense_cases, pin_bruteforce_topn, pin_exact_count, pin_ties, pin_stale_two_step,
-            pin_softmax_invariants, pin_single_and_empty, pin_vector_reads]
+            pin_softmax_invariants, pin_single_and_empty, pin_refresh_threshold_bruteforce, pin_capacity_growth,
+            pin_vector_reads]

@@ -89,9 +89,25 @@ def _m_dense_threshold_min(o):
     o.nth_largest = nth_largest
 
 
+def _m_refresh_threshold_short_row(o):
+    # the stand-alone refresh reads one token too few (the new token left out)
+    o.refresh_threshold = lambda q, k, L, n: o.threshold(o.scores(q, k, L - 1), n)
+
+
+def _m_grow_drops_rows(o):
+    # growth reallocates the caches without carrying the cached rows over
+    def _grow(self):
+        if self.length < self.k.shape[2]:
+            return
+        pad = max(64, self.k.shape[2] // 4)
+        self.k = np.zeros((*self.k.shape[:2], self.k.shape[2] + pad, self.k.shape[3]), np.float32)
+        self.v = np.zeros((*self.v.shape[:2], self.v.shape[2] + pad, self.v.shape[3]), np.float32)
+    o.OracleLayer._grow = _grow
+
+
 MUTANTS = [_m_key_head_mod, _m_value_head_interleaved, _m_no_scale, _m_negated_scores, _m_nth_off_by_one,
            _m_strict_compare, _m_refresh_every_step, _m_refresh_wrong_phase, _m_unnormalised, _m_append_off_by_one,
-           _m_dense_threshold_min]
+           _m_dense_threshold_min, _m_refresh_threshold_short_row, _m_grow_drops_rows]
 
 
 @pytest.mark.parametrize("mutate", MUTANTS, ids=lambda f: f.__name__[3:])
