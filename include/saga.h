@@ -178,20 +178,37 @@ SAGA_API int saga_trace_next_attention(void* ev_start, void* ev_end);
  *   - Shapes whose saga_workspace_bytes exceeds the scratch are rejected with
  *     SAGA_ERR_WORKSPACE and a message; use saga_decode_attn for those.
  *   - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
- *   - The first call on a device looks up the scratch's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - The scratch's device address comes from cudaGetSymbolAddress, looked up
+ *     on each call made outside stream capture; a call made during capture
+ *     uses the address an earlier call found, so make the first call on a
+ *     device before any stream capture (else SAGA_ERR_CUDA).
+ *   - Arguments are checked first; only then is the scratch's status word
+ *     cleared on the stream, ahead of the kernels.
  *   - Every call on a device shares the one scratch array, which keeps the
- *     previous call's contents; each call clears the status word it uses.
- *     Calls whose work overlaps on the GPU (other streams, other host
- *     threads) race on the scratch: serialize them.
- * saga_noalloc_last_error() describes the last failure of this entry point. */
+ *     previous call's contents.  Calls whose work overlaps on the GPU (other
+ *     streams, other host threads) race on the scratch: serialize them.
+ * saga_noalloc_last_error() describes the last failure of this entry point;
+ * saga_noalloc_get_status() reads the status word of the last call on the
+ * current device (after synchronizing `stream`). */
 #define SAGA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 SAGA_API size_t saga_noalloc_scratch_bytes(void);
 SAGA_API int saga_decode_attn_noalloc(const saga_shape* s, const void* q, const void* k_cache, const void* v_cache,
                                       int seq_len, const int* seq_len_dev, int n_top, int refresh_interval,
                                       long long step, float* tau, void* out, int out_dtype, int* sel_count,
                                       int* sel_idx, void* stream);
+SAGA_API int saga_noalloc_get_status(void* stream, unsigned* status);
 SAGA_API const char* saga_noalloc_last_error(void);
+
+/* Test hook for failure detection (no counterpart in the paper).  The next
+ * saga_decode_attn / saga_decode_step call on this host thread, if it is a
+ * reuse step (step % R != 0) run by the context-split attention kernel,
+ * makes that kernel's epilogue wait, for at most limit_ns, on a barrier
+ * that nothing arrives at, instead of running.  The wait gives up, the
+ * kernel's pipeline unwinds (in-flight copies drained, TMEM freed) and
+ * SAGA_STATUS_TIMEOUT is set in the status word; the call's results are then
+ * invalid and the context stays usable.  One-shot: consumed by that next
+ * call whatever its kind; limit_ns = 0 cancels a pending request. */
+SAGA_API int saga_test_expire_next_wait(unsigned limit_ns);
 
 /* Reads the workspace status word (SAGA_STATUS_* bits ORed by the kernels
  * since the workspace was zeroed) after synchronizing `stream`. */

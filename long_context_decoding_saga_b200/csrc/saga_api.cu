@@ -32,6 +32,7 @@ namespace {
 
 thread_local char g_err[512] = "";
 thread_local cudaEvent_t g_trace_start = nullptr, g_trace_end = nullptr;
+thread_local unsigned g_test_wait_ns = 0;  // saga_test_expire_next_wait
 
 cudaError_t trace_record(cudaEvent_t ev, cudaStream_t st) {
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
@@ -295,11 +296,17 @@ int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, int
   return SAGA_OK;
 }
 
+int clear_status_word(const Prepared& pr, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(pr.base + pr.ws.status, 0, 16, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  return SAGA_OK;
+}
+
 // Scores of every cached token, their top-byte histograms, and the exact
-// threshold (refresh).
+// threshold (refresh).  clear_status zeroes the status word first.
 int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const void* k_cache, int seq_len,
                 const int* seq_len_dev, int n_top, float* tau, cudaStream_t st, cudaEvent_t ev_start = nullptr,
-                const NewRows& nr = NewRows()) {
+                const NewRows& nr = NewRows(), bool clear_status = false) {
   const int hsplit = head_split(s);
   const int G = s->h_q / s->h_k / hsplit, NP = np_for_group(G);
   CUtensorMap tf, tp;
@@ -312,6 +319,10 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   if (rc) return rc;
   const size_t rows = (size_t)s->batch * s->h_q;
   uint32_t* hist = reinterpret_cast<uint32_t*>(pr.base + pr.ws.hist);
+  if (clear_status) {
+    rc = clear_status_word(pr, st);
+    if (rc) return rc;
+  }
   if (ev_start != nullptr) {
     cudaError_t et = trace_record(ev_start, st);
     if (et != cudaSuccess) return cuda_fail(et, "trace event record");
@@ -352,7 +363,7 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
 
 extern "C" {
 
-int saga_abi_version(void) { return 100; }
+int saga_abi_version(void) { return 101; }
 
 const char* saga_last_error(void) { return g_err; }
 
@@ -440,11 +451,13 @@ int atopn_select_threshold(const float* scores, int rows, int row_len, long long
 namespace {
 
 // One attention step; with nr set, the new token's rows are appended at
-// seq_len - 1 by the attention kernels themselves.
+// seq_len - 1 by the attention kernels themselves.  clear_status zeroes the
+// workspace status word once every argument has been checked, just before
+// the first enqueue.
 int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const void* v_cache, int seq_len,
                 const int* seq_len_dev, int n_top, int refresh_interval, long long step, float* tau, void* out,
                 int out_dtype, int* sel_count, int* sel_idx, void* workspace, size_t ws_bytes, void* stream,
-                const NewRows& nr) {
+                const NewRows& nr, bool clear_status = false) {
   int rc = validate_shape(s);
   if (rc) return rc;
   if (!q || !k_cache || !v_cache || !tau || !out) return fail(SAGA_ERR_ARG, "NULL tensor pointer");
@@ -474,6 +487,8 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
 
   cudaEvent_t ev0 = g_trace_start, ev1 = g_trace_end;
   g_trace_start = g_trace_end = nullptr;
+  const unsigned test_wait_ns = g_test_wait_ns;
+  g_test_wait_ns = 0;
 
   SplitParams p;
   fill_split_common(p, s, pr, q, k_cache, seq_len, seq_len_dev);
@@ -484,7 +499,7 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
   cudaError_t e;
   int S = 1;
   if (refresh && !no_threshold) {
-    rc = run_refresh(s, pr, q, k_cache, seq_len, seq_len_dev, n_top, tau, st, ev0, nr);
+    rc = run_refresh(s, pr, q, k_cache, seq_len, seq_len_dev, n_top, tau, st, ev0, nr, clear_status);
     if (rc) return rc;
     // the compare/gather pass reads scores, not keys: it runs with every
     // CTA slot filled (it is latency-bound on its score loads per tile)
@@ -515,6 +530,11 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
     rc = splits_for(s, pr, seq_len, NP, mode, tf, tp, &S, dense);
     if (rc) return rc;
     p.nsplit = S;
+    if (!dense) p.test_wait_ns = test_wait_ns;
+    if (clear_status) {
+      rc = clear_status_word(pr, st);
+      if (rc) return rc;
+    }
     if (ev0 != nullptr) {
       e = trace_record(ev0, st);
       if (e != cudaSuccess) return cuda_fail(e, "trace event record");
@@ -584,6 +604,11 @@ int saga_decode_step(const saga_shape* s, const void* q, const void* k_new, cons
                      sel_count, sel_idx, workspace, ws_bytes, stream, nr);
 }
 
+int saga_test_expire_next_wait(unsigned limit_ns) {
+  g_test_wait_ns = limit_ns;
+  return ok();
+}
+
 int saga_trace_next_attention(void* ev_start, void* ev_end) {
   if ((ev_start == nullptr) != (ev_end == nullptr)) return fail(SAGA_ERR_ARG, "pass both events or neither");
   g_trace_start = static_cast<cudaEvent_t>(ev_start);
@@ -601,3 +626,16 @@ int saga_get_status(const void* workspace, void* stream, unsigned* status) {
 }
 
 }  // extern "C"
+
+namespace saga {
+// saga_decode_attn that zeroes the workspace status word once the arguments
+// have been checked (used by the allocation-free entry point).
+int decode_attn_clearing_status(const saga_shape* s, const void* q, const void* k_cache, const void* v_cache,
+                                int seq_len, const int* seq_len_dev, int n_top, int refresh_interval, long long step,
+                                float* tau, void* out, int out_dtype, int* sel_count, int* sel_idx, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  return decode_impl(s, q, k_cache, v_cache, seq_len, seq_len_dev, n_top, refresh_interval, step, tau, out, out_dtype,
+                     sel_count, sel_idx, workspace, ws_bytes, stream, NewRows(), true);
+}
+}  // namespace saga
+

@@ -94,6 +94,10 @@ struct SplitParams {
   int hpv;       // query heads of the CTA per value head
   float scale;   // fp32(1/sqrt(d))
   int want_counts;
+  // failure-detection test hook: when nonzero, the epilogue of an attend
+  // launch first waits on a barrier nothing arrives at, for at most this many
+  // ns (the pipeline then unwinds and flags SAGA_STATUS_TIMEOUT)
+  unsigned test_wait_ns;
 };
 
 struct CombineParams {

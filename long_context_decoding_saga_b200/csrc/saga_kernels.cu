@@ -726,7 +726,7 @@ struct SplitSmem {
   // the ring takes 4 so that two CTAs share an SM (twice the epilogue warps
   // to hide latency, as many bytes in flight).
   static constexpr int NSTAGE_MAX = D == 128 ? 4 : 6;
-  static constexpr int FIXED = QPAD + EPI_BYTES + VST_BYTES + (2 * NSTAGE_MAX + 2 * acc_bufs<NP>() + 1) * 8 + 16 + 1024;
+  static constexpr int FIXED = QPAD + EPI_BYTES + VST_BYTES + (2 * NSTAGE_MAX + 2 * acc_bufs<NP>() + 2) * 8 + 16 + 1024;
   static constexpr int NSTAGE_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
   static constexpr int NSTAGE_HALF = (kSmemHalf - FIXED) / STAGE_BYTES;
   static constexpr bool TWO = D == 64 && NSTAGE_HALF >= 4;  // 2 x 32 KB at d = 128 measured slower
@@ -738,7 +738,7 @@ struct SplitSmem {
   static constexpr int EPI_OFF = Q_OFF + QPAD;
   static constexpr int VST_OFF = EPI_OFF + EPI_BYTES;
   static constexpr int BAR_OFF = VST_OFF + VST_BYTES;
-  static constexpr int NBARS = 2 * NSTAGE + 2 * acc_bufs<NP>() + 1;
+  static constexpr int NBARS = 2 * NSTAGE + 2 * acc_bufs<NP>() + 2;  // + fin, + the test hook's barrier
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int BYTES = MISC_OFF + 16;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
@@ -822,6 +822,7 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
   uint64_t* accf = empty + NSTAGE;
   uint64_t* acce = accf + NACC;
   uint64_t* fin = acce + NACC;
+  uint64_t* never = fin + 1;  // test hook: a barrier nothing arrives at
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM::MISC_OFF + 4);
 
@@ -847,6 +848,7 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
       mbar_init(&acce[i], 4);
     }
     mbar_init(fin, 1);
+    mbar_init(never, 1);
     mbar_init_fence();
     tma_prefetch_desc(&tmap_full);
     tma_prefetch_desc(&tmap_part);
@@ -859,6 +861,11 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     const int pend = min(pcap, pst + cap_rows);
     const uint16_t* kb = p.k_cache + (size_t)row_base * D;
     for (int r = pst; r < pend; r += kTile) prefetch_l2_bulk(kb + (size_t)r * D, (uint32_t)(min(kTile, pend - r) * D * 2));
+  } else if (warp == 2) {
+    // the group's query rows and thresholds, read right after the wait
+    const char* qg = reinterpret_cast<const char*>(p.q + ((size_t)b * p.h_q + j0) * D);
+    for (int i = lane; i < p.G * D * 2 / 128; i += 32) prefetch_l2_line(qg + 128 * i);
+    if (lane == 0 && p.tau != nullptr && !DUMP) prefetch_l2_line(p.tau + (size_t)b * p.h_q + j0);
   }
   if (UMMA && warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -988,7 +995,12 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     ListState ls{0, 0, -1, 0};
     const size_t srow = ((size_t)b * p.h_q + j0) * (size_t)p.ld_scores;
     int t = 0;
-    for (; t < ntiles; ++t) {
+    if (!DUMP && p.test_wait_ns != 0u) {
+      bool ok = __all_sync(0xffffffffu, mbar_wait(never, 0, abort_flag, p.test_wait_ns));
+      if (counting) ok = named_bar_and(1, kEpiThreads, ok);
+      if (!ok) t = -1;  // skips the tile loop; the tail drops the (empty) lists
+    }
+    for (; t >= 0 && t < ntiles; ++t) {
       float sc[NP];
       bool ok;
       {
@@ -1249,6 +1261,9 @@ __global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
       prefetch_l2_bulk(p.k_cache + ((size_t)krow + r) * D, bytes);
       prefetch_l2_bulk(p.v_cache + ((size_t)vrow + r) * D, bytes);
     }
+  } else if (warp == 2) {
+    const char* qg = reinterpret_cast<const char*>(p.q + ((size_t)b * p.h_q + j0) * D);
+    for (int i = lane; i < p.G * D * 2 / 128; i += 32) prefetch_l2_line(qg + 128 * i);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -1626,11 +1641,19 @@ __global__ void __launch_bounds__(kCombineThreads, 4) saga_combine_kernel(const 
 // Exact N-th largest per row: MSB-first 8-bit digits of the order-preserving
 // key; candidates of the current digit bin are moved to shared memory once
 // they fit, and the remaining digits are resolved there.
+// Adds one to hist[bin] for every lane with `valid` (lanes with the same bin
+// are grouped first, so each bin takes one shared-memory atomic per warp).
+// Called with warp-uniform control flow; a warp with no valid lane skips the
+// grouping.
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool valid) {
+  if (!__any_sync(0xffffffffu, valid)) return;
   const uint32_t key = valid ? bin : 0xFFFFFFFFu;
   const uint32_t peers = __match_any_sync(0xffffffffu, key);
   if (valid && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
 }
+
+// Float4 loads each thread keeps in flight in the row scans.
+constexpr int kScanUnroll = 4;
 
 // Calls f(key, valid) for every element of row[0, L) with warp-uniform trip
 // counts (so f may use full-warp primitives).  row is 16-byte aligned.
@@ -1639,13 +1662,24 @@ __device__ __forceinline__ void scan_row(const float* row, int L, F&& f) {
   const int nvec = L >> 2;
   const int nvec_pad = (nvec + 31) & ~31;
   const float4* row4 = reinterpret_cast<const float4*>(row);
-  for (int i = threadIdx.x; i < nvec_pad; i += kSelectThreads) {
-    const bool inb = i < nvec;
-    const float4 v = inb ? __ldg(row4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-    f(float_key(v.x), inb);
-    f(float_key(v.y), inb);
-    f(float_key(v.z), inb);
-    f(float_key(v.w), inb);
+  for (int i0 = threadIdx.x; i0 < nvec_pad; i0 += kSelectThreads * kScanUnroll) {
+    float4 v[kScanUnroll];
+#pragma unroll
+    for (int u = 0; u < kScanUnroll; ++u) {
+      const int i = i0 + u * kSelectThreads;
+      v[u] = i < nvec ? __ldg(row4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kScanUnroll; ++u) {
+      const int i = i0 + u * kSelectThreads;
+      if (i < nvec_pad) {  // warp-uniform (i is 32-aligned within a warp)
+        const bool inb = i < nvec;
+        f(float_key(v[u].x), inb);
+        f(float_key(v[u].y), inb);
+        f(float_key(v[u].z), inb);
+        f(float_key(v[u].w), inb);
+      }
+    }
   }
   if (threadIdx.x < 32) {
     const int i = 4 * nvec + threadIdx.x;
@@ -1777,13 +1811,25 @@ __device__ __forceinline__ void scan_range(const float* row, int begin, int end,
   const int nvec = max(0, v1 - v0);
   const int nvec_pad = (nvec + 31) & ~31;
   const float4* row4 = reinterpret_cast<const float4*>(row);
-  for (int i = threadIdx.x; i < nvec_pad; i += blockDim.x) {
-    const bool inb = i < nvec;
-    const float4 v = inb ? __ldg(row4 + v0 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-    f(float_key(v.x), inb);
-    f(float_key(v.y), inb);
-    f(float_key(v.z), inb);
-    f(float_key(v.w), inb);
+  const int nt = blockDim.x;
+  for (int i0 = threadIdx.x; i0 < nvec_pad; i0 += nt * kScanUnroll) {
+    float4 v[kScanUnroll];
+#pragma unroll
+    for (int u = 0; u < kScanUnroll; ++u) {
+      const int i = i0 + u * nt;
+      v[u] = i < nvec ? __ldg(row4 + v0 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kScanUnroll; ++u) {
+      const int i = i0 + u * nt;
+      if (i < nvec_pad) {  // warp-uniform (i is 32-aligned within a warp)
+        const bool inb = i < nvec;
+        f(float_key(v[u].x), inb);
+        f(float_key(v[u].y), inb);
+        f(float_key(v[u].z), inb);
+        f(float_key(v[u].w), inb);
+      }
+    }
   }
   if (threadIdx.x < 32) {  // the last 0..3 elements
     const int i = 4 * max(v1, v0) + threadIdx.x;

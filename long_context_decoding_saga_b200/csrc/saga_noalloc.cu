@@ -14,11 +14,19 @@
 
 #include "saga.h"
 
+namespace saga {
+int decode_attn_clearing_status(const saga_shape* s, const void* q, const void* k_cache, const void* v_cache,
+                                int seq_len, const int* seq_len_dev, int n_top, int refresh_interval, long long step,
+                                float* tau, void* out, int out_dtype, int* sel_count, int* sel_idx, void* workspace,
+                                size_t ws_bytes, void* stream);
+}
+
 namespace {
 
 // Scratch shared by every saga_decode_attn_noalloc call on a device.  It is
 // part of the library's device image: every device that loads the library
-// holds these bytes until the process exits.
+// holds these bytes until the process exits.  Its first 16 bytes hold the
+// status word (SAGA_STATUS_* bits), as at the start of a workspace.
 constexpr size_t kScratchBytes = SAGA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
@@ -33,8 +41,12 @@ std::mutex g_scratch_mu;
 
 // Device address of the scratch array for the current device.  In host code
 // the array's name only stands for the symbol, so the address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
-int scratch_for_current_device(void** out) {
+// cudaGetSymbolAddress, with that device current.  It is looked up again on
+// every call made outside stream capture (a cheap host query once the module
+// is loaded, and correct after a cudaDeviceReset has recreated the context);
+// during capture the address cached by an earlier call is used, so the first
+// call on a device must come before any capture.
+int scratch_for_current_device(cudaStream_t stream, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
@@ -45,8 +57,21 @@ int scratch_for_current_device(void** out) {
     snprintf(g_noalloc_err, sizeof(g_noalloc_err), "device ordinal %d out of range", dev);
     return SAGA_ERR_CUDA;
   }
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(stream, &cs);
+  if (e != cudaSuccess) {
+    snprintf(g_noalloc_err, sizeof(g_noalloc_err), "cudaStreamIsCapturing: %s", cudaGetErrorString(e));
+    return SAGA_ERR_CUDA;
+  }
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch[dev].ready) {
+  if (cs == cudaStreamCaptureStatusNone || !g_scratch[dev].ready) {
+    if (cs != cudaStreamCaptureStatusNone) {
+      snprintf(g_noalloc_err, sizeof(g_noalloc_err),
+               "saga_decode_attn_noalloc: first call on device %d made during stream capture; call it once before "
+               "capturing",
+               dev);
+      return SAGA_ERR_CUDA;
+    }
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
     if (e != cudaSuccess || ptr == nullptr) {
@@ -71,8 +96,9 @@ int saga_decode_attn_noalloc(const saga_shape* s, const void* q, const void* k_c
                              float* tau, void* out, int out_dtype, int* sel_count, int* sel_idx, void* stream) {
   g_noalloc_err[0] = '\0';
   const size_t need = saga_workspace_bytes(s);
-  if (need == 0) return saga_decode_attn(s, q, k_cache, v_cache, seq_len, seq_len_dev, n_top, refresh_interval, step,
-                                         tau, out, out_dtype, sel_count, sel_idx, nullptr, 0, stream);
+  if (need == 0)  // invalid shape: saga_decode_attn reports why, enqueueing nothing
+    return saga_decode_attn(s, q, k_cache, v_cache, seq_len, seq_len_dev, n_top, refresh_interval, step, tau, out,
+                            out_dtype, sel_count, sel_idx, nullptr, 0, stream);
   if (need > kScratchBytes) {
     snprintf(g_noalloc_err, sizeof(g_noalloc_err),
              "saga_decode_attn_noalloc: this shape needs %zu bytes of scratch, the built-in scratch holds %zu; "
@@ -81,16 +107,28 @@ int saga_decode_attn_noalloc(const saga_shape* s, const void* q, const void* k_c
     return SAGA_ERR_WORKSPACE;
   }
   void* scratch = nullptr;
-  int rc = scratch_for_current_device(&scratch);
+  int rc = scratch_for_current_device(static_cast<cudaStream_t>(stream), &scratch);
   if (rc != SAGA_OK) return rc;
-  // the status word is the only part a call reads before writing it
-  cudaError_t e = cudaMemsetAsync(scratch, 0, 16, static_cast<cudaStream_t>(stream));
+  // every argument is checked before anything is enqueued; the status word
+  // (the only part of the scratch a call reads before writing it) is then
+  // cleared on the stream ahead of the kernels
+  return saga::decode_attn_clearing_status(s, q, k_cache, v_cache, seq_len, seq_len_dev, n_top, refresh_interval, step,
+                                           tau, out, out_dtype, sel_count, sel_idx, scratch, kScratchBytes, stream);
+}
+
+int saga_noalloc_get_status(void* stream, unsigned* status) {
+  g_noalloc_err[0] = '\0';
+  if (status == nullptr) {
+    snprintf(g_noalloc_err, sizeof(g_noalloc_err), "status is NULL");
+    return SAGA_ERR_ARG;
+  }
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(status, g_noalloc_scratch, sizeof(unsigned), 0, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) {
-    snprintf(g_noalloc_err, sizeof(g_noalloc_err), "cudaMemsetAsync(status): %s", cudaGetErrorString(e));
+    snprintf(g_noalloc_err, sizeof(g_noalloc_err), "saga_noalloc_get_status: %s", cudaGetErrorString(e));
     return SAGA_ERR_CUDA;
   }
-  return saga_decode_attn(s, q, k_cache, v_cache, seq_len, seq_len_dev, n_top, refresh_interval, step, tau, out,
-                          out_dtype, sel_count, sel_idx, scratch, kScratchBytes, stream);
+  return SAGA_OK;
 }
 
 const char* saga_noalloc_last_error(void) {

@@ -29,7 +29,8 @@ SAGA_STATUS_TIMEOUT = 0x2
 
 EXPORTED = ("saga_workspace_bytes", "saga_kv_append", "atopn_refresh_threshold", "atopn_select_workspace_bytes",
             "atopn_select_threshold", "saga_decode_attn", "saga_trace_next_attention", "saga_get_status", "saga_last_error", "saga_abi_version",
-            "saga_noalloc_scratch_bytes", "saga_decode_attn_noalloc", "saga_noalloc_last_error", "saga_decode_step")
+            "saga_noalloc_scratch_bytes", "saga_decode_attn_noalloc", "saga_noalloc_get_status",
+            "saga_noalloc_last_error", "saga_decode_step", "saga_test_expire_next_wait")
 
 
 class SagaError(RuntimeError):
@@ -94,6 +95,10 @@ def load(path: Optional[str] = None):
     lib.saga_decode_attn_noalloc.argtypes = [sp, _P, _P, _P, _I, _P, _I, _I, ctypes.c_longlong, _P, _P, _I, _P, _P,
                                              _P]
     lib.saga_decode_attn_noalloc.restype = _I
+    lib.saga_noalloc_get_status.argtypes = [_P, ctypes.POINTER(ctypes.c_uint)]
+    lib.saga_noalloc_get_status.restype = _I
+    lib.saga_test_expire_next_wait.argtypes = [ctypes.c_uint]
+    lib.saga_test_expire_next_wait.restype = _I
     lib.saga_noalloc_last_error.argtypes = []
     lib.saga_noalloc_last_error.restype = ctypes.c_char_p
     _lib = lib
@@ -278,6 +283,22 @@ def saga_decode_attn_noalloc(shape: SagaShape, q, k_cache, v_cache, seq_len: int
                                       _ptr(out), out_dtype, _ptr(sel_count), _ptr(sel_idx), _stream(stream))
     if rc != SAGA_OK:
         raise SagaError(rc, lib.saga_noalloc_last_error().decode(errors="replace"))
+
+
+def saga_noalloc_get_status(stream=None) -> int:
+    """Status word (SAGA_STATUS_* bits) of the last saga_decode_attn_noalloc call on the current device."""
+    lib = load()
+    v = ctypes.c_uint(0)
+    rc = lib.saga_noalloc_get_status(_stream(stream), ctypes.byref(v))
+    if rc != SAGA_OK:
+        raise SagaError(rc, lib.saga_noalloc_last_error().decode(errors="replace"))
+    return int(v.value)
+
+
+def saga_test_expire_next_wait(limit_ns: int):
+    """Test hook: the next decode call's keep kernel (a sparse reuse step) waits on a barrier nothing arrives
+    at, for at most limit_ns, then unwinds and flags SAGA_STATUS_TIMEOUT (0 cancels)."""
+    _check(load().saga_test_expire_next_wait(int(limit_ns)))
 
 
 def saga_get_status(workspace, stream=None) -> int:

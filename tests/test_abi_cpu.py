@@ -31,7 +31,7 @@ def test_header_declares_the_binding_names():
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.saga_abi_version() == 100
+    assert lib.saga_abi_version() == 101
 
 
 def _shape(**kw):
