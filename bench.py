@@ -16,8 +16,15 @@ Printed JSON (rank 0, one line):
                pinned host memory and every layer's output copied back,
                inside the timed region
   roofline     the context-split attention kernel: algorithmic bytes of one
-               layer-step / its mean CUDA-event duration vs the measured HBM
-               copy bandwidth
+               layer-step / its in-step time (the reuse step's time per
+               layer, shared with the combine in proportion to their
+               CUDA-event durations measured in isolation, which are also
+               reported) vs the measured HBM copy bandwidth, and vs the
+               pure-read ceiling of the library's read probe
+  read_probe   that ceiling: one streaming read of 4 GiB, best of 5
+  workloads    (N=1) the other configurations, timed the same way with a
+               short window each: Llama-SAGA 32K, dense GQA 128K and the
+               128K sweep points at batch 1/4/16 with 1 and 8 key heads
   cpu_baseline the CPU oracle on a bounded sample (rank 0, N=1)
 
 Algorithmic bytes of one layer-step:
@@ -35,7 +42,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -265,6 +271,14 @@ def combine_rank_stats(per_rank, steps):
             "e2e_value": e_total / (e_ms / 1e3) / 1e9 if e_ms > 0 else None}
 
 
+def workload_config(wl, world):
+    """The `config` object of the JSON line: the workload and its shape, identical for both arms (the
+    run-specific window and L2 handling go in a separate `window` object)."""
+    return {"workload": wl.name, "batch_per_gpu": wl.batch, "l_kv": wl.l_kv, "h_q": wl.h_q, "h_k": wl.h_k,
+            "h_v": wl.h_v, "d": wl.d, "n_top": wl.n_top if not wl.dense else "dense", "refresh": wl.refresh,
+            "layers": wl.layers, "parallelism": f"replicas{world}"}
+
+
 def run_reference(args, wl, rank, world):
     if rank != 0:
         return 0
@@ -286,37 +300,28 @@ def run_reference(args, wl, rank, world):
     total = sum(times)
     value = nbytes / total / 1e9
     cores = oracle_threads()
+    sample = (f"each timed step: one decode step of layer 0 of the workload at full size (a bounded sample of "
+              f"the {wl.layers}-layer step; ms_per_step is that one layer-step as timed), numpy oracle")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3 * wl.layers, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": wl.batch, "l_kv": wl.l_kv, "h_q": wl.h_q, "h_k": wl.h_k,
-                   "h_v": wl.h_v, "d": wl.d, "n_top": wl.n_top, "refresh": wl.refresh, "layers": wl.layers},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": "each step: one decode step of layer 0 at full size (ms_per_step scaled to all "
-                                   "layers)"},
+        "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3, "timed_unit": "one layer-step (layer 0)",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, world),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def run_saga(args, wl, rank, world, local_rank):
+def make_session(wl, dev, rank, total_steps):
+    """A DecodeSession holding every layer of `wl` (caches prefilled with the seeded synthetic rows, one
+    rank's seed per rank) and the per-step inputs of `total_steps` decode steps, stacked [steps, layers, ...]."""
     import torch
-    import torch.distributed as dist
 
-    from long_context_decoding_saga_b200 import build as build_mod
     from long_context_decoding_saga_b200 import saga, workload
     from long_context_decoding_saga_b200.session import DecodeSession
 
-    build_mod.build()
-    saga.load()
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-
-    W, K = args.warmup, args.steps
-    plan = step_plan(W, K, wl.refresh, not args.no_e2e)
-    A, E, A2, T, total_steps = plan["A"], plan["E"], plan["A2"], plan["T"], plan["total"]
     l_cap = wl.l_kv + total_steps
     n_top = wl.n_for_kernel(l_cap)
     shape = saga.SagaShape.of(wl.batch, wl.h_q, wl.h_k, wl.h_v, wl.d, l_cap)
@@ -334,6 +339,186 @@ def run_saga(args, wl, rank, world, local_rank):
     v_all = torch.stack(vs, dim=1)
     del qs, ks, vs
     torch.cuda.synchronize()
+    return sess, (q_all, k_all, v_all), shape, n_top, l_cap
+
+
+def l2_flush_wanted(wl, mode, l2_bytes):
+    """Whether timed steps get a 2 x L2 write between them: a step whose streamed bytes are under twice the
+    L2 would find part of its inputs still in L2 from the step before."""
+    step_bytes = wl.layers * layer_bytes(wl, wl.l_kv)
+    return mode == "on" or (mode == "auto" and step_bytes < 2 * l2_bytes), step_bytes
+
+
+def l2_note(flush, step_bytes, l2_bytes):
+    if flush:
+        return "flushed between timed steps (a 2 x L2 write outside each step's events)"
+    if step_bytes >= 2 * l2_bytes:
+        return "inputs exceed twice the L2 (all layers' caches cycle through L2 each step)"
+    return "inputs fit in twice the L2; not flushed (--flush-l2 off)"
+
+
+def timed_window(sess, inputs, cur, K, wl, flush, scratch):
+    """K decode steps (graph replays), each bracketed by CUDA events: back to back (the end mark of one step
+    starts the next) or, with `flush`, one by one with the L2 write outside the events.  Returns per-step
+    ms, which steps refreshed, the algorithmic bytes and the next input index."""
+    import torch
+    q_all, k_all, v_all = inputs
+    marks = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    kinds, nbytes = [], 0
+    for s_i in range(K):
+        nbytes += wl.layers * layer_bytes(wl, sess.length + 1)
+        kinds.append(sess.t % wl.refresh == 0)
+        if flush or s_i == 0:
+            marks[s_i][0].record()
+        sess.stage(q_all[cur], k_all[cur], v_all[cur])
+        sess.replay()
+        marks[s_i][1].record()
+        if flush:
+            scratch.fill_(float(s_i))
+        cur += 1
+    torch.cuda.synchronize()
+    step_ms = []
+    for s_i in range(K):
+        start_ev = marks[s_i][0] if (flush or s_i == 0) else marks[s_i - 1][1]
+        step_ms.append(start_ev.elapsed_time(marks[s_i][1]))
+    return step_ms, kinds, nbytes, cur
+
+
+def read_peak_probe(dev, gib=4, repeats=5):
+    """The pure-read HBM ceiling: the library's read probe over a 4 GiB buffer (32 x the L2), best of
+    `repeats` CUDA-event timings."""
+    import torch
+
+    from long_context_decoding_saga_b200 import saga
+    buf = torch.empty(gib << 30, dtype=torch.uint8, device=dev)
+    buf.fill_(1)
+    sink = saga.read_probe(buf)  # warm-up
+    best = None
+    for _ in range(repeats):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        saga.read_probe(buf, sink)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        best = ms if best is None else min(best, ms)
+    del buf
+    return {"gbs": (gib << 30) / (best / 1e3) / 1e9, "bytes": gib << 30, "best_ms": best, "repeats": repeats,
+            "kernel": "saga_read_probe (16-byte streaming loads, 4 in flight per thread)"}
+
+
+# Workloads timed after the headline, in the same process, each with a short window: the Llama-shaped SAGA
+# configuration at 32K, the dense GQA configuration at 128K, and the 128K sweep points at batch 1, 4 and 16
+# with 1 and 8 key heads (N = 256, R = 16).  The batch-4/16 points hold fewer layers (their caches are
+# 0.6-4.3 GB per layer); every entry says how many it ran.
+EXTRA_WORKLOADS = (
+    ("llama3.2-1b_saga_32k", 0),
+    ("llama3.2-1b_dense_gqa_128k", 0),
+    ("sweep_l131072_b1_hk1_n256_r16", 0),
+    ("sweep_l131072_b1_hk8_n256_r16", 0),
+    ("sweep_l131072_b4_hk1_n256_r16", 8),
+    ("sweep_l131072_b4_hk8_n256_r16", 8),
+    ("sweep_l131072_b16_hk1_n256_r16", 4),
+    ("sweep_l131072_b16_hk8_n256_r16", 4),
+)
+
+
+def time_extra_workload(wl, dev, rank, args, peak, l2_bytes):
+    """One entry of the `workloads` object: graph-replayed decode steps of `wl` (K = max(16, R) when R is
+    at most 64, so the window holds refresh and reuse steps in their proportion), inputs resident."""
+    import torch
+    W = 3
+    K = wl.refresh if wl.refresh <= 64 and wl.refresh > 16 else 16
+    plan = step_plan(W, K, wl.refresh, e2e=False)
+    sess, inputs, _, _, _ = make_session(wl, dev, rank, plan["total"])
+    q_all, k_all, v_all = inputs
+    sess.step(q_all[0], k_all[0], v_all[0])
+    sess.capture(torch.cuda.Stream(dev))
+    cur = 1
+    for _ in range(W + plan["A"]):
+        sess.stage(q_all[cur], k_all[cur], v_all[cur])
+        sess.replay()
+        cur += 1
+    torch.cuda.synchronize()
+    flush, step_bytes = l2_flush_wanted(wl, args.flush_l2, l2_bytes)
+    scratch = torch.empty(2 * l2_bytes // 4, dtype=torch.float32, device=dev) if flush else None
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
+    step_ms, kinds, nbytes, cur = timed_window(sess, inputs, cur, K, wl, flush, scratch)
+    clocks = sampler.stop()
+    ms = sum(step_ms)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    entry = {"layers": wl.layers, "batch": wl.batch, "h_k": wl.h_k, "l_kv": wl.l_kv,
+             "n_top": wl.n_top if not wl.dense else "dense", "refresh": wl.refresh, "steps": K,
+             "refresh_steps": int(sum(kinds)), "us_per_step": ms / K * 1e3, "gb_s": gbs, "frac": gbs / peak,
+             "step_us": step_means(step_ms, kinds, wl.refresh), "l2": l2_note(flush, step_bytes, l2_bytes),
+             "clocks": clocks, "status_word": None}
+    from long_context_decoding_saga_b200 import saga
+    entry["status_word"] = saga.saga_get_status(sess.workspace)
+    del sess, inputs, q_all, k_all, v_all, scratch
+    torch.cuda.empty_cache()
+    return entry
+
+
+def kernel_timing(sess, shape, n_top, wl, inputs, cur, T, stream):
+    """Per-layer durations of the context-split attention kernel and of the cross-split combine on reuse
+    steps, each bracketed by CUDA events on the launching stream inside a freshly recorded graph (the events
+    serialise the kernels: these are isolated durations, without the launch overlap of the real step)."""
+    import torch
+
+    from long_context_decoding_saga_b200 import saga
+    q_all, k_all, v_all = inputs
+    split_ms, comb_ms = [], []
+    if wl.refresh <= 1 or T <= 0:
+        return split_ms, comb_ms, cur
+    # per layer: start of the split kernel, end of the split kernel = start of the combine; the combine of
+    # layer i ends where layer i + 1's split kernel starts (nothing else runs in between)
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(2)) for _ in range(wl.layers)]
+    g = torch.cuda.CUDAGraph()
+    L_est = sess.length + 1
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        sess.seq_len_dev.add_(1)
+        for i in range(wl.layers):
+            saga.saga_trace_next_attention(evs[i][0], evs[i][1])
+            saga.saga_decode_step(shape, sess.q_buf[i], sess.k_buf[i], sess.v_buf[i], sess.k_cache[i],
+                                  sess.v_cache[i], L_est, n_top, wl.refresh, 1, sess.tau[i], sess.out[i],
+                                  sess.workspace, seq_len_dev=sess.seq_len_dev)
+    sess.seq_len_dev.fill_(sess.length)
+    for _ in range(T):
+        sess.stage(q_all[cur], k_all[cur], v_all[cur])
+        if sess.t % wl.refresh == 0:  # keep the refresh schedule: refresh steps run with the step graphs
+            sess.replay()
+            cur += 1
+            continue
+        g.replay()
+        sess.length += 1
+        sess.t += 1
+        cur += 1
+        torch.cuda.synchronize()
+        split_ms.extend(a.elapsed_time(b) for a, b in evs)
+        comb_ms.extend(evs[i][1].elapsed_time(evs[i + 1][0]) for i in range(wl.layers - 1))
+    del g
+    return split_ms, comb_ms, cur
+
+
+def run_saga(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from long_context_decoding_saga_b200 import build as build_mod
+    from long_context_decoding_saga_b200 import saga, workload
+
+    build_mod.build()
+    saga.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+
+    W, K = args.warmup, args.steps
+    plan = step_plan(W, K, wl.refresh, not args.no_e2e)
+    A, E, A2, T = plan["A"], plan["E"], plan["A2"], plan["T"]
+    sess, inputs, shape, n_top, l_cap = make_session(wl, dev, rank, plan["total"])
+    q_all, k_all, v_all = inputs
 
     # step 0 eagerly (warms launch attributes), then record the step graphs
     sess.step(q_all[0], k_all[0], v_all[0])
@@ -353,52 +538,25 @@ def run_saga(args, wl, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    # L2: a step whose streamed bytes are under twice the L2 would find part of
-    # its inputs still in L2 from the step before, so such steps are timed one
-    # by one with a 2 x L2 write between them, outside their events
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
-    step_bytes = wl.layers * layer_bytes(wl, wl.l_kv)
-    flush = args.flush_l2 == "on" or (args.flush_l2 == "auto" and step_bytes < 2 * l2_bytes)
+    flush, step_bytes = l2_flush_wanted(wl, args.flush_l2, l2_bytes)
     scratch = torch.empty(2 * l2_bytes // 4, dtype=torch.float32, device=dev) if flush else None
     sampler = ClockSampler(dev.index if dev.index is not None else local_rank)
     sampler.start()
-    marks = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    bytes_timed = 0
-    refresh_steps = 0
-    kinds = []
     torch.cuda.nvtx.range_push("bench_timed")
-    for s_i in range(K):
-        L = sess.length + 1
-        bytes_timed += wl.layers * layer_bytes(wl, L)
-        kinds.append(sess.t % wl.refresh == 0)
-        refresh_steps += int(kinds[-1])
-        if flush or s_i == 0:
-            marks[s_i][0].record()
-        sess.stage(q_all[cur], k_all[cur], v_all[cur])
-        sess.replay()
-        marks[s_i][1].record()
-        if flush:
-            scratch.fill_(float(s_i))
-        cur += 1
+    step_ms, kinds, bytes_timed, cur = timed_window(sess, inputs, cur, K, wl, flush, scratch)
     torch.cuda.nvtx.range_pop()
-    torch.cuda.synchronize()
     clocks = sampler.stop()
-    # per-step durations: each step's own events when flushing, else from the
-    # previous step's end mark (back-to-back steps)
-    step_ms = []
-    for s_i in range(K):
-        start_ev = marks[s_i][0] if (flush or s_i == 0) else marks[s_i - 1][1]
-        step_ms.append(start_ev.elapsed_time(marks[s_i][1]))
     ms = sum(step_ms)
     step_stats = step_means(step_ms, kinds, wl.refresh)
-    if flush:
-        del scratch
+    refresh_steps = int(sum(kinds))
+    del scratch
     launches = refresh_steps * sess.launches_per_step(True) + (K - refresh_steps) * sess.launches_per_step(False)
     if world > 1:
         dist.barrier()
 
     # end to end: pinned host inputs in, every layer's output out, inside the timed region
-    e2e = None
+    e2e, e_bytes = None, 0
     if E > 0:
         replay_range(A2)
         hq = [q_all[cur + s].cpu().pin_memory() for s in range(E)]
@@ -408,7 +566,6 @@ def run_saga(args, wl, rank, world, local_rank):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        e_bytes = 0
         e_refresh = 0
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record()
@@ -427,44 +584,15 @@ def run_saga(args, wl, rank, world, local_rank):
         e2e = {"value": e_bytes / (e_ms / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / E, "steps": E, "refresh_steps": e_refresh}
 
-    # dominant kernel: the split-context attention kernel of reuse steps (with the fused append),
-    # bracketed by CUDA events on its stream inside a freshly recorded graph (one event pair per layer;
-    # the events serialise the kernels, so this is the kernel's own duration without launch overlap)
-    kernel_ms = []
-    if wl.refresh > 1 and T > 0:
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(wl.layers)]
-        g = torch.cuda.CUDAGraph()
-        L_est = sess.length + 1
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g, stream=stream):
-            sess.seq_len_dev.add_(1)
-            for i in range(wl.layers):
-                saga.saga_trace_next_attention(*evs[i])
-                saga.saga_decode_step(shape, sess.q_buf[i], sess.k_buf[i], sess.v_buf[i], sess.k_cache[i],
-                                      sess.v_cache[i], L_est, n_top, wl.refresh, 1, sess.tau[i], sess.out[i],
-                                      sess.workspace, seq_len_dev=sess.seq_len_dev)
-        sess.seq_len_dev.fill_(sess.length)
-        for _ in range(T):
-            if sess.t % wl.refresh == 0:  # keep the refresh schedule: run refresh steps with the step graphs
-                sess.stage(q_all[cur], k_all[cur], v_all[cur])
-                sess.replay()
-                cur += 1
-                continue
-            sess.stage(q_all[cur], k_all[cur], v_all[cur])
-            g.replay()
-            sess.length += 1
-            sess.t += 1
-            cur += 1
-            torch.cuda.synchronize()
-            kernel_ms.extend(a.elapsed_time(b) for a, b in evs)
-        del g
+    # dominant kernel: the split-context attention kernel of reuse steps (with the fused append) and the
+    # combine after it, isolated durations
+    split_ms, comb_ms, cur = kernel_timing(sess, shape, n_top, wl, inputs, cur, T, stream)
     # kept-count statistics of the last step (layer 0), from one untimed call with index lists; it
     # rewrites that layer's output and threshold with the same values and leaves the caches alone
     kept = None
     try:
-        B_, hq_ = wl.batch, wl.h_q
-        cnt = torch.zeros((B_, hq_), dtype=torch.int32, device=dev)
-        idx = torch.zeros((B_, hq_, l_cap), dtype=torch.int32, device=dev)
+        cnt = torch.zeros((wl.batch, wl.h_q), dtype=torch.int32, device=dev)
+        idx = torch.zeros((wl.batch, wl.h_q, l_cap), dtype=torch.int32, device=dev)
         saga.saga_decode_attn(shape, sess.q_buf[0], sess.k_cache[0], sess.v_cache[0], sess.length, n_top,
                               wl.refresh, sess.t - 1, sess.tau[0], sess.out[0], sess.workspace, sel_count=cnt,
                               sel_idx=idx)
@@ -475,6 +603,7 @@ def run_saga(args, wl, rank, world, local_rank):
     except Exception as exc:  # noqa: BLE001  (reported, never fatal to the benchmark line)
         kept = {"error": str(exc)[:200]}
     status = saga.saga_get_status(sess.workspace)
+    L_mid = sess.length
 
     # ---- gather over ranks (every rank takes part, whatever it measured)
     local = {"ms": ms, "bytes": bytes_timed, "e2e_ms": e2e["ms_per_step"] * E if e2e else 0.0,
@@ -482,31 +611,41 @@ def run_saga(args, wl, rank, world, local_rank):
     job = combine_rank_stats(gather_rank_stats(local, world), K)
     if rank != 0:
         return 0
+    del sess, inputs, q_all, k_all, v_all
+    torch.cuda.empty_cache()
     value = job["value"]
     ms_per_step = job["ms_per_step"]
     peak, peak_kind = load_peak()
+    read = read_peak_probe(dev)
     roofline = None
-    if kernel_ms:
-        k_mean = statistics.mean(kernel_ms)
-        L_mid = sess.length
-        achieved = layer_bytes(wl, L_mid) / (k_mean / 1e3) / 1e9
+    if split_ms and comb_ms and step_stats.get("reuse_mean_us"):
+        # in-step time of the split kernel: the reuse step's time per layer, shared between the split kernel
+        # and the combine in proportion to their isolated durations (in the step they overlap through
+        # programmatic dependent launch, so the isolated durations add up to more than the step)
+        s_mean, c_mean = statistics.mean(split_ms), statistics.mean(comb_ms)
+        share = s_mean / (s_mean + c_mean)
+        k_in_step = step_stats["reuse_mean_us"] / wl.layers * share
+        nbytes = layer_bytes(wl, L_mid)
+        achieved = nbytes / (k_in_step / 1e6) / 1e9
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                     "traffic": load_traffic(wl.name), "kernel": "saga_split_kernel (reuse step, per layer)",
-                    "kernel_us_mean": k_mean * 1e3, "launches_timed": len(kernel_ms), "peak_kind": peak_kind}
+                    "kernel_us_mean": k_in_step, "kernel_us_serialized": s_mean * 1e3,
+                    "combine_us_serialized": c_mean * 1e3, "share_of_layer": share,
+                    "achieved_serialized": nbytes / (s_mean / 1e3) / 1e9, "bytes_per_launch": nbytes,
+                    "launches_timed": len(split_ms), "peak_kind": peak_kind,
+                    "read_peak": read["gbs"], "frac_of_read_peak": achieved / read["gbs"]}
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "l_kv": wl.l_kv, "h_q": wl.h_q, "h_k": wl.h_k,
-                   "h_v": wl.h_v, "d": wl.d, "n_top": wl.n_top if not wl.dense else "dense", "refresh": wl.refresh,
-                   "layers": wl.layers, "parallelism": f"replicas{world}",
-                   "l2": ("flushed between timed steps (a 2 x L2 write outside each step's events)" if flush
-                          else "inputs exceed twice the L2 (all layers' caches cycle through L2 each step)"
-                          if step_bytes >= 2 * l2_bytes else "inputs fit in twice the L2; not flushed (--flush-l2 off)"),
-                   "refresh_steps_timed": refresh_steps, "alignment_steps": A},
+        "config": workload_config(wl, world),
+        "window": {"l2": l2_note(flush, step_bytes, l2_bytes), "refresh_steps_timed": refresh_steps,
+                   "alignment_steps": A},
         "step_us": step_stats,
+        "frac_of_peak": value / peak,
         "kept": kept,
         "roofline": roofline,
+        "read_probe": read,
         "e2e": ({"value": job["e2e_value"], "unit": "GB/s",
                  "h2d_bytes_per_step": e2e["h2d_bytes_per_step"] * world,
                  "d2h_bytes_per_step": e2e["d2h_bytes_per_step"] * world, "steps": e2e["steps"],
@@ -515,6 +654,17 @@ def run_saga(args, wl, rank, world, local_rank):
         "clocks": clocks,
         "status_word": status,
     }
+    if world == 1 and not args.no_extra:
+        extras = {}
+        for name, layers in EXTRA_WORKLOADS:
+            ewl = workload.by_name(name)
+            if layers:
+                ewl = ewl.with_(layers=layers)
+            try:
+                extras[name] = time_extra_workload(ewl, dev, 0, args, peak, l2_bytes)
+            except Exception as exc:  # noqa: BLE001  (reported, never fatal to the benchmark line)
+                extras[name] = {"error": str(exc)[:300]}
+        line["workloads"] = extras
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line), flush=True)
@@ -530,6 +680,8 @@ def main():
     ap.add_argument("--workload", default="qwen2.5-1.5b_saga_128k")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the extra workloads timed after the headline (the `workloads` object)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
     ap.add_argument("--flush-l2", default="auto", choices=["auto", "on", "off"],
                     help="write 2 x L2 between timed steps (auto: when a step streams less than 2 x L2)")

@@ -210,6 +210,17 @@ SAGA_API const char* saga_noalloc_last_error(void);
  * call whatever its kind; limit_ns = 0 cancels a pending request. */
 SAGA_API int saga_test_expire_next_wait(unsigned limit_ns);
 
+/* Measurement aid (no counterpart in the paper): one streaming read of
+ * `bytes` of device memory at buf (16-byte aligned; the last bytes % 16 are
+ * not read), 16-byte loads with four in flight per thread over a grid of up
+ * to four CTAs per SM.  Timed by the caller (events on `stream`), it gives
+ * the pure-read HBM ceiling that the read-dominated attention kernels are
+ * held to.  sink: device array of at least saga_read_probe_sink_words()
+ * words (written, so no load is dropped).  Errors: SAGA_ERR_ARG for a NULL
+ * or misaligned pointer or bytes < 16, SAGA_ERR_CUDA for a launch error. */
+SAGA_API size_t saga_read_probe_sink_words(void);
+SAGA_API int saga_read_probe(const void* buf, size_t bytes, unsigned* sink, void* stream);
+
 /* Reads the workspace status word (SAGA_STATUS_* bits ORed by the kernels
  * since the workspace was zeroed) after synchronizing `stream`. */
 SAGA_API int saga_get_status(const void* workspace, void* stream, unsigned* status);

@@ -30,7 +30,8 @@ SAGA_STATUS_TIMEOUT = 0x2
 EXPORTED = ("saga_workspace_bytes", "saga_kv_append", "atopn_refresh_threshold", "atopn_select_workspace_bytes",
             "atopn_select_threshold", "saga_decode_attn", "saga_trace_next_attention", "saga_get_status", "saga_last_error", "saga_abi_version",
             "saga_noalloc_scratch_bytes", "saga_decode_attn_noalloc", "saga_noalloc_get_status",
-            "saga_noalloc_last_error", "saga_decode_step", "saga_test_expire_next_wait")
+            "saga_noalloc_last_error", "saga_decode_step", "saga_test_expire_next_wait", "saga_read_probe_sink_words",
+            "saga_read_probe")
 
 
 class SagaError(RuntimeError):
@@ -99,6 +100,10 @@ def load(path: Optional[str] = None):
     lib.saga_noalloc_get_status.restype = _I
     lib.saga_test_expire_next_wait.argtypes = [ctypes.c_uint]
     lib.saga_test_expire_next_wait.restype = _I
+    lib.saga_read_probe_sink_words.argtypes = []
+    lib.saga_read_probe_sink_words.restype = ctypes.c_size_t
+    lib.saga_read_probe.argtypes = [_P, ctypes.c_size_t, _P, _P]
+    lib.saga_read_probe.restype = _I
     lib.saga_noalloc_last_error.argtypes = []
     lib.saga_noalloc_last_error.restype = ctypes.c_char_p
     _lib = lib
@@ -299,6 +304,20 @@ def saga_test_expire_next_wait(limit_ns: int):
     """Test hook: the next decode call's keep kernel (a sparse reuse step) waits on a barrier nothing arrives
     at, for at most limit_ns, then unwinds and flags SAGA_STATUS_TIMEOUT (0 cancels)."""
     _check(load().saga_test_expire_next_wait(int(limit_ns)))
+
+
+def read_probe(buf: torch.Tensor, sink: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One streaming read of buf (any CUDA tensor, 16-byte aligned) by the library's pure-read probe kernel;
+    returns the sink tensor it writes (pass it back in to reuse it)."""
+    if not buf.is_cuda:
+        raise ValueError("buf must be a CUDA tensor")
+    lib = load()
+    if sink is None:
+        sink = torch.empty(int(lib.saga_read_probe_sink_words()), dtype=torch.int32, device=buf.device)
+    rc = lib.saga_read_probe(_ptr(buf), buf.numel() * buf.element_size(), _ptr(sink), _stream(stream))
+    if rc != SAGA_OK:
+        raise SagaError(rc, "saga_read_probe failed")
+    return sink
 
 
 def saga_get_status(workspace, stream=None) -> int:

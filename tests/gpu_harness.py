@@ -225,3 +225,80 @@ def check_full_sampled(wl, got, inputs, n_top, track):
             mism = (keep_g != res["keep"]) & far
             assert not mism.any(), f"layer {i} step {t}: {int(mism.sum())} index mismatches outside the band"
     return worst
+
+
+# ---------------------------------------------------------------------------- full-size parity, every layer and step
+def layer_inputs_on_gpu(wl, steps):
+    """Every layer's inputs, drawn with the seeded generator on the CPU (so that a worker process can draw
+    the same bytes again) and moved to the GPU."""
+    layers = []
+    for i in range(wl.layers):
+        inp = workload.make_layer(wl, i, device="cpu", steps=steps)
+        layers.append({k: v.cuda() for k, v in inp.items()})
+        del inp
+    return layers
+
+
+def run_full_all(wl, inputs, steps, track=False, record_idx=False):
+    """All layers of `wl` per step through CUDA-graph replays with a device-side length (the benchmark's
+    launch configuration) for `steps` steps.  Returns, per layer, per step: out, tau and (track) the kept
+    counts and (record_idx) each row's kept positions."""
+    l_cap = wl.l_kv + steps
+    n_top = wl.n_for_kernel(l_cap)
+    shape = saga.SagaShape.of(wl.batch, wl.h_q, wl.h_k, wl.h_v, wl.d, l_cap)
+    sess = DecodeSession(shape, wl.layers, n_top, wl.refresh, device="cuda", track_selection=track)
+    for i, inp in enumerate(inputs):
+        sess.prefill(i, inp["K0"], inp["V0"])
+    q_all = torch.stack([inp["q"] for inp in inputs], 1)
+    k_all = torch.stack([inp["k_new"] for inp in inputs], 1)
+    v_all = torch.stack([inp["v_new"] for inp in inputs], 1)
+    per_layer = [[None] * steps for _ in range(wl.layers)]
+    H = wl.batch * wl.h_q
+
+    def grab(t):
+        torch.cuda.synchronize()
+        out = sess.out.float().cpu().numpy()
+        tau = sess.tau.cpu().numpy()
+        cnt = sess.sel_count.cpu().numpy() if track else None
+        idx = None
+        if record_idx:
+            m = max(1, int(cnt.max()))
+            idx = sess.sel_idx[..., :m].cpu().numpy()
+        for i in range(wl.layers):
+            row = {"out": out[i], "tau": tau[i]}
+            if track:
+                row["count"] = cnt[i]
+            if record_idx:
+                flat_c = cnt[i].reshape(H)
+                flat_i = idx[i].reshape(H, -1)
+                row["idx"] = [flat_i[r, :flat_c[r]].copy() for r in range(H)]
+            per_layer[i][t] = row
+
+    sess.step(q_all[0], k_all[0], v_all[0])  # step 0 eagerly, then the step graphs (as the benchmark does)
+    sess.capture()
+    grab(0)
+    for t in range(1, steps):
+        sess.stage(q_all[t], k_all[t], v_all[t])
+        sess.replay()
+        grab(t)
+    status = saga.saga_get_status(sess.workspace)
+    assert status & saga.SAGA_STATUS_TIMEOUT == 0
+    del sess
+    return per_layer, n_top, l_cap
+
+
+def check_full_all(wl, per_layer, n_top, l_cap, steps, workers=None):
+    """Every layer against the stepping oracle, one layer per worker process (spawned: the parent holds a
+    CUDA context).  Returns the workers' summaries."""
+    import concurrent.futures
+    import multiprocessing
+    import os
+    cores = len(os.sched_getaffinity(0))
+    workers = workers or max(1, min(wl.layers, cores // 2, 16))
+    threads = max(1, cores // workers)
+    from tests import fullsize_oracle
+    tasks = [{"wl": wl, "layer": i, "steps": steps, "n_top": n_top, "l_cap": l_cap, "gpu": per_layer[i],
+              "threads": threads} for i in range(wl.layers)]
+    ctx = multiprocessing.get_context("spawn")
+    with concurrent.futures.ProcessPoolExecutor(max_workers=workers, mp_context=ctx) as ex:
+        return list(ex.map(fullsize_oracle.check_layer, tasks))

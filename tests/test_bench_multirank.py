@@ -71,3 +71,9 @@ def test_reference_arm_prints_one_line():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+    # the same `config` object as the CUDA arm prints for this workload, and the time of what it ran
+    sys.path.insert(0, ROOT)
+    import bench
+    from long_context_decoding_saga_b200 import workload
+    assert line["config"] == bench.workload_config(workload.by_name("tiny_1k"), 1)
+    assert line["timed_unit"] == "one layer-step (layer 0)"

@@ -307,3 +307,18 @@ def test_refresh_select_heavy_bin_falls_back():
     assert (cnt.cpu().numpy() == res["keep"].sum(-1)).all()  # every tied token kept (more than N)
     assert int(cnt[0, 0]) > 16384
     assert np.max(np.abs(out.cpu().numpy() - res["out"])) <= gpu_harness.OUT_TOL
+
+
+def test_read_probe_reads_every_word():
+    """The pure-read probe touches every 16-byte chunk: the XOR of its per-CTA sink words equals the XOR of
+    all 32-bit words of the buffer (a length that is not a multiple of the grid stride)."""
+    g = torch.Generator(device="cuda").manual_seed(9)
+    n_words = (37 << 20) // 4 + 4 * 1237
+    buf = torch.randint(-(1 << 31), (1 << 31) - 1, (n_words,), generator=g, device="cuda", dtype=torch.int64)
+    buf = buf.to(torch.int32)
+    sink = torch.zeros(saga.load().saga_read_probe_sink_words(), dtype=torch.int32, device="cuda")
+    saga.read_probe(buf, sink)
+    torch.cuda.synchronize()
+    expect = np.bitwise_xor.reduce(buf.cpu().numpy().view(np.uint32))
+    got = np.bitwise_xor.reduce(sink.cpu().numpy().view(np.uint32))
+    assert got == expect
