@@ -172,7 +172,9 @@ struct EpiShared {
 // Bytes of value rows each warp stages per list buffer (2 KB at d = 64 with
 // 16 heads per group, which lets two CTAs share an SM).
 template <int D, int NP>
-__host__ __device__ constexpr int vstage_warp_bytes() { return (NP >= 64 || (D == 64 && NP == 16)) ? 2048 : 4096; }
+__host__ __device__ constexpr int vstage_warp_bytes() {
+  return (NP >= 64 || (D == 64 && NP == 16)) ? 2048 : (D == 128 && NP <= 16) ? 8192 : 4096;
+}
 
 struct EpiArgs {
   const uint16_t* vgroup;  // V of the group's first value head, batch b

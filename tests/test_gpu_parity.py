@@ -322,3 +322,4 @@ def test_read_probe_reads_every_word():
     expect = np.bitwise_xor.reduce(buf.cpu().numpy().view(np.uint32))
     got = np.bitwise_xor.reduce(sink.cpu().numpy().view(np.uint32))
     assert got == expect
+
