@@ -210,6 +210,49 @@ SAGA_API const char* saga_noalloc_last_error(void);
  * call whatever its kind; limit_ns = 0 cancels a pending request. */
 SAGA_API int saga_test_expire_next_wait(unsigned limit_ns);
 
+/* ---------------------------------------------------------------------------
+ * Closed-form GQA-to-SAGA key-head merge ("More Value per Key", Methodology >
+ * GQA-to-SAGA Conversion > Stage 1).  A teacher with h_k key heads is merged
+ * into h_k / 2 key heads: for every pair (a, b) of teacher heads, the merged
+ * key projection minimising the squared logit error of eq. 13,
+ *   L_ab(M) = sum_{j of a} ||Q^j (X M)^T - Q^j (X W_K^a)^T||_F^2 + (same over b),
+ * is M(a, b) = (W_K^a S_a + W_K^b S_b)(S_a + S_b)^+ with S_r = sum_{j of r}
+ * Q^j^T Q^j (Lemma 4.1, eq. 15); the pairing is the minimum-weight perfect
+ * matching with weights w(a, b) = L_ab(M(a, b)) (Theorem 4.2, eq. 14).
+ *
+ * Inputs (device memory, caller-owned, 16-byte aligned):
+ *   x     bf16 [tokens, hidden]   calibration hidden states X (rows = tokens)
+ *   q     bf16 [tokens, h_q, d]   the teacher's queries Q^j on the same tokens
+ *   w_k   fp32 [h_k, hidden, d]   teacher key projections (keys = X W_K^r)
+ * Query head j belongs to key head floor(j * h_k / h_q) (contiguous groups).
+ * Outputs:
+ *   pair_loss  fp32 [h_k, h_k]        w(a, b), symmetric, zero diagonal
+ *   pairing    int32 [h_k]            partner of every teacher head
+ *   w_k_merged fp32 [h_k/2, hidden, d] M(a, b) of the chosen pairs, ordered
+ *                                      by their smaller head
+ * Arithmetic: G = X^T X and the S_r are formed on the tensor cores (bf16
+ * products, fp32 sums); the pseudoinverse (Jacobi eigen-decomposition,
+ * eigenvalues below 1e-5 of the largest count as zero), M and the losses are
+ * fp64.  Ties between pairings go to the first in the order that pairs the
+ * lowest unmatched head with each remaining head in ascending order.
+ * Constraints: d in {64, 128}; h_k even, 2 <= h_k <= 16 (the matching is
+ * exhaustive); h_q % h_k == 0.  Errors as for the decode calls; the
+ * workspace (saga_merge_workspace_bytes, 256-byte aligned) starts with a
+ * status word readable by saga_get_status.  saga_merge_last_error()
+ * describes the last failure of these two calls. */
+typedef struct saga_merge_shape {
+  int tokens; /* T: calibration tokens */
+  int hidden; /* D: rows of each key projection */
+  int d;      /* head dimension */
+  int h_q;    /* teacher query heads */
+  int h_k;    /* teacher key heads (merged in pairs) */
+} saga_merge_shape;
+SAGA_API size_t saga_merge_workspace_bytes(const saga_merge_shape* s);
+SAGA_API int saga_key_head_merge(const saga_merge_shape* s, const void* x, const void* q, const float* w_k,
+                                 float* pair_loss, int* pairing, float* w_k_merged, void* workspace,
+                                 size_t ws_bytes, void* stream);
+SAGA_API const char* saga_merge_last_error(void);
+
 /* Measurement aid (no counterpart in the paper): one streaming read of
  * `bytes` of device memory at buf (16-byte aligned; the last bytes % 16 are
  * not read), 16-byte loads with four in flight per thread over a grid of up

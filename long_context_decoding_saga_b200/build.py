@@ -13,7 +13,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libsaga.so")
-SOURCES = ["saga_kernels.cu", "saga_api.cu", "saga_noalloc.cu", "saga_probe.cu"]
+SOURCES = ["saga_kernels.cu", "saga_api.cu", "saga_noalloc.cu", "saga_probe.cu", "saga_merge.cu"]
 HEADERS = ["saga_device.cuh", "saga_internal.h"]
 
 NVCC_FLAGS = [

@@ -117,14 +117,6 @@ __device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
   return out != 0;
 }
 
-// Time-bounded wait that ignores the abort flag (used to drain in-flight copies).
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const unsigned long long t0 = global_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 63u && global_ns() - t0 > kWaitLimitNs) return false;
-  }
-}
 
 
 template <int NP>

@@ -31,7 +31,7 @@ EXPORTED = ("saga_workspace_bytes", "saga_kv_append", "atopn_refresh_threshold",
             "atopn_select_threshold", "saga_decode_attn", "saga_trace_next_attention", "saga_get_status", "saga_last_error", "saga_abi_version",
             "saga_noalloc_scratch_bytes", "saga_decode_attn_noalloc", "saga_noalloc_get_status",
             "saga_noalloc_last_error", "saga_decode_step", "saga_test_expire_next_wait", "saga_read_probe_sink_words",
-            "saga_read_probe")
+            "saga_read_probe", "saga_merge_workspace_bytes", "saga_key_head_merge", "saga_merge_last_error")
 
 
 class SagaError(RuntimeError):
@@ -50,6 +50,11 @@ class SagaShape(ctypes.Structure):
 
     def astuple(self):
         return (self.batch, self.h_q, self.h_k, self.h_v, self.d, self.l_cap)
+
+
+class SagaMergeShape(ctypes.Structure):
+    _fields_ = [("tokens", ctypes.c_int), ("hidden", ctypes.c_int), ("d", ctypes.c_int), ("h_q", ctypes.c_int),
+                ("h_k", ctypes.c_int)]
 
 
 _lib = None
@@ -100,6 +105,13 @@ def load(path: Optional[str] = None):
     lib.saga_noalloc_get_status.restype = _I
     lib.saga_test_expire_next_wait.argtypes = [ctypes.c_uint]
     lib.saga_test_expire_next_wait.restype = _I
+    mp = ctypes.POINTER(SagaMergeShape)
+    lib.saga_merge_workspace_bytes.argtypes = [mp]
+    lib.saga_merge_workspace_bytes.restype = ctypes.c_size_t
+    lib.saga_key_head_merge.argtypes = [mp, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    lib.saga_key_head_merge.restype = _I
+    lib.saga_merge_last_error.argtypes = []
+    lib.saga_merge_last_error.restype = ctypes.c_char_p
     lib.saga_read_probe_sink_words.argtypes = []
     lib.saga_read_probe_sink_words.restype = ctypes.c_size_t
     lib.saga_read_probe.argtypes = [_P, ctypes.c_size_t, _P, _P]
@@ -304,6 +316,34 @@ def saga_test_expire_next_wait(limit_ns: int):
     """Test hook: the next decode call's keep kernel (a sparse reuse step) waits on a barrier nothing arrives
     at, for at most limit_ns, then unwinds and flags SAGA_STATUS_TIMEOUT (0 cancels)."""
     _check(load().saga_test_expire_next_wait(int(limit_ns)))
+
+
+def key_head_merge(x, q, w_k, h_k: int, workspace=None, stream=None):
+    """The closed-form GQA-to-SAGA key-head merge (saga_key_head_merge).  x: bf16 [T, D], q: bf16 [T, h_q, d],
+    w_k: fp32 [h_k, D, d].  Returns (pair_loss fp32 [h_k, h_k], pairing int32 [h_k], merged fp32
+    [h_k / 2, D, d], workspace)."""
+    _expect(x, "x", torch.bfloat16)
+    _expect(q, "q", torch.bfloat16)
+    _expect(w_k, "w_k", torch.float32)
+    T, D = x.shape
+    h_q, d = q.shape[1], q.shape[2]
+    if tuple(q.shape) != (T, h_q, d) or tuple(w_k.shape) != (h_k, D, d):
+        raise ValueError("shapes: x [T, D], q [T, h_q, d], w_k [h_k, D, d]")
+    shape = SagaMergeShape(int(T), int(D), int(d), int(h_q), int(h_k))
+    lib = load()
+    need = lib.saga_merge_workspace_bytes(ctypes.byref(shape))
+    if need == 0:
+        raise SagaError(SAGA_ERR_ARG, lib.saga_merge_last_error().decode(errors="replace"))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    loss = torch.empty((h_k, h_k), dtype=torch.float32, device=x.device)
+    pairing = torch.empty(h_k, dtype=torch.int32, device=x.device)
+    merged = torch.empty((h_k // 2, D, d), dtype=torch.float32, device=x.device)
+    rc = lib.saga_key_head_merge(ctypes.byref(shape), _ptr(x), _ptr(q), _ptr(w_k), _ptr(loss), _ptr(pairing),
+                                 _ptr(merged), _ptr(workspace), workspace.numel(), _stream(stream))
+    if rc != SAGA_OK:
+        raise SagaError(rc, lib.saga_merge_last_error().decode(errors="replace"))
+    return loss, pairing, merged, workspace
 
 
 def read_probe(buf: torch.Tensor, sink: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

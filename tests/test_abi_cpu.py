@@ -105,3 +105,33 @@ def test_decode_step_validation(lib):
     assert _step(lib, s, seq_len=0) == saga.SAGA_ERR_ARG
     assert _step(lib, _shape(d=96)) == saga.SAGA_ERR_UNSUPPORTED
     assert lib.saga_last_error()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), saga.SAGA_ERR_UNSUPPORTED),
+    (dict(h_k=3, h_q=6), saga.SAGA_ERR_UNSUPPORTED),
+    (dict(h_k=18, h_q=36), saga.SAGA_ERR_UNSUPPORTED),
+    (dict(h_q=10, h_k=4), saga.SAGA_ERR_ARG),
+    (dict(tokens=0), saga.SAGA_ERR_ARG),
+    (dict(hidden=0), saga.SAGA_ERR_ARG),
+    (dict(h_k=0), saga.SAGA_ERR_ARG),
+])
+def test_merge_rejects_bad_shapes(lib, kw, code):
+    base = dict(tokens=128, hidden=256, d=64, h_q=8, h_k=4)
+    base.update(kw)
+    s = saga.SagaMergeShape(base["tokens"], base["hidden"], base["d"], base["h_q"], base["h_k"])
+    assert lib.saga_merge_workspace_bytes(ctypes.byref(s)) == 0
+    rc = lib.saga_key_head_merge(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert rc == code
+    assert lib.saga_merge_last_error()
+
+
+def test_merge_rejects_null_and_misaligned(lib):
+    s = saga.SagaMergeShape(128, 256, 64, 8, 4)
+    odd = ctypes.c_void_p(0x100008)
+    assert lib.saga_key_head_merge(ctypes.byref(s), None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                                   None) == saga.SAGA_ERR_ARG
+    assert lib.saga_key_head_merge(ctypes.byref(s), odd, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                                   None) == saga.SAGA_ERR_ARG
+    assert lib.saga_key_head_merge(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1 << 30,
+                                   None) == saga.SAGA_ERR_WORKSPACE
