@@ -423,6 +423,90 @@ EXTRA_WORKLOADS = (
 )
 
 
+def time_key_head_merge(dev, tokens=4096, hidden=2048, d=64, h_q=32, h_k=8, repeats=3):
+    """The closed-form key-head merge on a Llama-3.2-1B-shaped teacher (8 key heads merged into 4), synthetic
+    bf16 X and Q, fp32 W_K: the whole call (transposes, tensor-core Gram products, fp64 pseudoinverses,
+    losses and matching), best of `repeats` CUDA-event timings after one warm-up call."""
+    import torch
+
+    from long_context_decoding_saga_b200 import saga
+    g = torch.Generator(device=dev).manual_seed(123)
+    x = torch.randn((tokens, hidden), generator=g, device=dev).to(torch.bfloat16)
+    q = torch.randn((tokens, h_q, d), generator=g, device=dev).to(torch.bfloat16)
+    w = torch.randn((h_k, hidden, d), generator=g, device=dev) * hidden ** -0.5
+    loss, pairing, merged, ws = saga.key_head_merge(x, q, w, h_k)
+    best = None
+    for _ in range(repeats):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        saga.key_head_merge(x, q, w, h_k, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        best = a.elapsed_time(b) if best is None else min(best, a.elapsed_time(b))
+    gram_flop = 2.0 * hidden * hidden * tokens + 2.0 * d * d * tokens * h_q
+    status = saga.saga_get_status(ws)
+    del x, q, w, ws, merged
+    return {"tokens": tokens, "hidden": hidden, "d": d, "h_q": h_q, "h_k": h_k, "us": best * 1e3,
+            "gram_tflop": gram_flop / 1e12, "gram_tflops_over_whole_call": gram_flop / (best / 1e3) / 1e12,
+            "pairing": pairing.cpu().tolist(), "status_word": status}
+
+
+QKV_SHAPES = (  # (name, batch, hidden, h_q, h_k, h_v, d): the SAGA students' decode-step projections
+    ("llama32_1b_saga_b1", 1, 2048, 32, 2, 8, 64),
+    ("llama32_1b_saga_b16", 16, 2048, 32, 2, 8, 64),
+    ("qwen25_1p5b_saga_b1", 1, 1536, 12, 1, 4, 128),
+    ("qwen25_1p5b_saga_b16", 16, 1536, 12, 1, 4, 128),
+)
+
+
+def time_qkv_projection(dev, peak_gbs, layers=24, replays=5):
+    """The fused QKV projection + KV-cache append (eq. 1 with SAGA head counts) as a model runs it: one
+    launch per layer, each layer with its own weights (24 layers of distinct weights exceed L2 for both
+    shapes, so every launch streams its weights from HBM), replayed as one CUDA graph; per-launch time =
+    graph time / layers, best of `replays`.  Algorithmic bytes per launch: the weight matrix, x, the
+    query and the new key/value rows."""
+    import torch
+
+    from long_context_decoding_saga_b200 import saga
+    out = {}
+    for name, B, D, h_q, h_k, h_v, d in QKV_SHAPES:
+        g = torch.Generator(device=dev).manual_seed(7)
+        n_cols = (h_q + h_k + h_v) * d
+        shape = saga.SagaShape.of(B, h_q, h_k, h_v, d, 64)
+        xs = [torch.randn((B, D), generator=g, device=dev).to(torch.bfloat16) for _ in range(layers)]
+        ws = [(torch.randn((n_cols, D), generator=g, device=dev) * D ** -0.5).to(torch.bfloat16)
+              for _ in range(layers)]
+        q = torch.empty((B, h_q, d), dtype=torch.bfloat16, device=dev)
+        kc = torch.zeros((B, h_k, 64, d), dtype=torch.bfloat16, device=dev)
+        vc = torch.zeros((B, h_v, 64, d), dtype=torch.bfloat16, device=dev)
+        stream = torch.cuda.Stream(device=dev)
+        with torch.cuda.stream(stream):
+            for i in range(layers):  # eager warm-up (also sets the kernels' shared-memory limits)
+                saga.saga_qkv_project(shape, xs[i], ws[i], q, kc, vc, 5, stream=stream)
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(layers):
+                saga.saga_qkv_project(shape, xs[i], ws[i], q, kc, vc, 5, stream=stream)
+        best = None
+        for _ in range(replays + 1):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                a.record(stream)
+                graph.replay()
+                b.record(stream)
+            stream.synchronize()
+            ms = a.elapsed_time(b) / layers
+            best = ms if best is None else min(best, ms)
+        nbytes = 2 * (n_cols * D + B * D + B * n_cols)
+        gbs = nbytes / (best * 1e-3) / 1e9
+        out[name] = {"batch": B, "hidden": D, "h_q": h_q, "h_k": h_k, "h_v": h_v, "d": d, "us_per_launch": best * 1e3,
+                     "bytes_per_launch": nbytes, "gbs": gbs, "frac_of_peak": gbs / peak_gbs, "layers": layers,
+                     "gpu_launches": layers * replays}
+        del graph, xs, ws, q, kc, vc
+    return out
+
+
 def time_extra_workload(wl, dev, rank, args, peak, l2_bytes):
     """One entry of the `workloads` object: graph-replayed decode steps of `wl` (K = max(16, R) when R is
     at most 64, so the window holds refresh and reuse steps in their proportion), inputs resident."""
@@ -665,6 +749,14 @@ def run_saga(args, wl, rank, world, local_rank):
             except Exception as exc:  # noqa: BLE001  (reported, never fatal to the benchmark line)
                 extras[name] = {"error": str(exc)[:300]}
         line["workloads"] = extras
+        try:
+            line["qkv_projection"] = time_qkv_projection(dev, peak)
+        except Exception as exc:  # noqa: BLE001  (reported, never fatal to the benchmark line)
+            line["qkv_projection"] = {"error": str(exc)[:300]}
+        try:
+            line["key_head_merge"] = time_key_head_merge(dev)
+        except Exception as exc:  # noqa: BLE001  (reported, never fatal to the benchmark line)
+            line["key_head_merge"] = {"error": str(exc)[:300]}
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line), flush=True)

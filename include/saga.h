@@ -110,6 +110,29 @@ SAGA_API size_t saga_workspace_bytes(const saga_shape* s);
 SAGA_API int saga_kv_append(const saga_shape* s, void* k_cache, void* v_cache, const void* k_new, const void* v_new, int pos,
                    const int* seq_len_dev, void* stream);
 
+/* Decode-step query/key/value projection fused with the KV cache append
+ * (eq. 1 of "More Value per Key: Asymmetric Sparse Attention for Faster LLM
+ * Decoding", Attention Mechanism Formalization, with the decoupled head counts
+ * of Methodology > SAGA Architecture: h_k key heads, h_v value heads).
+ *   x      bf16 [batch, hidden], the new token's hidden state per batch row;
+ *   w_qkv  bf16 [(h_q + h_k + h_v) * d, hidden], row-major; row n holds the
+ *          weights of output column n: rows [0, h_q d) are W_Q's columns
+ *          (query head n / d, dimension n % d), then h_k d rows of W_K, then
+ *          h_v d rows of W_V;
+ *   q_out  bf16 [batch, h_q, d] (written);
+ *   k_cache bf16 [batch, h_k, l_cap, d], v_cache bf16 [batch, h_v, l_cap, d]:
+ *          row pos of every head written, nothing else touched.
+ * Products accumulate in fp32; each output is rounded once to bf16 (nearest
+ * even).  If seq_len_dev is not NULL, pos is read on the device as
+ * (*seq_len_dev - 1), clamped into [0, l_cap), and the host pos only needs
+ * to be in range.  Requirements: 1 <= batch <= 16, hidden a positive multiple
+ * of 8, 0 <= pos < l_cap, all pointers device memory 16-byte aligned, q_out
+ * and the cache rows not overlapping x or w_qkv.  The caller owns every
+ * buffer.  Errors: SAGA_ERR_ARG / SAGA_ERR_UNSUPPORTED before anything is
+ * enqueued; SAGA_ERR_CUDA if the launch fails. */
+SAGA_API int saga_qkv_project(const saga_shape* s, int hidden, const void* x, const void* w_qkv, void* q_out,
+                              void* k_cache, void* v_cache, int pos, const int* seq_len_dev, void* stream);
+
 /* Atop-N threshold refresh (Atop-N step 1-2, "computed once every n
  * tokens"): tau[b, j] = the n_top-th largest of the fp32 scores
  * A[b, j, 0..seq_len) (eq. 2), counted with multiplicity; -inf when

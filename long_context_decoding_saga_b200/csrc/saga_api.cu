@@ -23,6 +23,7 @@ cudaError_t launch_combine(int D, const CombineParams& p, cudaStream_t st);
 cudaError_t launch_select(const SelectParams& p, int rows, cudaStream_t st);
 cudaError_t launch_select_parallel(const SelectParams& p, int rows, cudaStream_t st);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
+cudaError_t launch_qkv(const QkvParams& p, cudaStream_t st);
 cudaError_t launch_fill(float* dst, float v, int n, cudaStream_t st);
 }  // namespace saga
 
@@ -402,6 +403,39 @@ int saga_kv_append(const saga_shape* s, void* k_cache, void* v_cache, const void
   p.l_cap = s->l_cap;
   cudaError_t e = launch_append(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  return ok();
+}
+
+int saga_qkv_project(const saga_shape* s, int hidden, const void* x, const void* w_qkv, void* q_out, void* k_cache,
+                     void* v_cache, int pos, const int* seq_len_dev, void* stream) {
+  int rc = validate_shape(s);
+  if (rc) return rc;
+  if (s->batch > 16) return fail(SAGA_ERR_UNSUPPORTED, "saga_qkv_project supports batch <= 16 (got %d)", s->batch);
+  if (hidden < 8 || hidden % 8 != 0) return fail(SAGA_ERR_ARG, "hidden=%d must be a positive multiple of 8", hidden);
+  if (!x || !w_qkv || !q_out || !k_cache || !v_cache) return fail(SAGA_ERR_ARG, "NULL tensor pointer");
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q_out) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(SAGA_ERR_ARG, "tensor pointers must be 16-byte aligned");
+  if (pos < 0 || pos >= s->l_cap) return fail(SAGA_ERR_ARG, "pos=%d outside [0, l_cap=%d)", pos, s->l_cap);
+  const long long n_cols = (long long)(s->h_q + s->h_k + s->h_v) * s->d;
+  if (n_cols * hidden >= (1ll << 31)) return fail(SAGA_ERR_UNSUPPORTED, "projection too large for 32-bit indexing");
+  QkvParams p{};
+  p.x = static_cast<const uint16_t*>(x);
+  p.w = static_cast<const uint16_t*>(w_qkv);
+  p.q = static_cast<uint16_t*>(q_out);
+  p.k_cache = static_cast<uint16_t*>(k_cache);
+  p.v_cache = static_cast<uint16_t*>(v_cache);
+  p.seq_len_dev = seq_len_dev;
+  p.pos = pos;
+  p.batch = s->batch;
+  p.hidden = hidden;
+  p.n_cols = (int)n_cols;
+  p.h_q = s->h_q;
+  p.h_k = s->h_k;
+  p.h_v = s->h_v;
+  p.d = s->d;
+  p.l_cap = s->l_cap;
+  cudaError_t e = launch_qkv(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "qkv launch");
   return ok();
 }
 

@@ -137,6 +137,18 @@ struct SelectParams {
   int n_top;
 };
 
+// Decode-step QKV projection (eq. 1) fused with the KV-cache append.
+struct QkvParams {
+  const uint16_t* x;   // bf16 [B, hidden]
+  const uint16_t* w;   // bf16 [(h_q + h_k + h_v) d, hidden]: rows of W_Q, then W_K, then W_V
+  uint16_t* q;         // bf16 [B, h_q, d]
+  uint16_t* k_cache;   // bf16 [B, h_k, l_cap, d]: row pos written
+  uint16_t* v_cache;   // bf16 [B, h_v, l_cap, d]: row pos written
+  const int* seq_len_dev;  // nullable: pos = *seq_len_dev - 1 (clamped into [0, l_cap))
+  int pos;
+  int batch, hidden, n_cols, h_q, h_k, h_v, d, l_cap;
+};
+
 struct AppendParams {
   uint16_t* k_cache;
   uint16_t* v_cache;

@@ -30,6 +30,7 @@
 #include <stdint.h>
 
 #include <stdlib.h>
+#include <string.h>
 
 #include <atomic>
 #include <utility>
@@ -2014,6 +2015,103 @@ __global__ void saga_fill_kernel(float* dst, float v, int n) {
   if (i < n) dst[i] = v;
 }
 
+// ============================================================================ QKV projection
+// Eq. 1 for the new token: q = x W_Q, k = x W_K, v = x W_V with h_k key
+// heads and h_v value heads (SAGA: fewer key rows to stream), the key and
+// value rows written straight into the caches at the new position (the
+// append of the decode step).  A weight-streaming product at batch <= 16
+// (about 8 flops per weight byte at batch 16): HBM-bound, so CUDA cores with
+// wide loads.  One warp per output column: each lane reads 16-byte pieces
+// of the column's weight row (all of a lane's pieces in flight at once) and
+// multiplies them with the batch rows of x staged in shared memory; the warp
+// sums the lanes' partial dot products.  The weight rows, which no earlier
+// kernel writes, are prefetched into L2 before the dependency wait.
+constexpr int kQkvWarps = 8;                // output columns per CTA
+constexpr int kQkvChunk = 2048;             // x elements per row staged per pass
+constexpr int kQkvPieces = kQkvChunk / 256; // 16-byte weight pieces per lane per pass
+
+template <int NB>
+__global__ void __launch_bounds__(kQkvWarps * 32) saga_qkv_kernel(const QkvParams p) {
+  extern __shared__ __align__(16) uint16_t xs[];  // [NB][kQkvChunk]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * kQkvWarps + warp;
+  const uint16_t* wrow = p.w + (size_t)n * p.hidden;
+  if (n < p.n_cols)
+    for (int off = lane * 128; off < p.hidden * 2; off += 32 * 128)
+      prefetch_l2_line(reinterpret_cast<const char*>(wrow) + off);
+  pdl_trigger();
+  pdl_wait();
+  float acc[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) acc[b] = 0.f;
+  for (int k0 = 0; k0 < p.hidden; k0 += kQkvChunk) {
+    const int kn = min(kQkvChunk, p.hidden - k0);
+    __syncthreads();  // the previous pass is done with xs
+    for (int i = threadIdx.x; i < NB * (kn / 8); i += blockDim.x) {
+      const int b = i / (kn / 8), c = i % (kn / 8);
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (b < p.batch) v = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)b * p.hidden + k0) + c);
+      *reinterpret_cast<uint4*>(xs + b * kQkvChunk + c * 8) = v;
+    }
+    __syncthreads();
+    if (n < p.n_cols) {
+      uint4 wv[kQkvPieces];
+#pragma unroll
+      for (int i = 0; i < kQkvPieces; ++i) {
+        const int c = lane + 32 * i;  // piece index: elements 8c .. 8c + 7 of the pass
+        wv[i] = c * 8 < kn ? __ldg(reinterpret_cast<const uint4*>(wrow + k0) + c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < kQkvPieces; ++i) {
+        const int c = lane + 32 * i;
+        if (c * 8 >= kn) break;
+        const float w0 = bf16_lo(wv[i].x), w1 = bf16_hi(wv[i].x), w2 = bf16_lo(wv[i].y), w3 = bf16_hi(wv[i].y);
+        const float w4 = bf16_lo(wv[i].z), w5 = bf16_hi(wv[i].z), w6 = bf16_lo(wv[i].w), w7 = bf16_hi(wv[i].w);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const uint4 xv = *reinterpret_cast<const uint4*>(xs + b * kQkvChunk + c * 8);
+          float a = acc[b];
+          a = fmaf(w0, bf16_lo(xv.x), a);
+          a = fmaf(w1, bf16_hi(xv.x), a);
+          a = fmaf(w2, bf16_lo(xv.y), a);
+          a = fmaf(w3, bf16_hi(xv.y), a);
+          a = fmaf(w4, bf16_lo(xv.z), a);
+          a = fmaf(w5, bf16_hi(xv.z), a);
+          a = fmaf(w6, bf16_lo(xv.w), a);
+          a = fmaf(w7, bf16_hi(xv.w), a);
+          acc[b] = a;
+        }
+      }
+    }
+  }
+  if (n >= p.n_cols) return;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
+  // lane b writes batch row b of column n
+  int pos = p.pos;
+  if (p.seq_len_dev != nullptr) pos = device_seq_len(p.seq_len_dev, p.pos + 1, p.l_cap, nullptr) - 1;
+  float mine = 0.f;
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+    if (lane == b) mine = acc[b];
+  if (lane < p.batch && lane < NB) {
+    const int b = lane;
+    const int qcols = p.h_q * p.d, kcols = p.h_k * p.d;
+    const __nv_bfloat16 v = __float2bfloat16_rn(mine);
+    uint16_t bits;
+    memcpy(&bits, &v, 2);
+    if (n < qcols) {
+      p.q[(size_t)b * qcols + n] = bits;
+    } else if (n < qcols + kcols) {
+      const int h = (n - qcols) / p.d, c = (n - qcols) % p.d;
+      p.k_cache[(((size_t)b * p.h_k + h) * p.l_cap + pos) * p.d + c] = bits;
+    } else {
+      const int u = (n - qcols - kcols) / p.d, c = (n - qcols - kcols) % p.d;
+      p.v_cache[(((size_t)b * p.h_v + u) * p.l_cap + pos) * p.d + c] = bits;
+    }
+  }
+}
+
 // ============================================================================ launchers
 // Every kernel is launched with programmatic stream serialization: it may
 // start while the previous kernel on the stream finishes, runs its
@@ -2187,6 +2285,27 @@ cudaError_t launch_select_parallel(const SelectParams& p, int rows, cudaStream_t
   e = launch_k(atopn_collect_kernel, dim3(rows, parts), dim3(kSelPartThreads), 0, st, p);
   if (e != cudaSuccess) return e;
   return launch_k(atopn_resolve_kernel, dim3(rows), dim3(kSelectThreads), bytes, st, p);
+}
+
+template <int NB>
+static cudaError_t run_qkv(const QkvParams& p, cudaStream_t st) {
+  static std::atomic<uint64_t> prepared{0};
+  const int bytes = NB * kQkvChunk * 2;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(saga_qkv_kernel<NB>), bytes, prepared);
+  if (e != cudaSuccess) return e;
+  return launch_k(saga_qkv_kernel<NB>, dim3((p.n_cols + kQkvWarps - 1) / kQkvWarps), dim3(kQkvWarps * 32), bytes, st,
+                  p);
+}
+
+// The QKV projection for batch <= 16 (the register array is sized by the
+// smallest of 1, 2, 4, 8, 16 that holds the batch).
+cudaError_t launch_qkv(const QkvParams& p, cudaStream_t st) {
+  if (p.batch <= 1) return run_qkv<1>(p, st);
+  if (p.batch <= 2) return run_qkv<2>(p, st);
+  if (p.batch <= 4) return run_qkv<4>(p, st);
+  if (p.batch <= 8) return run_qkv<8>(p, st);
+  if (p.batch <= 16) return run_qkv<16>(p, st);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st) {

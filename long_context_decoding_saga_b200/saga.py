@@ -31,7 +31,8 @@ EXPORTED = ("saga_workspace_bytes", "saga_kv_append", "atopn_refresh_threshold",
             "atopn_select_threshold", "saga_decode_attn", "saga_trace_next_attention", "saga_get_status", "saga_last_error", "saga_abi_version",
             "saga_noalloc_scratch_bytes", "saga_decode_attn_noalloc", "saga_noalloc_get_status",
             "saga_noalloc_last_error", "saga_decode_step", "saga_test_expire_next_wait", "saga_read_probe_sink_words",
-            "saga_read_probe", "saga_merge_workspace_bytes", "saga_key_head_merge", "saga_merge_last_error")
+            "saga_read_probe", "saga_merge_workspace_bytes", "saga_key_head_merge", "saga_merge_last_error",
+            "saga_qkv_project")
 
 
 class SagaError(RuntimeError):
@@ -76,6 +77,8 @@ def load(path: Optional[str] = None):
     lib.saga_workspace_bytes.restype = ctypes.c_size_t
     lib.saga_kv_append.argtypes = [sp, _P, _P, _P, _P, _I, _P, _P]
     lib.saga_kv_append.restype = _I
+    lib.saga_qkv_project.argtypes = [sp, _I, _P, _P, _P, _P, _P, _I, _P, _P]
+    lib.saga_qkv_project.restype = _I
     lib.atopn_refresh_threshold.argtypes = [sp, _P, _P, _I, _P, _I, _P, _P, ctypes.c_size_t, _P]
     lib.atopn_refresh_threshold.restype = _I
     lib.atopn_select_workspace_bytes.argtypes = [_I]
@@ -176,6 +179,24 @@ def saga_kv_append(shape: SagaShape, k_cache, v_cache, k_new, v_new, pos: int, s
         _expect(seq_len_dev, "seq_len_dev", torch.int32)
     _check(load().saga_kv_append(ctypes.byref(shape), _ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new),
                                  int(pos), _ptr(seq_len_dev), _stream(stream)))
+
+
+def saga_qkv_project(shape: SagaShape, x, w_qkv, q_out, k_cache, v_cache, pos: int, seq_len_dev=None,
+                     stream=None):
+    """Eq. 1 for the new token: q_out = x W_Q, and x W_K, x W_V written into row pos of the caches."""
+    B, hq, hk, hv, d, lc = shape.astuple()
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise SagaError(SAGA_ERR_ARG, "x must be a 2-D tensor [batch, hidden]")
+    D = int(x.shape[1])
+    _expect(x, "x", torch.bfloat16, (B, D))
+    _expect(w_qkv, "w_qkv", torch.bfloat16, ((hq + hk + hv) * d, D))
+    _expect(q_out, "q_out", torch.bfloat16, (B, hq, d))
+    _expect(k_cache, "k_cache", torch.bfloat16, (B, hk, lc, d))
+    _expect(v_cache, "v_cache", torch.bfloat16, (B, hv, lc, d))
+    if seq_len_dev is not None:
+        _expect(seq_len_dev, "seq_len_dev", torch.int32)
+    _check(load().saga_qkv_project(ctypes.byref(shape), D, _ptr(x), _ptr(w_qkv), _ptr(q_out), _ptr(k_cache),
+                                   _ptr(v_cache), int(pos), _ptr(seq_len_dev), _stream(stream)))
 
 
 def atopn_refresh_threshold(shape: SagaShape, q, k_cache, seq_len: int, n_top: int, tau, workspace,

@@ -135,3 +135,21 @@ def test_merge_rejects_null_and_misaligned(lib):
                                    None) == saga.SAGA_ERR_ARG
     assert lib.saga_key_head_merge(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1 << 30,
                                    None) == saga.SAGA_ERR_WORKSPACE
+
+
+def _qkv(lib, shape, hidden=256, x=FAKE, pos=0):
+    return lib.saga_qkv_project(ctypes.byref(shape), hidden, x, FAKE, FAKE, FAKE, FAKE, pos, None, None)
+
+
+def test_qkv_projection_validation(lib):
+    s = _shape()
+    assert _qkv(lib, _shape(batch=17)) == saga.SAGA_ERR_UNSUPPORTED
+    assert _qkv(lib, s, hidden=0) == saga.SAGA_ERR_ARG
+    assert _qkv(lib, s, hidden=100) == saga.SAGA_ERR_ARG  # not a multiple of 8
+    assert _qkv(lib, s, x=None) == saga.SAGA_ERR_ARG
+    assert _qkv(lib, s, x=ctypes.c_void_p(0x100008)) == saga.SAGA_ERR_ARG  # not 16-byte aligned
+    assert _qkv(lib, s, pos=1024) == saga.SAGA_ERR_ARG
+    assert _qkv(lib, s, pos=-1) == saga.SAGA_ERR_ARG
+    assert _qkv(lib, _shape(d=96)) == saga.SAGA_ERR_UNSUPPORTED
+    assert _qkv(lib, _shape(h_q=4096, h_k=64, h_v=64, d=128), hidden=1 << 16) == saga.SAGA_ERR_UNSUPPORTED
+    assert lib.saga_last_error()
