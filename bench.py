@@ -479,15 +479,16 @@ def time_qkv_projection(dev, peak_gbs, layers=24, replays=5):
         q = torch.empty((B, h_q, d), dtype=torch.bfloat16, device=dev)
         kc = torch.zeros((B, h_k, 64, d), dtype=torch.bfloat16, device=dev)
         vc = torch.zeros((B, h_v, 64, d), dtype=torch.bfloat16, device=dev)
+        work = saga.alloc_qkv_workspace(shape, D, dev)
         stream = torch.cuda.Stream(device=dev)
         with torch.cuda.stream(stream):
             for i in range(layers):  # eager warm-up (also sets the kernels' shared-memory limits)
-                saga.saga_qkv_project(shape, xs[i], ws[i], q, kc, vc, 5, stream=stream)
+                saga.saga_qkv_project(shape, xs[i], ws[i], q, kc, vc, 5, workspace=work, stream=stream)
         stream.synchronize()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream):
             for i in range(layers):
-                saga.saga_qkv_project(shape, xs[i], ws[i], q, kc, vc, 5, stream=stream)
+                saga.saga_qkv_project(shape, xs[i], ws[i], q, kc, vc, 5, workspace=work, stream=stream)
         best = None
         for _ in range(replays + 1):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -502,8 +503,9 @@ def time_qkv_projection(dev, peak_gbs, layers=24, replays=5):
         gbs = nbytes / (best * 1e-3) / 1e9
         out[name] = {"batch": B, "hidden": D, "h_q": h_q, "h_k": h_k, "h_v": h_v, "d": d, "us_per_launch": best * 1e3,
                      "bytes_per_launch": nbytes, "gbs": gbs, "frac_of_peak": gbs / peak_gbs, "layers": layers,
-                     "gpu_launches": layers * replays}
-        del graph, xs, ws, q, kc, vc
+                     "gpu_launches": layers * (replays + 1), "status_word": saga.saga_get_status(work),
+                     "kernel": "saga_qkv_kernel (CUDA cores)" if B == 1 else "saga_qkv_mma_kernel (tcgen05)"}
+        del graph, xs, ws, q, kc, vc, work
     return out
 
 
@@ -775,6 +777,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the extra workloads timed after the headline (the `workloads` object)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs)")
+    ap.add_argument("--only", default="", choices=["", "qkv", "merge"],
+                    help="time only the QKV projection or the key-head merge and print their object (profiling runs)")
     ap.add_argument("--flush-l2", default="auto", choices=["auto", "on", "off"],
                     help="write 2 x L2 between timed steps (auto: when a step streams less than 2 x L2)")
     args = ap.parse_args()
@@ -786,6 +790,19 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.only:
+        import torch
+
+        from long_context_decoding_saga_b200 import build, saga
+        build.build()
+        saga.load()
+        dev = torch.device("cuda", 0)
+        peak, _ = load_peak()
+        if args.only == "qkv":
+            print(json.dumps({"qkv_projection": time_qkv_projection(dev, peak)}), flush=True)
+        else:
+            print(json.dumps({"key_head_merge": time_key_head_merge(dev)}), flush=True)
+        return 0
     if args.impl == "reference":
         return run_reference(args, wl, rank, world)
     if world > 1:

@@ -122,16 +122,28 @@ SAGA_API int saga_kv_append(const saga_shape* s, void* k_cache, void* v_cache, c
  *   q_out  bf16 [batch, h_q, d] (written);
  *   k_cache bf16 [batch, h_k, l_cap, d], v_cache bf16 [batch, h_v, l_cap, d]:
  *          row pos of every head written, nothing else touched.
- * Products accumulate in fp32; each output is rounded once to bf16 (nearest
- * even).  If seq_len_dev is not NULL, pos is read on the device as
- * (*seq_len_dev - 1), clamped into [0, l_cap), and the host pos only needs
- * to be in range.  Requirements: 1 <= batch <= 16, hidden a positive multiple
- * of 8, 0 <= pos < l_cap, all pointers device memory 16-byte aligned, q_out
- * and the cache rows not overlapping x or w_qkv.  The caller owns every
- * buffer.  Errors: SAGA_ERR_ARG / SAGA_ERR_UNSUPPORTED before anything is
- * enqueued; SAGA_ERR_CUDA if the launch fails. */
+ * Products accumulate in fp32 (batch 1 on CUDA cores; batch 2 .. 16 on the
+ * tensor cores, the hidden dimension split across CTAs and the fp32 partials
+ * added in a fixed order, so results are reproducible run to run); each
+ * output is rounded once to bf16 (nearest even).  If seq_len_dev is not NULL,
+ * pos is read on the device as (*seq_len_dev - 1), clamped into [0, l_cap),
+ * and the host pos only needs to be in range.  Requirements: 1 <= batch <=
+ * 16, hidden a positive multiple of 8, 0 <= pos < l_cap, all tensor pointers
+ * device memory 16-byte aligned, q_out and the cache rows not overlapping x
+ * or w_qkv.  workspace: device memory of saga_qkv_workspace_bytes(s, hidden)
+ * bytes, 256-byte aligned, zero-filled once before first use (every call
+ * leaves it ready for the next); word 0 is a sticky status word read by
+ * saga_get_status (SAGA_STATUS_TIMEOUT if a bounded wait gave up); calls on
+ * one workspace must not overlap in time.  The caller owns every buffer.
+ * Errors: SAGA_ERR_ARG / SAGA_ERR_UNSUPPORTED / SAGA_ERR_WORKSPACE before
+ * anything is enqueued; SAGA_ERR_CUDA if the launch fails. */
 SAGA_API int saga_qkv_project(const saga_shape* s, int hidden, const void* x, const void* w_qkv, void* q_out,
-                              void* k_cache, void* v_cache, int pos, const int* seq_len_dev, void* stream);
+                              void* k_cache, void* v_cache, int pos, const int* seq_len_dev, void* workspace,
+                              size_t ws_bytes, void* stream);
+
+/* Workspace bytes saga_qkv_project needs for this shape and hidden size on
+ * the current device (0 for invalid arguments or without a device). */
+SAGA_API size_t saga_qkv_workspace_bytes(const saga_shape* s, int hidden);
 
 /* Atop-N threshold refresh (Atop-N step 1-2, "computed once every n
  * tokens"): tau[b, j] = the n_top-th largest of the fp32 scores

@@ -23,7 +23,7 @@ cudaError_t launch_combine(int D, const CombineParams& p, cudaStream_t st);
 cudaError_t launch_select(const SelectParams& p, int rows, cudaStream_t st);
 cudaError_t launch_select_parallel(const SelectParams& p, int rows, cudaStream_t st);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
-cudaError_t launch_qkv(const QkvParams& p, cudaStream_t st);
+cudaError_t launch_qkv(const QkvParams& p, const CUtensorMap& tw, cudaStream_t st);
 cudaError_t launch_fill(float* dst, float v, int n, cudaStream_t st);
 }  // namespace saga
 
@@ -364,7 +364,7 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
 
 extern "C" {
 
-int saga_abi_version(void) { return 101; }
+int saga_abi_version(void) { return 102; }
 
 const char* saga_last_error(void) { return g_err; }
 
@@ -406,18 +406,39 @@ int saga_kv_append(const saga_shape* s, void* k_cache, void* v_cache, const void
   return ok();
 }
 
-int saga_qkv_project(const saga_shape* s, int hidden, const void* x, const void* w_qkv, void* q_out, void* k_cache,
-                     void* v_cache, int pos, const int* seq_len_dev, void* stream) {
+static int validate_qkv(const saga_shape* s, int hidden) {
   int rc = validate_shape(s);
   if (rc) return rc;
-  if (s->batch > 16) return fail(SAGA_ERR_UNSUPPORTED, "saga_qkv_project supports batch <= 16 (got %d)", s->batch);
+  if (s->batch > kQkvN) return fail(SAGA_ERR_UNSUPPORTED, "saga_qkv_project supports batch <= %d (got %d)", kQkvN, s->batch);
   if (hidden < 8 || hidden % 8 != 0) return fail(SAGA_ERR_ARG, "hidden=%d must be a positive multiple of 8", hidden);
+  if (hidden > kQkvMaxHidden) return fail(SAGA_ERR_UNSUPPORTED, "hidden=%d exceeds %d", hidden, kQkvMaxHidden);
+  const long long n_cols = (long long)(s->h_q + s->h_k + s->h_v) * s->d;
+  if (n_cols * hidden >= (1ll << 31)) return fail(SAGA_ERR_UNSUPPORTED, "projection too large for 32-bit indexing");
+  return SAGA_OK;
+}
+
+constexpr size_t kQkvWorkspaceBytes = 256;  // the status word at offset 0, the rest reserved
+
+size_t saga_qkv_workspace_bytes(const saga_shape* s, int hidden) {
+  if (validate_qkv(s, hidden)) return 0;
+  return kQkvWorkspaceBytes;
+}
+
+int saga_qkv_project(const saga_shape* s, int hidden, const void* x, const void* w_qkv, void* q_out, void* k_cache,
+                     void* v_cache, int pos, const int* seq_len_dev, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = validate_qkv(s, hidden);
+  if (rc) return rc;
   if (!x || !w_qkv || !q_out || !k_cache || !v_cache) return fail(SAGA_ERR_ARG, "NULL tensor pointer");
   if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q_out) || !aligned16(k_cache) || !aligned16(v_cache))
     return fail(SAGA_ERR_ARG, "tensor pointers must be 16-byte aligned");
   if (pos < 0 || pos >= s->l_cap) return fail(SAGA_ERR_ARG, "pos=%d outside [0, l_cap=%d)", pos, s->l_cap);
-  const long long n_cols = (long long)(s->h_q + s->h_k + s->h_v) * s->d;
-  if (n_cols * hidden >= (1ll << 31)) return fail(SAGA_ERR_UNSUPPORTED, "projection too large for 32-bit indexing");
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SAGA_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer");
+  if (ws_bytes < kQkvWorkspaceBytes)
+    return fail(SAGA_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", ws_bytes, kQkvWorkspaceBytes);
+  int sms = 0;
+  rc = device_sms(&sms);
+  if (rc) return rc;
   QkvParams p{};
   p.x = static_cast<const uint16_t*>(x);
   p.w = static_cast<const uint16_t*>(w_qkv);
@@ -425,16 +446,31 @@ int saga_qkv_project(const saga_shape* s, int hidden, const void* x, const void*
   p.k_cache = static_cast<uint16_t*>(k_cache);
   p.v_cache = static_cast<uint16_t*>(v_cache);
   p.seq_len_dev = seq_len_dev;
+  p.status = static_cast<unsigned*>(workspace);
   p.pos = pos;
   p.batch = s->batch;
   p.hidden = hidden;
-  p.n_cols = (int)n_cols;
+  p.n_cols = (s->h_q + s->h_k + s->h_v) * s->d;
   p.h_q = s->h_q;
   p.h_k = s->h_k;
   p.h_v = s->h_v;
   p.d = s->d;
   p.l_cap = s->l_cap;
-  cudaError_t e = launch_qkv(p, static_cast<cudaStream_t>(stream));
+  int m_tiles = 0;
+  qkv_mma_plan(p.n_cols, hidden, sms, &m_tiles, &p.splits, &p.kb_total, &p.stages, &p.kbs_max);
+  // w_qkv as rows of `hidden` bf16: boxes of 64 columns (one 128-byte swizzle row) by 128 rows
+  CUtensorMap tw;
+  EncodeTiledFn enc = get_encode();
+  if (enc == nullptr) return fail(SAGA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
+  cuuint64_t dims[2] = {(cuuint64_t)hidden, (cuuint64_t)p.n_cols};
+  cuuint64_t strides[1] = {(cuuint64_t)hidden * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kQkvTileK, (cuuint32_t)kQkvTileM};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w_qkv), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SAGA_ERR_CUDA, "cuTensorMapEncodeTiled (weights) failed (%d)", (int)r);
+  cudaError_t e = launch_qkv(p, tw, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "qkv launch");
   return ok();
 }

@@ -145,9 +145,26 @@ struct QkvParams {
   uint16_t* k_cache;   // bf16 [B, h_k, l_cap, d]: row pos written
   uint16_t* v_cache;   // bf16 [B, h_v, l_cap, d]: row pos written
   const int* seq_len_dev;  // nullable: pos = *seq_len_dev - 1 (clamped into [0, l_cap))
+  unsigned* status;
   int pos;
   int batch, hidden, n_cols, h_q, h_k, h_v, d, l_cap;
+  int splits, kb_total, stages, kbs_max;  // tensor-core path: hidden split (cluster size) and ring depth
 };
+
+// Tensor-core QKV projection tiling (shared by the kernel and the workspace sizing).
+constexpr int kQkvTileM = 128;    // output columns per tile (MMA M)
+constexpr int kQkvTileK = 64;     // hidden elements per k-block: one 128-byte swizzle row
+constexpr int kQkvN = 16;         // batch rows of the B operand (MMA N)
+constexpr int kQkvMaxStages = 5;  // weight-tile ring depth
+constexpr int kQkvMaxKb = 32;     // most k-blocks of x one CTA stages
+constexpr int kQkvMaxSplits = 8;  // splits of the hidden dimension: one portable cluster
+constexpr int kQkvMaxHidden = kQkvMaxSplits * kQkvMaxKb * kQkvTileK;  // 16384
+#ifndef SAGA_QKV_MMA_MIN_BATCH
+#define SAGA_QKV_MMA_MIN_BATCH 2
+#endif
+constexpr int kQkvMmaMinBatch = SAGA_QKV_MMA_MIN_BATCH;  // smallest batch sent to the tensor cores
+void qkv_mma_plan(int n_cols, int hidden, int sms, int* m_tiles, int* splits, int* kb_total, int* stages,
+                  int* kbs_max);
 
 struct AppendParams {
   uint16_t* k_cache;

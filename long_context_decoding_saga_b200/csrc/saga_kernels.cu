@@ -2019,25 +2019,59 @@ __global__ void saga_fill_kernel(float* dst, float v, int n) {
 // Eq. 1 for the new token: q = x W_Q, k = x W_K, v = x W_V with h_k key
 // heads and h_v value heads (SAGA: fewer key rows to stream), the key and
 // value rows written straight into the caches at the new position (the
-// append of the decode step).  A weight-streaming product at batch <= 16
-// (about 8 flops per weight byte at batch 16): HBM-bound, so CUDA cores with
-// wide loads.  One warp per output column: each lane reads 16-byte pieces
-// of the column's weight row (all of a lane's pieces in flight at once) and
-// multiplies them with the batch rows of x staged in shared memory; the warp
-// sums the lanes' partial dot products.  The weight rows, which no earlier
-// kernel writes, are prefetched into L2 before the dependency wait.
+// append of the decode step).  Both kernels stream the weight matrix once;
+// the weights, which no earlier kernel writes, are requested before the
+// dependency wait so their stream overlaps the tail of the preceding kernel.
+//
+// Batch 1 (a matrix-vector product, 2 flops per weight): CUDA cores.  One
+// warp per output column; each lane holds 16-byte pieces of the column's
+// weight row in registers (the whole row of a 2048-wide model in flight at
+// once) and multiplies them with x staged in shared memory; the warp sums the
+// lanes' partial dot products.
 constexpr int kQkvWarps = 8;                // output columns per CTA
 constexpr int kQkvChunk = 2048;             // x elements per row staged per pass
 constexpr int kQkvPieces = kQkvChunk / 256; // 16-byte weight pieces per lane per pass
 
+// The new token's position: the host value, or seq_len - 1 read on the device.
+__device__ __forceinline__ int qkv_position(const QkvParams& p) {
+  return p.seq_len_dev != nullptr ? device_seq_len(p.seq_len_dev, p.pos + 1, p.l_cap, nullptr) - 1 : p.pos;
+}
+
+// Output column n of batch row b: the query, or row pos of a key or value head.
+__device__ __forceinline__ void qkv_store(const QkvParams& p, int n, int b, int pos, float val) {
+  const int qcols = p.h_q * p.d, kcols = p.h_k * p.d;
+  const __nv_bfloat16 v = __float2bfloat16_rn(val);
+  uint16_t bits;
+  memcpy(&bits, &v, 2);
+  if (n < qcols) {
+    p.q[(size_t)b * qcols + n] = bits;
+  } else if (n < qcols + kcols) {
+    const int h = (n - qcols) / p.d, c = (n - qcols) % p.d;
+    p.k_cache[(((size_t)b * p.h_k + h) * p.l_cap + pos) * p.d + c] = bits;
+  } else {
+    const int u = (n - qcols - kcols) / p.d, c = (n - qcols - kcols) % p.d;
+    p.v_cache[(((size_t)b * p.h_v + u) * p.l_cap + pos) * p.d + c] = bits;
+  }
+}
+
 template <int NB>
-__global__ void __launch_bounds__(kQkvWarps * 32) saga_qkv_kernel(const QkvParams p) {
+__global__ void __launch_bounds__(kQkvWarps * 32, NB == 1 ? 4 : 2) saga_qkv_kernel(const QkvParams p) {
   extern __shared__ __align__(16) uint16_t xs[];  // [NB][kQkvChunk]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = blockIdx.x * kQkvWarps + warp;
-  const uint16_t* wrow = p.w + (size_t)n * p.hidden;
-  if (n < p.n_cols)
-    for (int off = lane * 128; off < p.hidden * 2; off += 32 * 128)
+  const bool live = n < p.n_cols;
+  const uint16_t* wrow = p.w + (size_t)(live ? n : 0) * p.hidden;
+  uint4 wv[kQkvPieces];
+  auto load_pass = [&](int k0, int kn) {
+#pragma unroll
+    for (int i = 0; i < kQkvPieces; ++i) {
+      const int c = lane + 32 * i;  // piece index: elements 8c .. 8c + 7 of the pass
+      wv[i] = live && c * 8 < kn ? __ldg(reinterpret_cast<const uint4*>(wrow + k0) + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+  load_pass(0, min(kQkvChunk, p.hidden));
+  if (live)  // later passes of a wider model: into L2 meanwhile
+    for (int off = kQkvChunk * 2 + lane * 128; off < p.hidden * 2; off += 32 * 128)
       prefetch_l2_line(reinterpret_cast<const char*>(wrow) + off);
   pdl_trigger();
   pdl_wait();
@@ -2046,6 +2080,7 @@ __global__ void __launch_bounds__(kQkvWarps * 32) saga_qkv_kernel(const QkvParam
   for (int b = 0; b < NB; ++b) acc[b] = 0.f;
   for (int k0 = 0; k0 < p.hidden; k0 += kQkvChunk) {
     const int kn = min(kQkvChunk, p.hidden - k0);
+    if (k0 > 0) load_pass(k0, kn);
     __syncthreads();  // the previous pass is done with xs
     for (int i = threadIdx.x; i < NB * (kn / 8); i += blockDim.x) {
       const int b = i / (kn / 8), c = i % (kn / 8);
@@ -2054,61 +2089,205 @@ __global__ void __launch_bounds__(kQkvWarps * 32) saga_qkv_kernel(const QkvParam
       *reinterpret_cast<uint4*>(xs + b * kQkvChunk + c * 8) = v;
     }
     __syncthreads();
-    if (n < p.n_cols) {
-      uint4 wv[kQkvPieces];
 #pragma unroll
-      for (int i = 0; i < kQkvPieces; ++i) {
-        const int c = lane + 32 * i;  // piece index: elements 8c .. 8c + 7 of the pass
-        wv[i] = c * 8 < kn ? __ldg(reinterpret_cast<const uint4*>(wrow + k0) + c) : make_uint4(0u, 0u, 0u, 0u);
-      }
+    for (int i = 0; i < kQkvPieces; ++i) {
+      const int c = lane + 32 * i;
+      if (c * 8 >= kn) break;
+      const float w0 = bf16_lo(wv[i].x), w1 = bf16_hi(wv[i].x), w2 = bf16_lo(wv[i].y), w3 = bf16_hi(wv[i].y);
+      const float w4 = bf16_lo(wv[i].z), w5 = bf16_hi(wv[i].z), w6 = bf16_lo(wv[i].w), w7 = bf16_hi(wv[i].w);
 #pragma unroll
-      for (int i = 0; i < kQkvPieces; ++i) {
-        const int c = lane + 32 * i;
-        if (c * 8 >= kn) break;
-        const float w0 = bf16_lo(wv[i].x), w1 = bf16_hi(wv[i].x), w2 = bf16_lo(wv[i].y), w3 = bf16_hi(wv[i].y);
-        const float w4 = bf16_lo(wv[i].z), w5 = bf16_hi(wv[i].z), w6 = bf16_lo(wv[i].w), w7 = bf16_hi(wv[i].w);
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(xs + b * kQkvChunk + c * 8);
-          float a = acc[b];
-          a = fmaf(w0, bf16_lo(xv.x), a);
-          a = fmaf(w1, bf16_hi(xv.x), a);
-          a = fmaf(w2, bf16_lo(xv.y), a);
-          a = fmaf(w3, bf16_hi(xv.y), a);
-          a = fmaf(w4, bf16_lo(xv.z), a);
-          a = fmaf(w5, bf16_hi(xv.z), a);
-          a = fmaf(w6, bf16_lo(xv.w), a);
-          a = fmaf(w7, bf16_hi(xv.w), a);
-          acc[b] = a;
-        }
+      for (int b = 0; b < NB; ++b) {
+        const uint4 xv = *reinterpret_cast<const uint4*>(xs + b * kQkvChunk + c * 8);
+        float a = acc[b];
+        a = fmaf(w0, bf16_lo(xv.x), a);
+        a = fmaf(w1, bf16_hi(xv.x), a);
+        a = fmaf(w2, bf16_lo(xv.y), a);
+        a = fmaf(w3, bf16_hi(xv.y), a);
+        a = fmaf(w4, bf16_lo(xv.z), a);
+        a = fmaf(w5, bf16_hi(xv.z), a);
+        a = fmaf(w6, bf16_lo(xv.w), a);
+        a = fmaf(w7, bf16_hi(xv.w), a);
+        acc[b] = a;
       }
     }
   }
-  if (n >= p.n_cols) return;
+  if (!live) return;
 #pragma unroll
   for (int b = 0; b < NB; ++b) acc[b] = warp_sum(acc[b]);
   // lane b writes batch row b of column n
-  int pos = p.pos;
-  if (p.seq_len_dev != nullptr) pos = device_seq_len(p.seq_len_dev, p.pos + 1, p.l_cap, nullptr) - 1;
   float mine = 0.f;
 #pragma unroll
   for (int b = 0; b < NB; ++b)
     if (lane == b) mine = acc[b];
-  if (lane < p.batch && lane < NB) {
-    const int b = lane;
-    const int qcols = p.h_q * p.d, kcols = p.h_k * p.d;
-    const __nv_bfloat16 v = __float2bfloat16_rn(mine);
-    uint16_t bits;
-    memcpy(&bits, &v, 2);
-    if (n < qcols) {
-      p.q[(size_t)b * qcols + n] = bits;
-    } else if (n < qcols + kcols) {
-      const int h = (n - qcols) / p.d, c = (n - qcols) % p.d;
-      p.k_cache[(((size_t)b * p.h_k + h) * p.l_cap + pos) * p.d + c] = bits;
-    } else {
-      const int u = (n - qcols - kcols) / p.d, c = (n - qcols - kcols) % p.d;
-      p.v_cache[(((size_t)b * p.h_v + u) * p.l_cap + pos) * p.d + c] = bits;
+  if (lane < p.batch && lane < NB) qkv_store(p, n, lane, qkv_position(p), mine);
+}
+
+// Batch 2 .. 16 (up to 32 flops per weight byte pair: too many for CUDA cores
+// to keep up with the weight stream): tcgen05.  The weight matrix is the A
+// operand (M = 128 output columns per tile, K-major: row n of w_qkv), x the B
+// operand (N = 16 batch rows, zero-padded); D[n][b] accumulates in TMEM.  The
+// hidden dimension is split `splits` (<= 8) ways so that about one CTA per SM
+// streams a share of the weights through a TMA ring; the splits of a tile form
+// one thread-block cluster, each leaves its fp32 partial tile in its shared
+// memory, and after a cluster barrier CTA r adds the partials of batch rows
+// r, r + splits, ... in split order over distributed shared memory (the sum
+// does not depend on timing) and writes the bf16 outputs.
+constexpr int kQkvABytes = kQkvTileM * kQkvTileK * 2;   // 16 KB weight tile
+constexpr int kQkvBBytes = kQkvN * kQkvTileK * 2;       // 2 KB x tile
+constexpr int kQkvPartBytes = kQkvN * kQkvTileM * 4;    // 8 KB fp32 partial tile
+constexpr int kQkvMmaThreads = 128;
+
+__host__ __device__ constexpr int qkv_mma_part_offset(int stages, int kbs_max) {
+  return stages * kQkvABytes + kbs_max * kQkvBBytes;
+}
+__host__ __device__ constexpr int qkv_mma_bar_offset(int stages, int kbs_max) {
+  return qkv_mma_part_offset(stages, kbs_max) + kQkvPartBytes;
+}
+__host__ __device__ constexpr int qkv_mma_smem_bytes(int stages, int kbs_max) {
+  return qkv_mma_bar_offset(stages, kbs_max) + 256 + 1024;  // barriers and flags, alignment slack
+}
+
+__global__ void __launch_bounds__(kQkvMmaThreads)
+    saga_qkv_mma_kernel(const __grid_constant__ CUtensorMap tw, const QkvParams p) {
+  constexpr uint32_t IDESC = umma_idesc_bf16(kQkvTileM, kQkvN);
+  constexpr uint32_t TMEM_COLS = 32;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* xs = smem + p.stages * kQkvABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + qkv_mma_bar_offset(p.stages, p.kbs_max));
+  uint64_t* empty = full + 8;
+  uint64_t* accf = empty + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, tile = blockIdx.y;
+  const int kb0 = (int)((long long)split * p.kb_total / p.splits);
+  const int nkb = (int)((long long)(split + 1) * p.kb_total / p.splits) - kb0;  // >= 1: splits <= kb_total
+  const int m0 = tile * kQkvTileM;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < p.stages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
     }
+    mbar_init(accf, 1);
+    mbar_init_fence();
+    tma_prefetch_desc(&tw);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  int issued = 0;
+  if (threadIdx.x == 0) {  // the first ring's worth of weight tiles, before the dependency wait
+    const int first = min(nkb, p.stages);
+    for (int i = 0; i < first; ++i) {
+      mbar_arrive_expect_tx(&full[i], kQkvABytes);
+      tma_load_2d(smem + i * kQkvABytes, &tw, &full[i], (kb0 + i) * kQkvTileK, m0);
+    }
+    issued = first;
+  }
+  pdl_trigger();
+  pdl_wait();
+  // x rows of this split's k-blocks into the 128-byte swizzle layout (16-byte
+  // chunk c of row b at chunk position c ^ (b mod 8)); rows past the batch and
+  // elements past hidden are zero.  Thread t owns chunk c = t mod 8 of row
+  // b = t / 8 in every k-block; eight k-blocks' loads are in flight at once.
+  static_assert(kQkvMmaThreads == kQkvN * 8, "one thread per 16-byte chunk of a k-block's x tile");
+  {
+    const int c = threadIdx.x & 7, b = threadIdx.x >> 3;
+    const bool row_live = b < p.batch;
+    const uint16_t* xrow = p.x + (size_t)(row_live ? b : 0) * p.hidden;
+    uint8_t* xdst = xs + b * 128 + ((c ^ (b & 7)) << 4);
+    for (int kq = 0; kq < nkb; kq += 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int k = (kb0 + kq + j) * kQkvTileK + c * 8;
+        v[j] = make_uint4(0u, 0u, 0u, 0u);
+        if (row_live && kq + j < nkb && k < p.hidden) v[j] = __ldg(reinterpret_cast<const uint4*>(xrow + k));
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (kq + j < nkb) *reinterpret_cast<uint4*>(xdst + (kq + j) * kQkvBBytes) = v[j];
+    }
+  }
+  fence_proxy_async_shared();  // the generic-proxy writes above, seen by the tensor core
+  __syncthreads();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kb = issued; kb < nkb; ++kb) {
+        const int st = kb % p.stages, round = kb / p.stages;
+        if (!mbar_wait(&empty[st], (round - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[st], kQkvABytes);
+        tma_load_2d(smem + st * kQkvABytes, &tw, &full[st], (kb0 + kb) * kQkvTileK, m0);
+        issued = kb + 1;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int st = kb % p.stages, round = kb / p.stages;
+        if (!mbar_wait(&full[st], round & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(smem + st * kQkvABytes), b0 = smem_u32(xs + kb * kQkvBBytes);
+#pragma unroll
+        for (int k = 0; k < kQkvTileK / 16; ++k)
+          umma_bf16(tmem_base, umma_sdesc_sw128(a0 + k * 32), umma_sdesc_sw128(b0 + k * 32), IDESC,
+                    (kb > 0 || k > 0) ? 1u : 0u);
+        umma_commit(&empty[st]);
+      }
+      umma_commit(accf);  // arrives once every MMA issued has completed (also after an abort)
+    }
+    __syncwarp();
+  }
+  // epilogue: thread t holds output column m0 + t (TMEM lane t), batch rows in columns 0 .. 15
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, abort_flag) && *abort_flag == 0);
+  tc_fence_after();
+  float v[kQkvN];
+  if (ok) {
+    tmem_ld16(tmem_base + ((uint32_t)(warp * 32) << 16), v);
+  } else {
+#pragma unroll
+    for (int b = 0; b < kQkvN; ++b) v[b] = 0.f;
+  }
+  const int n = m0 + threadIdx.x;
+  const int pos = qkv_position(p);
+  float* part = reinterpret_cast<float*>(smem + qkv_mma_part_offset(p.stages, p.kbs_max)) + threadIdx.x;
+#pragma unroll
+  for (int b = 0; b < kQkvN; ++b) part[b * kQkvTileM] = v[b];
+  cluster_sync_all();  // every split's partial tile is in place
+  for (int b = split; b < p.batch; b += p.splits) {
+    float pv[kQkvMaxSplits];
+#pragma unroll
+    for (int r = 0; r < kQkvMaxSplits; ++r) pv[r] = r < p.splits ? ld_dsmem_f32(part + b * kQkvTileM, r) : 0.f;
+    float acc = pv[0];
+#pragma unroll
+    for (int r = 1; r < kQkvMaxSplits; ++r)
+      if (r < p.splits) acc += pv[r];
+    if (n < p.n_cols) qkv_store(p, n, b, pos, acc);
+  }
+  cluster_sync_all();  // no CTA leaves while a peer may still read its partial
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag != 0) {
+    if (threadIdx.x == 0) {
+      flag_status(p.status, SAGA_STATUS_TIMEOUT);
+      for (int t = (issued > p.stages ? issued - p.stages : 0); t < issued; ++t)
+        mbar_wait_drain(&full[t % p.stages], (t / p.stages) & 1);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -2297,15 +2476,48 @@ static cudaError_t run_qkv(const QkvParams& p, cudaStream_t st) {
                   p);
 }
 
-// The QKV projection for batch <= 16 (the register array is sized by the
-// smallest of 1, 2, 4, 8, 16 that holds the batch).
-cudaError_t launch_qkv(const QkvParams& p, cudaStream_t st) {
-  if (p.batch <= 1) return run_qkv<1>(p, st);
-  if (p.batch <= 2) return run_qkv<2>(p, st);
-  if (p.batch <= 4) return run_qkv<4>(p, st);
-  if (p.batch <= 8) return run_qkv<8>(p, st);
-  if (p.batch <= 16) return run_qkv<16>(p, st);
-  return cudaErrorInvalidValue;
+// Split of the hidden dimension for the tensor-core projection: about one CTA
+// per SM over all tiles, each split holding at most kQkvMaxKb k-blocks of x.
+void qkv_mma_plan(int n_cols, int hidden, int sms, int* m_tiles, int* splits, int* kb_total, int* stages,
+                  int* kbs_max) {
+  *m_tiles = (n_cols + kQkvTileM - 1) / kQkvTileM;
+  *kb_total = (hidden + kQkvTileK - 1) / kQkvTileK;
+  int sp = std::min(kQkvMaxSplits, std::max(1, sms / *m_tiles));
+  sp = std::max(sp, (*kb_total + kQkvMaxKb - 1) / kQkvMaxKb);  // <= kQkvMaxSplits: hidden is bounded
+  *splits = std::min(sp, *kb_total);
+  *kbs_max = (*kb_total + *splits - 1) / *splits;
+  *stages = std::min(*kbs_max, kQkvMaxStages);
+}
+
+// The QKV projection: batch 1 on CUDA cores, batch 2 .. 16 on the tensor cores.
+cudaError_t launch_qkv(const QkvParams& p, const CUtensorMap& tw, cudaStream_t st) {
+  if (p.batch < kQkvMmaMinBatch) {
+    if (p.batch <= 1) return run_qkv<1>(p, st);
+    if (p.batch <= 2) return run_qkv<2>(p, st);
+    if (p.batch <= 4) return run_qkv<4>(p, st);
+    if (p.batch <= 8) return run_qkv<8>(p, st);
+    return run_qkv<16>(p, st);
+  }
+  static std::atomic<uint64_t> prepared{0};
+  const int bytes = qkv_mma_smem_bytes(p.stages, p.kbs_max);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(saga_qkv_mma_kernel), qkv_mma_smem_bytes(kQkvMaxStages, kQkvMaxKb),
+                              prepared);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.splits, (p.n_cols + kQkvTileM - 1) / kQkvTileM);
+  cfg.blockDim = dim3(kQkvMmaThreads);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;  // the splits of a tile: one cluster
+  attr[0].val.clusterDim.x = p.splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, saga_qkv_mma_kernel, tw, p);
 }
 
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st) {

@@ -32,7 +32,7 @@ EXPORTED = ("saga_workspace_bytes", "saga_kv_append", "atopn_refresh_threshold",
             "saga_noalloc_scratch_bytes", "saga_decode_attn_noalloc", "saga_noalloc_get_status",
             "saga_noalloc_last_error", "saga_decode_step", "saga_test_expire_next_wait", "saga_read_probe_sink_words",
             "saga_read_probe", "saga_merge_workspace_bytes", "saga_key_head_merge", "saga_merge_last_error",
-            "saga_qkv_project")
+            "saga_qkv_project", "saga_qkv_workspace_bytes")
 
 
 class SagaError(RuntimeError):
@@ -77,8 +77,10 @@ def load(path: Optional[str] = None):
     lib.saga_workspace_bytes.restype = ctypes.c_size_t
     lib.saga_kv_append.argtypes = [sp, _P, _P, _P, _P, _I, _P, _P]
     lib.saga_kv_append.restype = _I
-    lib.saga_qkv_project.argtypes = [sp, _I, _P, _P, _P, _P, _P, _I, _P, _P]
+    lib.saga_qkv_project.argtypes = [sp, _I, _P, _P, _P, _P, _P, _I, _P, _P, ctypes.c_size_t, _P]
     lib.saga_qkv_project.restype = _I
+    lib.saga_qkv_workspace_bytes.argtypes = [sp, _I]
+    lib.saga_qkv_workspace_bytes.restype = ctypes.c_size_t
     lib.atopn_refresh_threshold.argtypes = [sp, _P, _P, _I, _P, _I, _P, _P, ctypes.c_size_t, _P]
     lib.atopn_refresh_threshold.restype = _I
     lib.atopn_select_workspace_bytes.argtypes = [_I]
@@ -181,9 +183,22 @@ def saga_kv_append(shape: SagaShape, k_cache, v_cache, k_new, v_new, pos: int, s
                                  int(pos), _ptr(seq_len_dev), _stream(stream)))
 
 
-def saga_qkv_project(shape: SagaShape, x, w_qkv, q_out, k_cache, v_cache, pos: int, seq_len_dev=None,
-                     stream=None):
-    """Eq. 1 for the new token: q_out = x W_Q, and x W_K, x W_V written into row pos of the caches."""
+def saga_qkv_workspace_bytes(shape: SagaShape, hidden: int) -> int:
+    n = load().saga_qkv_workspace_bytes(ctypes.byref(shape), int(hidden))
+    if n == 0:
+        raise SagaError(SAGA_ERR_ARG, load().saga_last_error().decode(errors="replace"))
+    return int(n)
+
+
+def alloc_qkv_workspace(shape: SagaShape, hidden: int, device=None) -> torch.Tensor:
+    """Zero-filled workspace of saga_qkv_workspace_bytes(shape, hidden) bytes on `device`."""
+    return torch.zeros(saga_qkv_workspace_bytes(shape, hidden), dtype=torch.uint8, device=device or "cuda")
+
+
+def saga_qkv_project(shape: SagaShape, x, w_qkv, q_out, k_cache, v_cache, pos: int, workspace=None,
+                     seq_len_dev=None, stream=None):
+    """Eq. 1 for the new token: q_out = x W_Q, and x W_K, x W_V written into row pos of the caches.
+    Returns the workspace (a fresh zero-filled one when none is passed)."""
     B, hq, hk, hv, d, lc = shape.astuple()
     if not isinstance(x, torch.Tensor) or x.dim() != 2:
         raise SagaError(SAGA_ERR_ARG, "x must be a 2-D tensor [batch, hidden]")
@@ -195,8 +210,16 @@ def saga_qkv_project(shape: SagaShape, x, w_qkv, q_out, k_cache, v_cache, pos: i
     _expect(v_cache, "v_cache", torch.bfloat16, (B, hv, lc, d))
     if seq_len_dev is not None:
         _expect(seq_len_dev, "seq_len_dev", torch.int32)
+    if workspace is None:
+        n = load().saga_qkv_workspace_bytes(ctypes.byref(shape), D)
+        if n:  # else the call below reports why
+            workspace = torch.zeros(n, dtype=torch.uint8, device=x.device)
+    if workspace is not None:
+        _expect(workspace, "workspace", torch.uint8)
     _check(load().saga_qkv_project(ctypes.byref(shape), D, _ptr(x), _ptr(w_qkv), _ptr(q_out), _ptr(k_cache),
-                                   _ptr(v_cache), int(pos), _ptr(seq_len_dev), _stream(stream)))
+                                   _ptr(v_cache), int(pos), _ptr(seq_len_dev), _ptr(workspace),
+                                   0 if workspace is None else workspace.numel(), _stream(stream)))
+    return workspace
 
 
 def atopn_refresh_threshold(shape: SagaShape, q, k_cache, seq_len: int, n_top: int, tau, workspace,

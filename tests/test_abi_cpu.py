@@ -31,7 +31,7 @@ def test_header_declares_the_binding_names():
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.saga_abi_version() == 101
+    assert lib.saga_abi_version() == 102
 
 
 def _shape(**kw):
@@ -137,8 +137,11 @@ def test_merge_rejects_null_and_misaligned(lib):
                                    None) == saga.SAGA_ERR_WORKSPACE
 
 
-def _qkv(lib, shape, hidden=256, x=FAKE, pos=0):
-    return lib.saga_qkv_project(ctypes.byref(shape), hidden, x, FAKE, FAKE, FAKE, FAKE, pos, None, None)
+WS = ctypes.c_void_p(0x100000)  # 256-byte aligned, never dereferenced
+
+
+def _qkv(lib, shape, hidden=256, x=FAKE, pos=0, ws=WS):
+    return lib.saga_qkv_project(ctypes.byref(shape), hidden, x, FAKE, FAKE, FAKE, FAKE, pos, None, ws, 1 << 30, None)
 
 
 def test_qkv_projection_validation(lib):
@@ -152,4 +155,10 @@ def test_qkv_projection_validation(lib):
     assert _qkv(lib, s, pos=-1) == saga.SAGA_ERR_ARG
     assert _qkv(lib, _shape(d=96)) == saga.SAGA_ERR_UNSUPPORTED
     assert _qkv(lib, _shape(h_q=4096, h_k=64, h_v=64, d=128), hidden=1 << 16) == saga.SAGA_ERR_UNSUPPORTED
+    assert _qkv(lib, s, ws=None) == saga.SAGA_ERR_WORKSPACE
+    assert _qkv(lib, s, ws=ctypes.c_void_p(0x100010)) == saga.SAGA_ERR_WORKSPACE  # not 256-byte aligned
+    assert lib.saga_qkv_workspace_bytes(ctypes.byref(_shape(batch=17)), 256) == 0
+    assert lib.saga_qkv_workspace_bytes(ctypes.byref(s), 12) == 0
+    assert lib.saga_qkv_workspace_bytes(ctypes.byref(s), 16384) == 256
+    assert _qkv(lib, s, hidden=16392) == saga.SAGA_ERR_UNSUPPORTED
     assert lib.saga_last_error()

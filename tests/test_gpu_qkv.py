@@ -1,12 +1,16 @@
 """The decode-step QKV projection (eq. 1 with SAGA head counts) on the GPU against the fp64 oracle.
 
 Inputs: x ~ N(0, 1) and weights ~ N(0, 1/D), both rounded to bf16 on the CPU (the oracle reads the same
-bf16 values, so every product x_k w_kn is exact in fp32 and only the summation order differs).  The
-kernel sums each column in fp32: every lane a sequential run of D / 32 products, then a 5-level
-shuffle tree, so its sum is within e = (D / 32 + 8) 2^-24 sum_k |x_k w_kn| of the exact value; the one
-rounding to bf16 adds at most 2^-8 of the value (half a bf16 ulp).  The test bound is
-|out - exact| <= 2^-8 (|exact| + e) + e, element by element.  Rows of the caches other than pos must be
-bit-identical to what was there.
+bf16 values, so every product x_k w_kn is exact in fp32 and only the summation order differs).  Batch 1
+runs on CUDA cores: every lane a sequential run of D / 32 products, then a 5-level shuffle tree, at most
+D / 32 + 5 roundings of half an ulp.  Batch 2 .. 16 runs on the tensor cores: one accumulation per
+16-element MMA step (the tensor core may truncate rather than round: a full ulp each), then at most 8
+split partials added in order.  Both stay within e = (D / 8 + 64) 2^-24 sum_k |x_k w_kn| of
+the exact value; the one rounding to bf16 adds at most 2^-8 of the value
+(half a bf16 ulp).  The test bound is |out - exact| <= 2^-8 (|exact| + e) + e, element by element.  Rows of
+the caches other than pos must be bit-identical to what was there, and a second call on the same
+workspace must reproduce the first bit for bit (the split partials are added in a fixed order).
+Cases that need a split of the hidden dimension run the cluster reduction; the 8-wide hidden runs one split.
 """
 import numpy as np
 import pytest
@@ -37,7 +41,7 @@ def _inputs(B, D, h_q, h_k, h_v, d, l_cap, seed):
 
 
 def _bound(x, w, exact, B, D):
-    e = (D / 32 + 8) * 2.0 ** -24 * (np.abs(x) @ np.abs(w).T)  # [B, n_cols]
+    e = (D / 8 + 64) * 2.0 ** -24 * (np.abs(x) @ np.abs(w).T)  # [B, n_cols]
     return 2.0 ** -8 * (np.abs(exact) + e) + e
 
 
@@ -47,8 +51,13 @@ def _run(B, D, h_q, h_k, h_v, d, l_cap, pos, seed, dev_len=None):
     xg, wg, kcg, vcg = x.cuda(), w.cuda(), kc0.cuda(), vc0.cuda()
     q = torch.full((B, h_q, d), float("nan"), dtype=torch.bfloat16, device="cuda")
     sl = None if dev_len is None else torch.tensor([dev_len], dtype=torch.int32, device="cuda")
-    saga.saga_qkv_project(shape, xg, wg, q, kcg, vcg, pos, seq_len_dev=sl)
+    ws = saga.saga_qkv_project(shape, xg, wg, q, kcg, vcg, pos, seq_len_dev=sl)
     torch.cuda.synchronize()
+    first = (q.clone(), kcg.clone(), vcg.clone())
+    saga.saga_qkv_project(shape, xg, wg, q, kcg, vcg, pos, workspace=ws, seq_len_dev=sl)
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(first, (q, kcg, vcg))), "second call differs"
+    assert saga.saga_get_status(ws) == 0
     return x, w, kc0, vc0, q.cpu(), kcg.cpu(), vcg.cpu()
 
 
@@ -77,9 +86,11 @@ def _check(B, D, h_q, h_k, h_v, d, l_cap, pos, seed, dev_len=None, expect_pos=No
     assert torch.equal(kc[:, :, other], kc0[:, :, other]) and torch.equal(vc[:, :, other], vc0[:, :, other])
 
 
-# (B, D, h_q, h_k, h_v, d, l_cap, pos): the two SAGA models' projection shapes at batch 1 and 16, a ragged
-# batch, hidden sizes that leave a ragged last chunk (1000, 2056) or a single 8-element piece, and
-# the first and last cache rows.
+# (B, D, h_q, h_k, h_v, d, l_cap, pos): the two SAGA models' projection shapes at batch 1 and 16, ragged
+# batches, hidden sizes that leave a ragged last chunk or k-block (1000, 2056, 4104) or a single 8-element
+# piece, output widths that end in a partial 128-column tile (448, 2816), splits longer than the weight
+# ring (4096: 8 k-blocks per split), a projection of 148 tiles whose splits stage 32 k-blocks of x each,
+# and the first and last cache rows.
 CASES = [
     (1, 2048, 32, 2, 8, 64, 40, 17),      # Llama-3.2-1B SAGA projection
     (16, 2048, 32, 2, 8, 64, 9, 8),
@@ -88,7 +99,10 @@ CASES = [
     (3, 1000, 8, 8, 8, 64, 7, 3),         # plain MHA head counts, ragged batch and hidden
     (5, 2056, 16, 2, 4, 128, 6, 5),
     (2, 8, 4, 1, 2, 64, 3, 1),
+    (1, 8, 4, 1, 2, 64, 3, 2),
     (9, 4096, 8, 1, 8, 128, 4, 2),
+    (1, 4104, 8, 1, 8, 128, 4, 1),
+    (4, 4096, 128, 4, 16, 128, 2, 1),
 ]
 
 
@@ -103,6 +117,20 @@ def test_qkv_position_from_device():
     # out-of-range lengths clamp into the cache, as the attention kernels do
     _check(2, 512, 8, 2, 4, 64, 12, pos=3, seed=6, dev_len=0, expect_pos=0)
     _check(2, 512, 8, 2, 4, 64, 12, pos=3, seed=7, dev_len=99, expect_pos=11)
+
+
+def test_qkv_workspace_too_small():
+    shape = saga.SagaShape(4, 8, 1, 8, 64, 4)
+    x = torch.zeros((4, 2048), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((17 * 64, 2048), dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros((4, 8, 64), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((4, 1, 4, 64), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros((4, 8, 4, 64), dtype=torch.bfloat16, device="cuda")
+    need = saga.saga_qkv_workspace_bytes(shape, 2048)
+    ws = torch.zeros(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(saga.SagaError) as e:
+        saga.saga_qkv_project(shape, x, w, q, kc, vc, 0, workspace=ws)
+    assert e.value.code == saga.SAGA_ERR_WORKSPACE
 
 
 def test_qkv_rejects_bad_arguments():
