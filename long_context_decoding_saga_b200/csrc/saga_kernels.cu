@@ -1135,6 +1135,11 @@ __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const Spl
 // they come in by TMA with its key rows, and each epilogue warp runs the
 // softmax and the value sum of its 32 rows per tile (online, no lists).
 // Warp roles as in the split kernel; the partials feed the same combine.
+#ifndef SAGA_DENSE_SETS
+#define SAGA_DENSE_SETS 2
+#endif
+constexpr int kDenseSetsSmallGroups = SAGA_DENSE_SETS;  // epilogue sets of the dense kernel at <= 4 heads
+
 template <int D, int NP>
 struct DenseSmem {
   static constexpr int NATOM = D / 64;
@@ -1143,7 +1148,11 @@ struct DenseSmem {
   static constexpr int NPM = mma_n<NP>();
   static constexpr int NACC = acc_bufs<NP>();
   static constexpr int QPAD = ((NATOM * NPM * 128 + 1023) / 1024) * 1024;
-  static constexpr int PBUF_BYTES = 4 * 32 * NP * 4;  // each warp's weights of a tile, [32][NP]
+  // epilogue sets: with 4 heads a set of four warps is issue-bound on the
+  // value sums, so two sets take alternate tiles (8 epilogue warps)
+  static constexpr int ESETS = NP <= 4 ? kDenseSetsSmallGroups : 1;
+  static constexpr int THREADS = 64 + 128 * ESETS;
+  static constexpr int PBUF_BYTES = 4 * ESETS * 32 * NP * 4;  // each epilogue warp's weights of a tile, [32][NP]
   static constexpr int FIXED = QPAD + PBUF_BYTES + (2 * 4 + 2 * NACC + 1) * 8 + 16 + 1024;
   static constexpr int NSTAGE_HALF = (kSmemHalf - FIXED) / STAGE_BYTES;
   static constexpr bool TWO = NSTAGE_HALF >= 3;  // two CTAs per SM with 3 stages each
@@ -1160,7 +1169,7 @@ struct DenseSmem {
   static_assert(NSTAGE >= 2, "ring too shallow");
   static_assert(ALLOC <= kSmemLimit, "shared memory over the per-CTA limit");
   static_assert(!TWO || ALLOC <= kSmemHalf, "two CTAs per SM must fit in half the shared memory");
-  static_assert(4 * NP * (D + 2) * 4 <= NSTAGE * STAGE_BYTES, "merge buffer must fit in the ring");
+  static_assert(4 * ESETS * NP * (D + 2) * 4 <= NSTAGE * STAGE_BYTES, "merge buffer must fit in the ring");
 };
 
 // Key and value rows of tile t into its stage (128-row boxes, or 32-row
@@ -1193,7 +1202,7 @@ __device__ __forceinline__ void issue_kv_tile(int t, int start, int end, int kro
 }
 
 template <int D, int NP>
-__global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
+__global__ void __launch_bounds__(DenseSmem<D, NP>::THREADS, DenseSmem<D, NP>::CTAS_PER_SM)
     saga_dense_kernel(const __grid_constant__ CUtensorMap tk_full, const __grid_constant__ CUtensorMap tk_part,
                       const __grid_constant__ CUtensorMap tv_full, const __grid_constant__ CUtensorMap tv_part,
                       const SplitParams p) {
@@ -1204,6 +1213,8 @@ __global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
   constexpr int KBYTES = SM::KBYTES;
   constexpr int NPM = SM::NPM;
   constexpr int NACC = SM::NACC;
+  constexpr int ESETS = SM::ESETS;
+  constexpr int NEPI = 128 * ESETS;  // epilogue threads
   constexpr int DPL = D / 32;
   constexpr uint32_t TMEM_COLS = NACC * NPM <= 32 ? 32u : NACC * NPM <= 64 ? 64u : NACC * NPM <= 128 ? 128u : 256u;
   constexpr uint32_t IDESC = umma_idesc_bf16(128, NPM);
@@ -1272,7 +1283,8 @@ __global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
   constexpr int QV = (QCH + kEpiThreads - 1) / kEpiThreads;
   const int eth = threadIdx.x - 64;
   uint4 qv[QV];
-  if (warp >= 2) {
+  const bool qstage = warp >= 2 && warp < 6;  // the first epilogue set stages q
+  if (qstage) {
 #pragma unroll
     for (int k = 0; k < QV; ++k) {
       const int i = eth + k * kEpiThreads;
@@ -1295,7 +1307,7 @@ __global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
                                                         &tv_full, &tv_part);
     }
   }
-  if (warp >= 2) {
+  if (qstage) {
 #pragma unroll
     for (int k = 0; k < QV; ++k) {
       const int i = eth + k * kEpiThreads;
@@ -1350,8 +1362,12 @@ __global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    // set es of four warps takes tiles es, es + ESETS, ...; within a set the
+    // warps own the TMEM lane quarters (warp mod 4)
     const int et = threadIdx.x - 64;
-    const int q = warp & 3;  // TMEM lane quarter: rows 32q .. 32q+31 of every tile
+    const int ew = warp - 2;    // epilogue warp 0 .. 4 * ESETS - 1
+    const int eset = ew >> 2;
+    const int q = warp & 3;     // TMEM lane quarter: rows 32q .. 32q+31 of every tile
     const int erow = 32 * q + lane;
     const bool counting = p.want_counts != 0;
     float m[NP], lp[NP], o[NP][DPL];  // running max (warp-uniform), per-lane weight sums, columns of the lane
@@ -1362,11 +1378,10 @@ __global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
 #pragma unroll
       for (int e = 0; e < DPL; ++e) o[jl][e] = 0.f;
     }
-    float* pw = pbuf + q * 32 * NP;
+    float* pw = pbuf + ew * 32 * NP;
     // the lane's columns of a value row: atom (lane*DPL)/64, byte offset within the 128-byte row
     const int vcol = ((lane * DPL) / 64) * 16384 + ((lane * DPL) % 64) * 2;
-    int t = 0;
-    for (; t < ntiles; ++t) {
+    for (int t = eset; t < ntiles; t += ESETS) {
       const int stage = t % NSTAGE;
       const int abuf = t % NACC;
       if (!__all_sync(0xffffffffu, mbar_wait(&accf[abuf], (t / NACC) & 1, abort_flag))) break;
@@ -1446,14 +1461,15 @@ __global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[stage]);
     }
-    // ---- merge the four warps' states and write the split's partial
+    // ---- merge the epilogue warps' states and write the split's partial
     constexpr int REG = NP * (D + 2);
+    constexpr int NW = 4 * ESETS;
     float lw[NP];
 #pragma unroll
     for (int jl = 0; jl < NP; ++jl) lw[jl] = warp_sum(lp[jl]);
-    named_bar_sync(1, kEpiThreads);  // every warp is done with the ring (value rows)
+    named_bar_sync(1, NEPI);  // every warp is done with the ring (value rows)
     float* mrg = reinterpret_cast<float*>(ring);
-    float* mine = mrg + q * REG;
+    float* mine = mrg + ew * REG;
     if (lane == 0) {
 #pragma unroll
       for (int jl = 0; jl < NP; ++jl) {
@@ -1465,20 +1481,20 @@ __global__ void __launch_bounds__(192, DenseSmem<D, NP>::CTAS_PER_SM)
     for (int jl = 0; jl < NP; ++jl)
 #pragma unroll
       for (int e = 0; e < DPL; ++e) mine[2 * NP + jl * D + lane * DPL + e] = o[jl][e];
-    named_bar_sync(1, kEpiThreads);
+    named_bar_sync(1, NEPI);
     const size_t row0 = (size_t)b * p.h_q + j0;
-    for (int idx = et; idx < p.G * (D / 4); idx += kEpiThreads) {
+    for (int idx = et; idx < p.G * (D / 4); idx += NEPI) {
       const int jl = idx / (D / 4), c4 = idx % (D / 4);
-      float m4[4], M = -INFINITY;
+      float m4[NW], M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
+      for (int w = 0; w < NW; ++w) {
         m4[w] = mrg[w * REG + jl];
         M = fmaxf(M, m4[w]);
       }
       float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
       float lsum = 0.f;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
+      for (int w = 0; w < NW; ++w) {
         const float f = (m4[w] == -INFINITY) ? 0.f : __expf(m4[w] - M);
         const float4 v = *reinterpret_cast<const float4*>(&mrg[w * REG + 2 * NP + jl * D + c4 * 4]);
         acc4.x = fmaf(f, v.x, acc4.x);
@@ -2398,8 +2414,8 @@ static cudaError_t run_dense(const CUtensorMap& kf, const CUtensorMap& kp, const
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(saga_dense_kernel<D, NP>), K::ALLOC, prepared);
   if (e != cudaSuccess) return e;
   if (occ != nullptr)
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, saga_dense_kernel<D, NP>, 192, K::ALLOC);
-  return launch_k(saga_dense_kernel<D, NP>, grid, dim3(192), K::ALLOC, st, kf, kp, vf, vp, p);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, saga_dense_kernel<D, NP>, K::THREADS, K::ALLOC);
+  return launch_k(saga_dense_kernel<D, NP>, grid, dim3(K::THREADS), K::ALLOC, st, kf, kp, vf, vp, p);
 }
 
 // Dense attention (every token kept) for groups whose query heads share one
