@@ -16,9 +16,11 @@
 //   2. the Gram matrices G = X^T X [D, D] and S_r [d, d] on tcgen05 (bf16
 //      products, fp32 accumulation in TMEM), one kernel for both;
 //   3. per pair, in fp64: S = S_a + S_b, its eigen-decomposition by parallel
-//      cyclic Jacobi rotations, the pseudoinverse, and M(a, b);
-//   4. per pair and head r in {a, b}: the loss term tr(D^T G D S_r) with
-//      D = M(a, b) - W_K^r (eq. 13 through the Gram matrices), in fp64;
+//      cyclic Jacobi rotations, the pseudoinverse, and the factors A, B of
+//      M(a, b) = W_K^a A + W_K^b B;
+//   4. G W_K^r per head, then per pair M(a, b) and the loss terms
+//      tr(D^T G D S_r) with D = M(a, b) - W_K^r, r in {a, b} (eq. 13 through
+//      the Gram matrices), in fp64;
 //   5. the minimum-weight perfect matching by enumerating every matching,
 //      and the merged projections of the chosen pairs.
 #include <cuda.h>
@@ -210,88 +212,98 @@ __host__ __device__ inline void pair_of(int p, int h, int* a, int* b) {
 
 struct PairParams {
   const float* Sg;  // [h_k][128][128] fp32 Gram blocks S_r (top-left d x d)
-  double* V;        // [npairs][d][d] eigenvectors (work)
+  double* V;        // [npairs][d][d] eigenvectors (work, used where they do not fit in shared memory)
   double* A;        // [npairs][d][d] S_a (S_a + S_b)^+
   double* B;        // [npairs][d][d] S_b (S_a + S_b)^+
-  int d, h_k;
+  int h_k;
   int max_sweeps;
   double rtol;      // eigenvalues at most rtol * max |eigenvalue| count as zero
 };
 
+// Shared memory of the pseudoinverse kernel: S, and V where it fits (d = 64),
+// rows padded by one element so that column walks do not hit one bank.
+__host__ __device__ constexpr int pinv_smem_bytes(int d) { return (d == 64 ? 2 : 1) * d * (d + 1) * 8; }
+
 // One CTA per pair: S = S_a + S_b (fp64, in shared memory) is diagonalised by
-// parallel cyclic Jacobi rotations (each round rotates d/2 disjoint index
-// pairs chosen by the circle method, angles computed from the round's start;
-// S <- J^T S J, V <- V J), until the off-diagonal mass is below 1e-30 of the
-// total or after max_sweeps sweeps.  Then S^+ = V diag(1/lambda) V^T over the
-// eigenvalues above the cut, and A = S_a S^+, B = S_b S^+.
-__global__ void __launch_bounds__(256) merge_pinv_kernel(const PairParams p) {
-  extern __shared__ double sh[];  // S [d][d], later S^+
-  __shared__ double cs[64], sn[64];
-  __shared__ int pp[64], qq[64];
-  __shared__ double red[256 / 32];
+// parallel cyclic Jacobi rotations.  Each round rotates the d/2 disjoint index
+// pairs of the circle method, all angles computed from the round's start;
+// S <- J^T S J is applied one 2 x 2 block (row pair, column pair) per thread
+// step (the blocks partition S, so one barrier separates rounds) and V <- V J
+// one (row, column pair) per step.  Sweeps stop once the off-diagonal mass is
+// below 1e-30 of the total, or after max_sweeps.  Then S^+ = V diag(1/lambda)
+// V^T over the eigenvalues above the cut, and A = S_a S^+, B = S_b S^+.
+template <int DD, int NT>
+__global__ void __launch_bounds__(NT) merge_pinv_kernel(const PairParams p) {
+  constexpr int H = DD / 2;
+  constexpr bool VSH = DD == 64;  // V beside S in shared memory
+  constexpr int LS = DD + 1;                // row stride of S
+  constexpr int LV = VSH ? DD + 1 : DD;     // row stride of V
+  extern __shared__ double sh[];
+  __shared__ double cs[H], sn[H];
+  __shared__ int pp[H], qq[H];
+  __shared__ double red_off[NT / 32], red_tot[NT / 32];
+  __shared__ double inv[DD];
   __shared__ int done;
-  const int d = p.d, pair = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
+  __shared__ double lmax;
+  const int pair = blockIdx.x, tid = threadIdx.x;
   int a, b;
   pair_of(pair, p.h_k, &a, &b);
   double* S = sh;
-  double* V = p.V + (size_t)pair * d * d;
+  double* V = VSH ? sh + DD * LS : p.V + (size_t)pair * DD * DD;
   const float* Sa = p.Sg + (size_t)a * 128 * 128;
   const float* Sb = p.Sg + (size_t)b * 128 * 128;
-  for (int e = tid; e < d * d; e += nt) {
-    const int i = e / d, j = e % d;
-    S[e] = (double)Sa[i * 128 + j] + (double)Sb[i * 128 + j];
-    V[e] = i == j ? 1.0 : 0.0;
+  for (int e = tid; e < DD * DD; e += NT) {
+    const int i = e / DD, j = e % DD;
+    S[i * LS + j] = (double)Sa[i * 128 + j] + (double)Sb[i * 128 + j];
+    V[i * LV + j] = i == j ? 1.0 : 0.0;
   }
   __syncthreads();
   for (int sweep = 0; sweep < p.max_sweeps; ++sweep) {
     // convergence: off-diagonal mass against the total
     double off = 0.0, tot = 0.0;
-    for (int e = tid; e < d * d; e += nt) {
-      const double v = S[e] * S[e];
+    for (int e = tid; e < DD * DD; e += NT) {
+      const int i = e / DD, j = e % DD;
+      const double v = S[i * LS + j] * S[i * LS + j];
       tot += v;
-      if (e / d != e % d) off += v;
+      if (i != j) off += v;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       off += __shfl_xor_sync(0xffffffffu, off, o);
       tot += __shfl_xor_sync(0xffffffffu, tot, o);
     }
-    if ((tid & 31) == 0) red[tid >> 5] = off;
-    __syncthreads();
-    if (tid == 0) {
-      double o2 = 0.0;
-      for (int w = 0; w < nt / 32; ++w) o2 += red[w];
-      red[0] = o2;
+    if ((tid & 31) == 0) {
+      red_off[tid >> 5] = off;
+      red_tot[tid >> 5] = tot;
     }
     __syncthreads();
-    const double off_all = red[0];
-    __syncthreads();
-    if ((tid & 31) == 0) red[tid >> 5] = tot;
-    __syncthreads();
     if (tid == 0) {
-      double t2 = 0.0;
-      for (int w = 0; w < nt / 32; ++w) t2 += red[w];
-      done = (off_all <= 1e-30 * t2) ? 1 : 0;
+      double o2 = 0.0, t2 = 0.0;
+      for (int w = 0; w < NT / 32; ++w) {
+        o2 += red_off[w];
+        t2 += red_tot[w];
+      }
+      done = (o2 <= 1e-30 * t2) ? 1 : 0;
     }
     __syncthreads();
     if (done) break;
-    for (int r = 0; r < d - 1; ++r) {
+    for (int r = 0; r < DD - 1; ++r) {
       // round r of the circle method: (r, d-1) and ((r+k) mod (d-1), (r-k) mod (d-1)), k = 1 .. d/2-1
-      if (tid < d / 2) {
+      if (tid < H) {
         int i, j;
         if (tid == 0) {
           i = r;
-          j = d - 1;
+          j = DD - 1;
         } else {
-          i = (r + tid) % (d - 1);
-          j = (r - tid + (d - 1)) % (d - 1);
+          i = (r + tid) % (DD - 1);
+          j = (r - tid + (DD - 1)) % (DD - 1);
         }
         if (i > j) {
           const int x = i;
           i = j;
           j = x;
         }
-        const double apq = S[i * d + j], app = S[i * d + i], aqq = S[j * d + j];
+        const double apq = S[i * LS + j], app = S[i * LS + i], aqq = S[j * LS + j];
         double c = 1.0, s = 0.0;
         if (apq != 0.0) {
           const double theta = (aqq - app) / (2.0 * apq);
@@ -305,164 +317,329 @@ __global__ void __launch_bounds__(256) merge_pinv_kernel(const PairParams p) {
         qq[tid] = j;
       }
       __syncthreads();
-      // rows: S <- J^T S
-      for (int e = tid; e < (d / 2) * d; e += nt) {
-        const int k = e / d, col = e % d;
-        const int i = pp[k], j = qq[k];
-        const double c = cs[k], s = sn[k];
-        const double si = S[i * d + col], sj = S[j * d + col];
-        S[i * d + col] = c * si - s * sj;
-        S[j * d + col] = s * si + c * sj;
+      // S <- J^T S J, block (row pair m, column pair n): rows first, then columns
+      for (int e = tid; e < H * H; e += NT) {
+        const int m = e / H, n = e % H;
+        const int i = pp[m], j = qq[m], k = pp[n], l = qq[n];
+        const double cm = cs[m], sm = sn[m], cn = cs[n], snn = sn[n];
+        const double xik = S[i * LS + k], xil = S[i * LS + l], xjk = S[j * LS + k], xjl = S[j * LS + l];
+        const double yik = cm * xik - sm * xjk, yjk = sm * xik + cm * xjk;
+        const double yil = cm * xil - sm * xjl, yjl = sm * xil + cm * xjl;
+        S[i * LS + k] = cn * yik - snn * yil;
+        S[i * LS + l] = snn * yik + cn * yil;
+        S[j * LS + k] = cn * yjk - snn * yjl;
+        S[j * LS + l] = snn * yjk + cn * yjl;
       }
-      __syncthreads();
-      // columns: S <- S J, V <- V J
-      for (int e = tid; e < (d / 2) * d; e += nt) {
-        const int k = e / d, row = e % d;
-        const int i = pp[k], j = qq[k];
-        const double c = cs[k], s = sn[k];
-        const double si = S[row * d + i], sj = S[row * d + j];
-        S[row * d + i] = c * si - s * sj;
-        S[row * d + j] = s * si + c * sj;
-        const double vi = V[row * d + i], vj = V[row * d + j];
-        V[row * d + i] = c * vi - s * vj;
-        V[row * d + j] = s * vi + c * vj;
+      // V <- V J
+      for (int e = tid; e < DD * H; e += NT) {
+        const int row = e / H, n = e % H;
+        const int k = pp[n], l = qq[n];
+        const double cn = cs[n], snn = sn[n];
+        const double vk = V[row * LV + k], vl = V[row * LV + l];
+        V[row * LV + k] = cn * vk - snn * vl;
+        V[row * LV + l] = snn * vk + cn * vl;
       }
       __syncthreads();
     }
   }
   // eigenvalues on the diagonal; the cut, then S^+ = V diag(inv) V^T (into shared memory over S)
-  __shared__ double inv[128];
-  __shared__ double lmax;
   if (tid == 0) {
-    double m = 0.0;
-    for (int i = 0; i < d; ++i) m = fmax(m, fabs(S[i * d + i]));
-    lmax = m;
+    double mx = 0.0;
+    for (int i = 0; i < DD; ++i) mx = fmax(mx, fabs(S[i * LS + i]));
+    lmax = mx;
   }
   __syncthreads();
-  if (tid < d) {
-    const double l = S[tid * d + tid];
+  if (tid < DD) {
+    const double l = S[tid * LS + tid];
     inv[tid] = fabs(l) > p.rtol * lmax ? 1.0 / l : 0.0;
   }
   __syncthreads();
-  for (int e = tid; e < d * d; e += nt) {
-    const int i = e / d, j = e % d;
+  for (int e = tid; e < DD * DD; e += NT) {
+    const int i = e / DD, j = e % DD;
     double acc = 0.0;
-    for (int k = 0; k < d; ++k) acc += V[i * d + k] * inv[k] * V[j * d + k];
-    S[e] = acc;
+    for (int k = 0; k < DD; ++k) acc += V[i * LV + k] * inv[k] * V[j * LV + k];
+    S[i * LS + j] = acc;
   }
   __syncthreads();
-  double* A = p.A + (size_t)pair * d * d;
-  double* B = p.B + (size_t)pair * d * d;
-  for (int e = tid; e < d * d; e += nt) {
-    const int i = e / d, j = e % d;
+  double* A = p.A + (size_t)pair * DD * DD;
+  double* B = p.B + (size_t)pair * DD * DD;
+  for (int e = tid; e < DD * DD; e += NT) {
+    const int i = e / DD, j = e % DD;
     double x = 0.0, y = 0.0;
-    for (int k = 0; k < d; ++k) {
-      x += (double)Sa[i * 128 + k] * S[k * d + j];
-      y += (double)Sb[i * 128 + k] * S[k * d + j];
+    for (int k = 0; k < DD; ++k) {
+      x += (double)Sa[i * 128 + k] * S[k * LS + j];
+      y += (double)Sb[i * 128 + k] * S[k * LS + j];
     }
     A[e] = x;
     B[e] = y;
   }
 }
 
-// ---------------------------------------------------------------- merged projections
-// M(a, b)[i][:] = W_a[i][:] A + W_b[i][:] B (eq. 15), fp64, one warp per row i.
-struct ProjectParams {
-  const float* W;  // [h_k][D][d]
-  const double* A;
-  const double* B;
-  double* M;       // [npairs][D][d]
-  int D, d, h_k;
-};
-
-__global__ void __launch_bounds__(256) merge_project_kernel(const ProjectParams p) {
-  const int pair = blockIdx.y, d = p.d;
-  int a, b;
-  pair_of(pair, p.h_k, &a, &b);
-  const double* A = p.A + (size_t)pair * d * d;
-  const double* B = p.B + (size_t)pair * d * d;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x * 8 + warp;
-  if (i >= p.D) return;
-  const float* wa = p.W + ((size_t)a * p.D + i) * d;
-  const float* wb = p.W + ((size_t)b * p.D + i) * d;
-  double* out = p.M + ((size_t)pair * p.D + i) * d;
-  for (int j = lane; j < d; j += 32) {
-    double acc = 0.0;
-    for (int k = 0; k < d; ++k) acc += (double)wa[k] * A[k * d + j] + (double)wb[k] * B[k * d + j];
-    out[j] = acc;
-  }
-}
-
 // ---------------------------------------------------------------- 4. loss terms
-// For pair p and head r (side 0: a, side 1: b), with D_r = M(a, b) - W_r:
-//   tr(D_r^T G D_r S_r) = sum_{i, c} (G D_r)[i][c] (D_r S_r)[i][c]
-// (eq. 13 written through G = X^T X and S_r).  One CTA per (64-row block of
-// i, side, pair): G D_r for its rows in 32-wide steps of k through shared
-// memory, D_r S_r for its rows, and the block's partial sum in a fixed order.
-struct LossParams {
+// Eq. 13 through the Gram matrices: for pair (a, b) and head r in {a, b},
+// with D_r = M(a, b) - W_r, the term is tr(D_r^T G D_r S_r) =
+// sum_{i, c} (G D_r)[i][c] (D_r S_r)[i][c].  Since M(a, b) = W_a A + W_b B,
+// G D_r = (GW_a A + GW_b B) - GW_r with GW_r = G W_r computed once per head;
+// that leaves per pair two (D x 2d) x (2d x d) products and two D x d x d ones
+// instead of a D x D x d product per pair and head.  All sums in fp64.
+//
+// Thread tile of both kernels: 4 rows (4 ty .. 4 ty + 3 of a 64-row block) by
+// DD / 16 columns (tx, tx + 16, ...), 256 threads.
+constexpr int kRows = 64;  // rows per CTA
+constexpr int kKc = 16;    // k-chunk staged in shared memory
+
+struct GwParams {
   const float* G;  // [Dp][Dp] (ld = ldg)
   long long ldg;
   const float* W;  // [h_k][D][d]
-  const float* Sg; // [h_k][128][128]
-  const double* M; // [npairs][D][d]
-  double* partial; // [npairs][2][nblk]
-  int D, d, h_k, nblk;
+  double* GW;      // [h_k][D][d]
+  int D;
 };
 
-constexpr int kLossRows = 64, kLossK = 32;
+constexpr int kGwRows = 128;  // rows of G W_r per CTA (8 per thread)
+constexpr int kGwKc = 32;     // k-chunk of the G W_r product
+constexpr int kGwLd = kGwKc + 4;  // padded row of the staged G chunk (16-byte rows, no common bank)
 
-template <int DH>
+// Two buffers of raw fp32 chunks: G [kGwRows][kGwLd] and W_r [kGwKc][DD].
+template <int DD>
+__host__ __device__ constexpr int gw_smem_bytes() { return 2 * (kGwRows * kGwLd + kGwKc * DD) * 4; }
+
+// GW_r = G W_r: grid (row blocks of 128, h_k); thread tile 8 rows (8 ty .. 8 ty + 7)
+// by DD / 16 columns (tx, tx + 16, ...).  The next k-chunk is copied into the
+// other buffer by cp.async while the current one is multiplied.
+template <int DD>
+__global__ void __launch_bounds__(256) merge_gw_kernel(const GwParams p) {
+  constexpr int CT = DD / 16;
+  extern __shared__ __align__(16) float gsf[];
+  float* Gs = gsf;                          // [2][kGwRows][kGwLd]
+  float* Ws = gsf + 2 * kGwRows * kGwLd;    // [2][kGwKc][DD]
+  const int r = blockIdx.y, i0 = blockIdx.x * kGwRows, tid = threadIdx.x;
+  const int ty = tid >> 4, tx = tid & 15;
+  const float* Wr = p.W + (size_t)r * p.D * DD;
+  // rows i0 .. i0 + 127 and columns below the padded size are inside G (zero past D)
+  auto issue = [&](int k0, int buf) {
+    float* gd = Gs + buf * kGwRows * kGwLd;
+    for (int c = tid; c < kGwRows * (kGwKc / 4); c += 256) {
+      const int rr = c / (kGwKc / 4), q4 = c % (kGwKc / 4);
+      cp_async16(gd + rr * kGwLd + q4 * 4, p.G + (size_t)(i0 + rr) * p.ldg + k0 + q4 * 4);
+    }
+    float* wd = Ws + buf * kGwKc * DD;
+    for (int c = tid; c < kGwKc * (DD / 4); c += 256) {
+      const int kk = c / (DD / 4), q4 = c % (DD / 4), gk = k0 + kk;
+      cp_async16_zfill(wd + kk * DD + q4 * 4, Wr + (size_t)(gk < p.D ? gk : 0) * DD + q4 * 4, gk < p.D);
+    }
+    cp_async_commit();
+  };
+  double acc[8][CT];
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+#pragma unroll
+    for (int c = 0; c < CT; ++c) acc[q][c] = 0.0;
+  issue(0, 0);
+  int buf = 0;
+  for (int k0 = 0; k0 < p.D; k0 += kGwKc, buf ^= 1) {
+    const bool more = k0 + kGwKc < p.D;
+    if (more) {
+      issue(k0 + kGwKc, buf ^ 1);
+      cp_async_wait_one();
+    } else {
+      cp_async_wait_all();
+    }
+    __syncthreads();
+    const float* gs = Gs + buf * kGwRows * kGwLd;
+    const float* ws = Ws + buf * kGwKc * DD;
+#pragma unroll 4
+    for (int kk = 0; kk < kGwKc; ++kk) {
+      double g[8], w[CT];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) g[q] = (double)gs[(8 * ty + q) * kGwLd + kk];
+#pragma unroll
+      for (int c = 0; c < CT; ++c) w[c] = (double)ws[kk * DD + tx + 16 * c];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+#pragma unroll
+        for (int c = 0; c < CT; ++c) acc[q][c] = fma(g[q], w[c], acc[q][c]);
+    }
+    __syncthreads();  // this buffer is refilled two chunks on
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int gi = i0 + 8 * ty + q;
+    if (gi < p.D)
+#pragma unroll
+      for (int c = 0; c < CT; ++c) p.GW[((size_t)r * p.D + gi) * DD + tx + 16 * c] = acc[q][c];
+  }
+}
+
+struct LossParams {
+  const float* W;     // [h_k][D][d]
+  const double* GW;   // [h_k][D][d]
+  const double* A;    // [npairs][d][d]
+  const double* B;    // [npairs][d][d]
+  const float* Sg;    // [h_k][128][128]
+  double* M;          // [npairs][D][d] (written)
+  double* partial;    // [npairs][nblk] (written)
+  int D, h_k, nblk;
+};
+
+template <int DD>
+struct LossSmem {
+  // phase 1, two buffers of raw k-chunks: A and B rows (fp64), the block's
+  // W_a and W_b columns (fp32) and GW_a and GW_b columns (fp64)
+  static constexpr int AB = 2 * kKc * DD * 8;
+  static constexpr int XW = 2 * kRows * kKc * 4;
+  static constexpr int YW = 2 * kRows * kKc * 8;
+  static constexpr int BUF = AB + XW + YW;
+  static constexpr int P1 = 2 * BUF;
+  // phase 2: M rows (fp64), W_r rows and S_r (fp32)
+  static constexpr int M_OFF = 0;
+  static constexpr int W_OFF = kRows * DD * 8;
+  static constexpr int S_OFF = W_OFF + kRows * DD * 4;
+  static constexpr int P2 = S_OFF + DD * DD * 4;
+  static constexpr int BYTES = P1 > P2 ? P1 : P2;
+};
+
+// Merged projections and the pair's loss over one 64-row block: grid (row blocks, pairs).
+template <int DD>
 __global__ void __launch_bounds__(256) merge_loss_kernel(const LossParams p) {
-  extern __shared__ double lsh[];  // Gs [64][32], Ds [32][d]
+  using SM = LossSmem<DD>;
+  constexpr int CT = DD / 16;
+  extern __shared__ double lsh[];
   __shared__ double red[8];
-  constexpr int d = DH;
-  const int blk = blockIdx.x, side = blockIdx.y, pair = blockIdx.z, tid = threadIdx.x;
+  const int blk = blockIdx.x, pair = blockIdx.y, tid = threadIdx.x;
+  const int ty = tid >> 4, tx = tid & 15;
+  const int i0 = blk * kRows;
   int a, b;
   pair_of(pair, p.h_k, &a, &b);
-  const int r = side == 0 ? a : b;
-  const double* M = p.M + (size_t)pair * p.D * d;
-  const float* Wr = p.W + (size_t)r * p.D * d;
-  double* Gs = lsh;
-  double* Ds = lsh + kLossRows * kLossK;
-  // thread layout for the 64 x d block of G D: row ri = tid / 4 (64 rows), columns cj = (tid % 4) + 4 c
-  const int ri = tid >> 2, c0 = tid & 3;
-  constexpr int CPT = d / 4;  // columns per thread
-  double acc[CPT];
+  const double* A = p.A + (size_t)pair * DD * DD;
+  const double* B = p.B + (size_t)pair * DD * DD;
+  const float* Wa = p.W + (size_t)a * p.D * DD;
+  const float* Wb = p.W + (size_t)b * p.D * DD;
+  const double* GWa = p.GW + (size_t)a * p.D * DD;
+  const double* GWb = p.GW + (size_t)b * p.D * DD;
+  // phase 1: M = W_a A + W_b B and GM = GW_a A + GW_b B for this thread's rows and columns
+  double m[4][CT], gm[4][CT];
 #pragma unroll
-  for (int c = 0; c < CPT; ++c) acc[c] = 0.0;
-  const int i0 = blk * kLossRows;
-  for (int k0 = 0; k0 < p.D; k0 += kLossK) {
-    for (int e = tid; e < kLossRows * kLossK; e += 256) {
-      const int rr = e / kLossK, kk = e % kLossK;
-      const int gi = i0 + rr, gk = k0 + kk;
-      Gs[e] = (gi < p.D && gk < p.D) ? (double)p.G[(size_t)gi * p.ldg + gk] : 0.0;
-    }
-    for (int e = tid; e < kLossK * d; e += 256) {
-      const int kk = e / d, c = e % d, gk = k0 + kk;
-      Ds[e] = gk < p.D ? M[(size_t)gk * d + c] - (double)Wr[(size_t)gk * d + c] : 0.0;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int kk = 0; kk < kLossK; ++kk) {
-      const double g = Gs[ri * kLossK + kk];
+  for (int q = 0; q < 4; ++q)
 #pragma unroll
-      for (int c = 0; c < CPT; ++c) acc[c] += g * Ds[kk * d + c0 + 4 * c];
+    for (int c = 0; c < CT; ++c) m[q][c] = gm[q][c] = 0.0;
+  {
+    uint8_t* base = reinterpret_cast<uint8_t*>(lsh);
+    auto issue = [&](int k0, int buf) {
+      uint8_t* bb = base + buf * SM::BUF;
+      double* As = reinterpret_cast<double*>(bb);  // [kKc][DD], then Bs
+      float* Xa = reinterpret_cast<float*>(bb + SM::AB);  // [kRows][kKc], then Xb
+      double* Ya = reinterpret_cast<double*>(bb + SM::AB + SM::XW);  // [kRows][kKc], then Yb
+      for (int c = tid; c < kKc * DD / 2; c += 256) {
+        cp_async16(As + 2 * c, A + (size_t)k0 * DD + 2 * c);
+        cp_async16(As + kKc * DD + 2 * c, B + (size_t)k0 * DD + 2 * c);
+      }
+      for (int c = tid; c < kRows * (kKc / 4); c += 256) {
+        const int rr = c / (kKc / 4), q4 = c % (kKc / 4), gi = i0 + rr;
+        const size_t o = (size_t)(gi < p.D ? gi : 0) * DD + k0 + q4 * 4;
+        cp_async16_zfill(Xa + rr * kKc + q4 * 4, Wa + o, gi < p.D);
+        cp_async16_zfill(Xa + kRows * kKc + rr * kKc + q4 * 4, Wb + o, gi < p.D);
+      }
+      for (int c = tid; c < kRows * (kKc / 2); c += 256) {
+        const int rr = c / (kKc / 2), q2 = c % (kKc / 2), gi = i0 + rr;
+        const size_t o = (size_t)(gi < p.D ? gi : 0) * DD + k0 + q2 * 2;
+        cp_async16_zfill(Ya + rr * kKc + q2 * 2, GWa + o, gi < p.D);
+        cp_async16_zfill(Ya + kRows * kKc + rr * kKc + q2 * 2, GWb + o, gi < p.D);
+      }
+      cp_async_commit();
+    };
+    issue(0, 0);
+    int buf = 0;
+    for (int k0 = 0; k0 < DD; k0 += kKc, buf ^= 1) {
+      const bool more = k0 + kKc < DD;
+      if (more) {
+        issue(k0 + kKc, buf ^ 1);
+        cp_async_wait_one();
+      } else {
+        cp_async_wait_all();
+      }
+      __syncthreads();
+      const uint8_t* bb = base + buf * SM::BUF;
+      const double* As = reinterpret_cast<const double*>(bb);
+      const double* Bs = As + kKc * DD;
+      const float* Xa = reinterpret_cast<const float*>(bb + SM::AB);
+      const float* Xb = Xa + kRows * kKc;
+      const double* Ya = reinterpret_cast<const double*>(bb + SM::AB + SM::XW);
+      const double* Yb = Ya + kRows * kKc;
+#pragma unroll 2
+      for (int kk = 0; kk < kKc; ++kk) {
+        double av[CT], bv[CT];
+#pragma unroll
+        for (int c = 0; c < CT; ++c) {
+          av[c] = As[kk * DD + tx + 16 * c];
+          bv[c] = Bs[kk * DD + tx + 16 * c];
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int rr = 4 * ty + q;
+          const double xa = (double)Xa[rr * kKc + kk], xb = (double)Xb[rr * kKc + kk];
+          const double ya = Ya[rr * kKc + kk], yb = Yb[rr * kKc + kk];
+#pragma unroll
+          for (int c = 0; c < CT; ++c) {
+            m[q][c] = fma(xa, av[c], fma(xb, bv[c], m[q][c]));
+            gm[q][c] = fma(ya, av[c], fma(yb, bv[c], gm[q][c]));
+          }
+        }
+      }
+      __syncthreads();  // this buffer is refilled two chunks on
     }
-    __syncthreads();
   }
-  // (D S_r)[i][c] for this thread's row and columns, and the product with G D
-  double part = 0.0;
-  const int gi = i0 + ri;
-  if (gi < p.D) {
-    const float* Sr = p.Sg + (size_t)r * 128 * 128;
+  // phase 2: M rows to global and shared memory; then for r in {a, b}: (M - W_r) S_r against GM - GW_r
+  double* Ms = reinterpret_cast<double*>(reinterpret_cast<char*>(lsh) + SM::M_OFF);  // [kRows][DD]
+  float* Wsm = reinterpret_cast<float*>(reinterpret_cast<char*>(lsh) + SM::W_OFF);  // [kRows][DD]
+  float* Ss = reinterpret_cast<float*>(reinterpret_cast<char*>(lsh) + SM::S_OFF);   // [DD][DD]
+  double* Mout = p.M + (size_t)pair * p.D * DD;
 #pragma unroll
-    for (int c = 0; c < CPT; ++c) {
-      const int col = c0 + 4 * c;
-      double ds = 0.0;
-      for (int k = 0; k < d; ++k)
-        ds += (M[(size_t)gi * d + k] - (double)Wr[(size_t)gi * d + k]) * (double)Sr[k * 128 + col];
-      part += acc[c] * ds;
+  for (int q = 0; q < 4; ++q) {
+    const int rr = 4 * ty + q, gi = i0 + rr;
+#pragma unroll
+    for (int c = 0; c < CT; ++c) {
+      Ms[rr * DD + tx + 16 * c] = m[q][c];
+      if (gi < p.D) Mout[(size_t)gi * DD + tx + 16 * c] = m[q][c];
+    }
+  }
+  double part = 0.0;
+  for (int side = 0; side < 2; ++side) {
+    const int r = side == 0 ? a : b;
+    const float* Wr = side == 0 ? Wa : Wb;
+    const double* GWr = side == 0 ? GWa : GWb;
+    const float* Sr = p.Sg + (size_t)r * 128 * 128;
+    __syncthreads();  // Ms written / the previous side is done with Wsm and Ss
+    for (int e = tid; e < kRows * DD; e += 256) {
+      const int rr = e / DD, c = e % DD, gi = i0 + rr;
+      Wsm[e] = gi < p.D ? Wr[(size_t)gi * DD + c] : 0.f;
+    }
+    for (int e = tid; e < DD * DD; e += 256) Ss[e] = Sr[(e / DD) * 128 + (e % DD)];
+    __syncthreads();
+    double ds[4][CT];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int c = 0; c < CT; ++c) ds[q][c] = 0.0;
+#pragma unroll 2
+    for (int k = 0; k < DD; ++k) {
+      double sv[CT];
+#pragma unroll
+      for (int c = 0; c < CT; ++c) sv[c] = (double)Ss[k * DD + tx + 16 * c];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int rr = 4 * ty + q;
+        const double dk = Ms[rr * DD + k] - (double)Wsm[rr * DD + k];
+#pragma unroll
+        for (int c = 0; c < CT; ++c) ds[q][c] = fma(dk, sv[c], ds[q][c]);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int gi = i0 + 4 * ty + q;
+      if (gi < p.D)
+#pragma unroll
+        for (int c = 0; c < CT; ++c) part += (gm[q][c] - GWr[(size_t)gi * DD + tx + 16 * c]) * ds[q][c];
     }
   }
 #pragma unroll
@@ -472,7 +649,7 @@ __global__ void __launch_bounds__(256) merge_loss_kernel(const LossParams p) {
   if (tid == 0) {
     double s = 0.0;
     for (int w = 0; w < 8; ++w) s += red[w];
-    p.partial[((size_t)pair * 2 + side) * p.nblk + blk] = s;
+    p.partial[(size_t)pair * p.nblk + blk] = s;
   }
 }
 
@@ -482,10 +659,9 @@ __global__ void __launch_bounds__(256) merge_loss_kernel(const LossParams p) {
 // with the c-th remaining one at each level, c taken as mixed-radix digits
 // (most significant first), so indices follow the order of the usual
 // recursive enumeration.  Each thread scores a range of indices; the lowest
-// total wins (ties: the lowest index).  The chosen pairs' merged projections
-// are then written out as fp32, pairs ordered by their smaller head.
+// total wins (ties: the lowest index).
 struct MatchParams {
-  const double* partial;  // [npairs][2][nblk]
+  const double* partial;  // [npairs][nblk]
   const double* M;        // [npairs][D][d]
   float* pair_loss;       // [h_k][h_k]
   int* pairing;           // [h_k]
@@ -511,8 +687,7 @@ __global__ void __launch_bounds__(1024) merge_match_kernel(const MatchParams p) 
     int a, b;
     pair_of(pr, h, &a, &b);
     double s = 0.0;
-    for (int side = 0; side < 2; ++side)
-      for (int k = 0; k < p.nblk; ++k) s += p.partial[((size_t)pr * 2 + side) * p.nblk + k];
+    for (int k = 0; k < p.nblk; ++k) s += p.partial[(size_t)pr * p.nblk + k];
     w[a][b] = w[b][a] = s;
   }
   __syncthreads();
@@ -582,20 +757,24 @@ __global__ void __launch_bounds__(1024) merge_match_kernel(const MatchParams p) 
     }
     for (int i = 0; i < h; ++i) p.pairing[i] = partner[i];
   }
-  __syncthreads();
-  // merged projections of the chosen pairs, pairs ordered by their smaller head
-  int slot = 0;
-  for (int a = 0; a < h; ++a) {
-    const int b = partner[a];
-    if (b < a) continue;
-    int pr = 0;
-    for (int x = 0; x < a; ++x) pr += h - 1 - x;
-    pr += b - a - 1;
-    const double* src = p.M + (size_t)pr * p.D * p.d;
-    float* dst = p.merged + (size_t)slot * p.D * p.d;
-    for (long long e = tid; e < (long long)p.D * p.d; e += blockDim.x) dst[e] = (float)src[e];
-    ++slot;
+}
+
+// The merged projections of the chosen pairs as fp32, pairs ordered by their
+// smaller head: grid (ceil(D d / 1024), h_k / 2), one element per thread.
+__global__ void __launch_bounds__(1024) merge_emit_kernel(const MatchParams p) {
+  const int slot = blockIdx.y;
+  int a = 0, seen = -1, b = 0;
+  for (; a < p.h_k; ++a) {
+    b = p.pairing[a];
+    if (b > a && ++seen == slot) break;
   }
+  if (a >= p.h_k) return;
+  int pr = 0;
+  for (int x = 0; x < a; ++x) pr += p.h_k - 1 - x;
+  pr += b - a - 1;
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < (long long)p.D * p.d)
+    p.merged[(size_t)slot * p.D * p.d + e] = (float)p.M[(size_t)pr * p.D * p.d + e];
 }
 
 }  // namespace merge
@@ -615,7 +794,7 @@ int merge_fail(int code, const char* msg) {
 
 struct MergeLayout {
   long long Dp, Tp, Kq;
-  size_t status, xt, qt, g, sg, v, a, b, m, partial, total;
+  size_t status, xt, qt, g, sg, v, a, b, gw, m, partial, total;
   int npairs, nblk;
 };
 
@@ -628,7 +807,7 @@ MergeLayout merge_layout(const saga_merge_shape* s) {
   L.Tp = round_up(s->tokens, kTileK);
   L.Kq = round_up((long long)g * s->tokens, kTileK);
   L.npairs = s->h_k * (s->h_k - 1) / 2;
-  L.nblk = (s->hidden + kLossRows - 1) / kLossRows;
+  L.nblk = (s->hidden + kRows - 1) / kRows;
   size_t off = 0;
   L.status = off;
   off = a256(off + 16);
@@ -646,10 +825,12 @@ MergeLayout merge_layout(const saga_merge_shape* s) {
   off = a256(off + (size_t)L.npairs * s->d * s->d * 8);
   L.b = off;
   off = a256(off + (size_t)L.npairs * s->d * s->d * 8);
+  L.gw = off;
+  off = a256(off + (size_t)s->h_k * s->hidden * s->d * 8);
   L.m = off;
   off = a256(off + (size_t)L.npairs * s->hidden * s->d * 8);
   L.partial = off;
-  off = a256(off + (size_t)L.npairs * 2 * L.nblk * 8);
+  off = a256(off + (size_t)L.npairs * L.nblk * 8);
   L.total = off;
   return L;
 }
@@ -751,13 +932,22 @@ int saga_key_head_merge(const saga_merge_shape* s, const void* x, const void* q,
   if (!(g_smem_set.load() & bit)) {
     e = cudaFuncSetAttribute(merge_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmSmem::ALLOC);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(merge_pinv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 128 * 8);
+      e = cudaFuncSetAttribute(merge_pinv_kernel<64, 1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               pinv_smem_bytes(64));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(merge_pinv_kernel<128, 1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               pinv_smem_bytes(128));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(merge_gw_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, gw_smem_bytes<64>());
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(merge_gw_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               gw_smem_bytes<128>());
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(merge_loss_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (kLossRows * kLossK + kLossK * 64) * 8);
+                               LossSmem<64>::BYTES);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(merge_loss_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (kLossRows * kLossK + kLossK * 128) * 8);
+                               LossSmem<128>::BYTES);
     if (e != cudaSuccess) return cuda_err(e, "cudaFuncSetAttribute");
     g_smem_set.fetch_or(bit);
   }
@@ -791,39 +981,43 @@ int saga_key_head_merge(const saga_merge_shape* s, const void* x, const void* q,
   pp.V = reinterpret_cast<double*>(base + L.v);
   pp.A = reinterpret_cast<double*>(base + L.a);
   pp.B = reinterpret_cast<double*>(base + L.b);
-  pp.d = s->d;
   pp.h_k = s->h_k;
   pp.max_sweeps = 30;
   pp.rtol = 1e-5;  // the Gram matrices carry fp32 rounding: smaller eigenvalues are noise
-  merge_pinv_kernel<<<L.npairs, 256, (size_t)s->d * s->d * 8, st>>>(pp);
-  ProjectParams jp{};
-  jp.W = w_k;
-  jp.A = pp.A;
-  jp.B = pp.B;
-  jp.M = reinterpret_cast<double*>(base + L.m);
-  jp.D = s->hidden;
-  jp.d = s->d;
-  jp.h_k = s->h_k;
-  merge_project_kernel<<<dim3((s->hidden + 7) / 8, L.npairs), 256, 0, st>>>(jp);
+  if (s->d == 64)
+    merge_pinv_kernel<64, 1024><<<L.npairs, 1024, pinv_smem_bytes(64), st>>>(pp);
+  else
+    merge_pinv_kernel<128, 1024><<<L.npairs, 1024, pinv_smem_bytes(128), st>>>(pp);
+  GwParams gw{};
+  gw.G = G;
+  gw.ldg = L.Dp;
+  gw.W = w_k;
+  gw.GW = reinterpret_cast<double*>(base + L.gw);
+  gw.D = s->hidden;
+  const dim3 ggrid((unsigned)((s->hidden + kGwRows - 1) / kGwRows), (unsigned)s->h_k);
+  if (s->d == 64)
+    merge_gw_kernel<64><<<ggrid, 256, gw_smem_bytes<64>(), st>>>(gw);
+  else
+    merge_gw_kernel<128><<<ggrid, 256, gw_smem_bytes<128>(), st>>>(gw);
   LossParams lp{};
-  lp.G = G;
-  lp.ldg = L.Dp;
   lp.W = w_k;
+  lp.GW = gw.GW;
+  lp.A = pp.A;
+  lp.B = pp.B;
   lp.Sg = Sg;
-  lp.M = jp.M;
+  lp.M = reinterpret_cast<double*>(base + L.m);
   lp.partial = reinterpret_cast<double*>(base + L.partial);
   lp.D = s->hidden;
-  lp.d = s->d;
   lp.h_k = s->h_k;
   lp.nblk = L.nblk;
-  const size_t loss_smem = (size_t)(kLossRows * kLossK + kLossK * s->d) * 8;
+  const dim3 lgrid((unsigned)L.nblk, (unsigned)L.npairs);
   if (s->d == 64)
-    merge_loss_kernel<64><<<dim3(L.nblk, 2, L.npairs), 256, loss_smem, st>>>(lp);
+    merge_loss_kernel<64><<<lgrid, 256, LossSmem<64>::BYTES, st>>>(lp);
   else
-    merge_loss_kernel<128><<<dim3(L.nblk, 2, L.npairs), 256, loss_smem, st>>>(lp);
+    merge_loss_kernel<128><<<lgrid, 256, LossSmem<128>::BYTES, st>>>(lp);
   MatchParams mp{};
   mp.partial = lp.partial;
-  mp.M = jp.M;
+  mp.M = lp.M;
   mp.pair_loss = pair_loss;
   mp.pairing = pairing;
   mp.merged = w_k_merged;
@@ -833,6 +1027,8 @@ int saga_key_head_merge(const saga_merge_shape* s, const void* x, const void* q,
   mp.D = s->hidden;
   mp.d = s->d;
   merge_match_kernel<<<1, 1024, 0, st>>>(mp);
+  merge_emit_kernel<<<dim3((unsigned)(((long long)s->hidden * s->d + 1023) / 1024), (unsigned)(s->h_k / 2)), 1024, 0,
+                      st>>>(mp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_err(e, "merge launch");
   return SAGA_OK;
