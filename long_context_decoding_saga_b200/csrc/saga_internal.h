@@ -163,8 +163,38 @@ constexpr int kQkvMaxHidden = kQkvMaxSplits * kQkvMaxKb * kQkvTileK;  // 16384
 #define SAGA_QKV_MMA_MIN_BATCH 2
 #endif
 constexpr int kQkvMmaMinBatch = SAGA_QKV_MMA_MIN_BATCH;  // smallest batch sent to the tensor cores
-void qkv_mma_plan(int n_cols, int hidden, int sms, int* m_tiles, int* splits, int* kb_total, int* stages,
-                  int* kbs_max);
+
+// Split of the hidden dimension for the tensor-core projection: about one CTA
+// per SM over all tiles (at most kQkvMaxSplits, one cluster), each split
+// holding at most kQkvMaxKb k-blocks of x (so hidden <= kQkvMaxHidden).
+__host__ inline void qkv_mma_plan(int n_cols, int hidden, int sms, int* m_tiles, int* splits, int* kb_total,
+                                  int* stages, int* kbs_max) {
+  *m_tiles = (n_cols + kQkvTileM - 1) / kQkvTileM;
+  *kb_total = (hidden + kQkvTileK - 1) / kQkvTileK;
+  int sp = sms / *m_tiles;
+  if (sp > kQkvMaxSplits) sp = kQkvMaxSplits;
+  if (sp < 1) sp = 1;
+  const int need = (*kb_total + kQkvMaxKb - 1) / kQkvMaxKb;
+  if (sp < need) sp = need;
+  *splits = sp < *kb_total ? sp : *kb_total;
+  *kbs_max = (*kb_total + *splits - 1) / *splits;
+  *stages = *kbs_max < kQkvMaxStages ? *kbs_max : kQkvMaxStages;
+}
+
+// Shared memory of the tensor-core projection: weight ring, x tiles, the fp32
+// partial tile, barriers (and 1024 bytes of alignment slack).
+constexpr int kQkvABytes = kQkvTileM * kQkvTileK * 2;   // 16 KB weight tile
+constexpr int kQkvBBytes = kQkvN * kQkvTileK * 2;       // 2 KB x tile
+constexpr int kQkvPartBytes = kQkvN * kQkvTileM * 4;    // 8 KB fp32 partial tile
+__host__ __device__ constexpr int qkv_mma_part_offset(int stages, int kbs_max) {
+  return stages * kQkvABytes + kbs_max * kQkvBBytes;
+}
+__host__ __device__ constexpr int qkv_mma_bar_offset(int stages, int kbs_max) {
+  return qkv_mma_part_offset(stages, kbs_max) + kQkvPartBytes;
+}
+__host__ __device__ constexpr int qkv_mma_smem_bytes(int stages, int kbs_max) {
+  return qkv_mma_bar_offset(stages, kbs_max) + 256 + 1024;
+}
 
 struct AppendParams {
   uint16_t* k_cache;

@@ -2148,20 +2148,7 @@ __global__ void __launch_bounds__(kQkvWarps * 32, NB == 1 ? 4 : 2) saga_qkv_kern
 // memory, and after a cluster barrier CTA r adds the partials of batch rows
 // r, r + splits, ... in split order over distributed shared memory (the sum
 // does not depend on timing) and writes the bf16 outputs.
-constexpr int kQkvABytes = kQkvTileM * kQkvTileK * 2;   // 16 KB weight tile
-constexpr int kQkvBBytes = kQkvN * kQkvTileK * 2;       // 2 KB x tile
-constexpr int kQkvPartBytes = kQkvN * kQkvTileM * 4;    // 8 KB fp32 partial tile
 constexpr int kQkvMmaThreads = 128;
-
-__host__ __device__ constexpr int qkv_mma_part_offset(int stages, int kbs_max) {
-  return stages * kQkvABytes + kbs_max * kQkvBBytes;
-}
-__host__ __device__ constexpr int qkv_mma_bar_offset(int stages, int kbs_max) {
-  return qkv_mma_part_offset(stages, kbs_max) + kQkvPartBytes;
-}
-__host__ __device__ constexpr int qkv_mma_smem_bytes(int stages, int kbs_max) {
-  return qkv_mma_bar_offset(stages, kbs_max) + 256 + 1024;  // barriers and flags, alignment slack
-}
 
 __global__ void __launch_bounds__(kQkvMmaThreads)
     saga_qkv_mma_kernel(const __grid_constant__ CUtensorMap tw, const QkvParams p) {
@@ -2490,19 +2477,6 @@ static cudaError_t run_qkv(const QkvParams& p, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   return launch_k(saga_qkv_kernel<NB>, dim3((p.n_cols + kQkvWarps - 1) / kQkvWarps), dim3(kQkvWarps * 32), bytes, st,
                   p);
-}
-
-// Split of the hidden dimension for the tensor-core projection: about one CTA
-// per SM over all tiles, each split holding at most kQkvMaxKb k-blocks of x.
-void qkv_mma_plan(int n_cols, int hidden, int sms, int* m_tiles, int* splits, int* kb_total, int* stages,
-                  int* kbs_max) {
-  *m_tiles = (n_cols + kQkvTileM - 1) / kQkvTileM;
-  *kb_total = (hidden + kQkvTileK - 1) / kQkvTileK;
-  int sp = std::min(kQkvMaxSplits, std::max(1, sms / *m_tiles));
-  sp = std::max(sp, (*kb_total + kQkvMaxKb - 1) / kQkvMaxKb);  // <= kQkvMaxSplits: hidden is bounded
-  *splits = std::min(sp, *kb_total);
-  *kbs_max = (*kb_total + *splits - 1) / *splits;
-  *stages = std::min(*kbs_max, kQkvMaxStages);
 }
 
 // The QKV projection: batch 1 on CUDA cores, batch 2 .. 16 on the tensor cores.

@@ -1,8 +1,10 @@
 """Host-side index logic of the CUDA path, compiled with g++ and run on the CPU:
 the context-split ranges partition [0, L) at multiples of the 32-token unit,
-the prefetch ranges cover them for every length up to the capacity, and the
+the prefetch ranges cover them for every length up to the capacity, the
 CTA coordinates of a split grid (with head sub-groups) cover every query head
-of every batch exactly once per split."""
+of every batch exactly once per split, and the tensor-core QKV projection's
+split of the hidden dimension stays within its cluster, its shared memory and
+its staged x region."""
 import os
 import shutil
 import subprocess
@@ -69,6 +71,23 @@ int main() {
           }
         }
     for (size_t i = 0; i < seen.size(); ++i) CHECK(seen[i] == 1, "hsplit %d: (split, batch, head) %zu seen %d times", hsplit, i, seen[i]);
+  }
+  // tensor-core QKV projection plan: splits in [1, 8] and <= the k-blocks, every
+  // split non-empty and within the staged x region, shared memory within a CTA's
+  const int ncols[] = {1, 64, 127, 128, 129, 448, 1088, 2176, 2688, 18944, 40000};
+  const int hiddens[] = {8, 64, 72, 1000, 1536, 2048, 2056, 4096, 4104, 8192, 16384};
+  const int smss[] = {1, 132, 148};
+  for (int nc : ncols) for (int hd : hiddens) for (int sms : smss) {
+    int mt, sp, kbt, st, kbm;
+    qkv_mma_plan(nc, hd, sms, &mt, &sp, &kbt, &st, &kbm);
+    CHECK(mt * kQkvTileM >= nc && (mt - 1) * kQkvTileM < nc, "qkv n=%d: %d tiles", nc, mt);
+    CHECK(sp >= 1 && sp <= kQkvMaxSplits && sp <= kbt, "qkv n=%d D=%d: %d splits of %d k-blocks", nc, hd, sp, kbt);
+    CHECK(kbm <= kQkvMaxKb && st >= 1 && st <= kQkvMaxStages && st <= kbm, "qkv D=%d: kbs_max %d stages %d", hd, kbm, st);
+    CHECK(qkv_mma_smem_bytes(st, kbm) <= 232448, "qkv D=%d: %d bytes of shared memory", hd, qkv_mma_smem_bytes(st, kbm));
+    for (int s = 0; s < sp; ++s) {
+      const int kb0 = (int)((long long)s * kbt / sp), nkb = (int)((long long)(s + 1) * kbt / sp) - kb0;
+      CHECK(nkb >= 1 && nkb <= kbm, "qkv D=%d split %d: %d k-blocks (max %d)", hd, s, nkb, kbm);
+    }
   }
   std::printf(fails ? "FAIL %d\n" : "ok\n", fails);
   return fails ? 1 : 0;
