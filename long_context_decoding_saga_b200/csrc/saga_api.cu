@@ -87,9 +87,16 @@ int device_sms(int* sms) {
 // as CTAs of 8 heads each (the 8-head kernel keeps two CTAs per SM and a
 // light epilogue; the sub-groups' repeated key tiles come from L2), when the
 // sub-groups split along value-head boundaries.
-int head_split(const saga_shape* s) {
+// Query heads per CTA.  At d = 64 a group of many query heads runs as
+// sub-group CTAs that share each key tile through L2: 16 heads a CTA on
+// reuse steps, 8 on the refresh path (score dump and compare/gather from the
+// scores).  Measured per step against 8 everywhere: reuse steps of the
+// 32-head groups 578 vs 725 us (batch 16) and 329 vs 418 us (batch 4);
+// refresh steps 2786 vs 2551 us with 16.
+int head_split(const saga_shape* s, bool refresh_path) {
   const int G = s->h_q / s->h_k, hpv = s->h_q / s->h_v;
-  if (s->d == 64 && G >= 16 && G % 8 == 0 && (8 % hpv == 0 || hpv % 8 == 0)) return G / 8;
+  const int sub = refresh_path ? 8 : 16;
+  if (s->d == 64 && G >= 2 * sub && G % sub == 0 && (sub % hpv == 0 || hpv % sub == 0)) return G / sub;
   return 1;
 }
 
@@ -246,7 +253,7 @@ struct NewRows {
 };
 
 void fill_split_common(SplitParams& p, const saga_shape* s, const Prepared& pr, const void* q, const void* k_cache,
-                       int seq_len, const int* seq_len_dev) {
+                       int seq_len, const int* seq_len_dev, bool refresh_path) {
   memset(&p, 0, sizeof(p));
   p.q = static_cast<const uint16_t*>(q);
   p.k_cache = static_cast<const uint16_t*>(k_cache);
@@ -260,7 +267,7 @@ void fill_split_common(SplitParams& p, const saga_shape* s, const Prepared& pr, 
   p.l_cap = s->l_cap;
   p.s_cap = pr.ws.s_cap;
   p.ld_scores = pr.ws.ld_scores;
-  p.hsplit = head_split(s);
+  p.hsplit = head_split(s, refresh_path);
   p.G = s->h_q / s->h_k / p.hsplit;
   const int hpv = s->h_q / s->h_v;  // query heads per value head
   p.nvh = p.G >= hpv ? p.G / hpv : 1;
@@ -272,8 +279,8 @@ void fill_split_common(SplitParams& p, const saga_shape* s, const Prepared& pr, 
   p.part_cnt = reinterpret_cast<int*>(pr.base + pr.ws.part_cnt);
 }
 
-int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, int mode, const CUtensorMap& tf,
-               const CUtensorMap& tp, int* S, bool dense = false) {
+int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, int hsplit, int mode,
+               const CUtensorMap& tf, const CUtensorMap& tp, int* S, bool dense = false) {
   int occ = 0;
   SplitParams dummy{};
   cudaError_t e = dense ? launch_dense(s->d, NP, tf, tp, tf, tp, dummy, dim3(1), nullptr, &occ)
@@ -283,7 +290,7 @@ int splits_for(const saga_shape* s, const Prepared& pr, int seq_len, int NP, int
   // A small step (at most 16 key tiles per SM) is latency-bound: one split
   // per SM, which leaves a second CTA slot to the next call's kernel (it
   // starts its setup and L2 prefetch early).  Larger steps fill every slot.
-  const int groups = s->batch * s->h_k * head_split(s);
+  const int groups = s->batch * s->h_k * hsplit;
   const long long tiles = (long long)groups * ((seq_len + kTile - 1) / kTile);
   int slots = (occ > 1 && tiles <= 16ll * pr.sms) ? pr.sms : occ * pr.sms;
   // With one split CTA per SM, the combine CTAs of the previous call (up to
@@ -308,7 +315,7 @@ int clear_status_word(const Prepared& pr, cudaStream_t st) {
 int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const void* k_cache, int seq_len,
                 const int* seq_len_dev, int n_top, float* tau, cudaStream_t st, cudaEvent_t ev_start = nullptr,
                 const NewRows& nr = NewRows(), bool clear_status = false) {
-  const int hsplit = head_split(s);
+  const int hsplit = head_split(s, true);
   const int G = s->h_q / s->h_k / hsplit, NP = np_for_group(G);
   CUtensorMap tf, tp;
   int rc = make_key_map(&tf, k_cache, s, kTile);
@@ -316,7 +323,7 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   rc = make_key_map(&tp, k_cache, s, kUnit);
   if (rc) return rc;
   int S = 1;
-  rc = splits_for(s, pr, seq_len, NP, kSplitDump, tf, tp, &S);
+  rc = splits_for(s, pr, seq_len, NP, hsplit, kSplitDump, tf, tp, &S);
   if (rc) return rc;
   const size_t rows = (size_t)s->batch * s->h_q;
   uint32_t* hist = reinterpret_cast<uint32_t*>(pr.base + pr.ws.hist);
@@ -331,7 +338,7 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   cudaError_t e = cudaMemsetAsync(hist, 0, rows * (2 * 256 + 1) * 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(hist)");
   SplitParams p;
-  fill_split_common(p, s, pr, q, k_cache, seq_len, seq_len_dev);
+  fill_split_common(p, s, pr, q, k_cache, seq_len, seq_len_dev, true);
   p.k_cache_w = nr.k_cache;
   p.v_cache_w = nr.v_cache;
   p.k_new = nr.k_new;
@@ -550,10 +557,11 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
   rc = prepare_ws(s, workspace, ws_bytes, &pr);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int hsplit = head_split(s);
-  const int G = s->h_q / s->h_k / hsplit, NP = np_for_group(G);
   const bool refresh = (step % refresh_interval) == 0;
   const bool no_threshold = n_top >= s->l_cap;  // every possible length is covered by N
+  const bool refresh_path = refresh && !no_threshold;
+  const int hsplit = head_split(s, refresh_path);
+  const int G = s->h_q / s->h_k / hsplit, NP = np_for_group(G);
   const int rows = s->batch * s->h_q;
 
   CUtensorMap tf, tp;
@@ -568,14 +576,14 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
   g_test_wait_ns = 0;
 
   SplitParams p;
-  fill_split_common(p, s, pr, q, k_cache, seq_len, seq_len_dev);
+  fill_split_common(p, s, pr, q, k_cache, seq_len, seq_len_dev, refresh_path);
   p.v_cache = static_cast<const uint16_t*>(v_cache);
   p.tau = tau;
   p.want_counts = sel_count != nullptr;
   p.idxbuf = sel_idx != nullptr ? reinterpret_cast<int*>(pr.base + pr.ws.idx) : nullptr;
   cudaError_t e;
   int S = 1;
-  if (refresh && !no_threshold) {
+  if (refresh_path) {
     rc = run_refresh(s, pr, q, k_cache, seq_len, seq_len_dev, n_top, tau, st, ev0, nr, clear_status);
     if (rc) return rc;
     // the compare/gather pass reads scores, not keys: it runs with every
@@ -604,7 +612,7 @@ int decode_impl(const saga_shape* s, const void* q, const void* k_cache, const v
       rc = make_value_map(&vp, v_cache, s, kUnit);
       if (rc) return rc;
     }
-    rc = splits_for(s, pr, seq_len, NP, mode, tf, tp, &S, dense);
+    rc = splits_for(s, pr, seq_len, NP, hsplit, mode, tf, tp, &S, dense);
     if (rc) return rc;
     p.nsplit = S;
     if (!dense) p.test_wait_ns = test_wait_ns;
