@@ -202,7 +202,7 @@ struct ListState {
   int cur, n, pend, npend;
 };
 
-template <int D, int NP>
+template <int D, int NP, int VSB = vstage_warp_bytes<D, NP>()>
 __device__ __forceinline__ EpiArgs epi_args(const SplitParams& p, int b, int j0) {
   EpiArgs ea;
   const int v_base = (int)(((long long)j0 * p.h_v) / p.h_q);
@@ -211,7 +211,7 @@ __device__ __forceinline__ EpiArgs epi_args(const SplitParams& p, int b, int j0)
   ea.G = p.G;
   ea.hpv = p.hpv;
   ea.nvh = p.nvh;
-  ea.rcapw = min(kBatch, vstage_warp_bytes<D, NP>() / (p.nvh * D * 2));
+  ea.rcapw = min(kBatch, VSB / (p.nvh * D * 2));
   ea.cpr = p.nvh * D / 8;
   ea.hmul = (65536 + p.hpv - 1) / p.hpv;
   ea.scale = p.scale;
@@ -515,14 +515,14 @@ __device__ __forceinline__ void tile_epilogue(EpiShared<NP>& es, WarpAcc<D, NP>&
 template <int D, int NP>
 __host__ __device__ constexpr int merge_floats() { return 4 * NP * (D + 2); }
 
-template <int D, int NP>
+template <int D, int NP, int VSB = vstage_warp_bytes<D, NP>()>
 __device__ __forceinline__ void tail_merge(EpiShared<NP>& es, float* mrg, const WarpAcc<D, NP>& acc,
                                            const ListState& ls, const EpiArgs& ea, const uint16_t* vstage, int q,
                                            int lane, int et, const SplitParams& p, int b, int j0, int s,
                                            bool drop_lists) {
   constexpr int DPL = WarpAcc<D, NP>::DPL;
   constexpr int REG = NP * (D + 2);
-  constexpr int VWE = vstage_warp_bytes<D, NP>();  // elements of one warp's staging area (two buffers)
+  constexpr int VWE = VSB;  // elements of one warp's staging area (two buffers)
   float* mine = mrg + q * REG;                  // m[NP], l[NP], o[NP][D]
   if (lane == 0) {
 #pragma unroll
@@ -1080,10 +1080,17 @@ __device__ __forceinline__ void load_scores(float (&dst)[NP], const float* srow,
   for (int jl = 0; jl < NP; ++jl) dst[jl] = (jl < G && tok < end) ? __ldg(srow + (size_t)jl * ld + tok) : -INFINITY;
 }
 
+// Value staging of the compare/gather pass: 4 KB per warp list buffer at
+// d = 128 (half the split kernel's), so that two of its CTAs share an SM.
+template <int D, int NP>
+__host__ __device__ constexpr int fs_vstage_warp_bytes() {
+  return (D == 128 && NP <= 16) ? 4096 : vstage_warp_bytes<D, NP>();
+}
+
 template <int D, int NP>
 struct FromScoresSmem {
   static constexpr int VST_OFF = ((int)sizeof(EpiShared<NP>) + 127) / 128 * 128;
-  static constexpr int MRG_OFF = VST_OFF + 4 * 2 * vstage_warp_bytes<D, NP>();
+  static constexpr int MRG_OFF = VST_OFF + 4 * 2 * fs_vstage_warp_bytes<D, NP>();
   static constexpr int BYTES = MRG_OFF + merge_floats<D, NP>() * 4;
 };
 
@@ -1107,9 +1114,10 @@ __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const Spl
   const bool counting = p.want_counts != 0;
 
   epi_setup<NP>(es, et, p, load_tau<NP>(et, p, b, j0, true));  // dumped scores are scaled: compare as they are
-  EpiArgs ea = epi_args<D, NP>(p, b, j0);
+  constexpr int VSB = fs_vstage_warp_bytes<D, NP>();
+  EpiArgs ea = epi_args<D, NP, VSB>(p, b, j0);
   ea.scale = 1.f;  // the dumped scores are scaled already
-  uint16_t* vstage_w = vstage + (size_t)q * 2 * (vstage_warp_bytes<D, NP>() / 2);
+  uint16_t* vstage_w = vstage + (size_t)q * 2 * (VSB / 2);
   WarpAcc<D, NP> acc;
   acc.init();
   ListState ls{0, 0, -1, 0};
@@ -1126,7 +1134,7 @@ __global__ void __launch_bounds__(kEpiThreads) saga_from_scores_kernel(const Spl
     const int tok = start + t * kTile + et;
     tile_epilogue<D, NP>(es, acc, ea, ls, q, lane, et, sc, tok, tok < end, counting, p, b, j0, start, vstage_w);
   }
-  tail_merge<D, NP>(es, mrg, acc, ls, ea, vstage, q, lane, et, p, b, j0, s, false);
+  tail_merge<D, NP, VSB>(es, mrg, acc, ls, ea, vstage, q, lane, et, p, b, j0, s, false);
 }
 
 // ============================================================================ dense kernel
