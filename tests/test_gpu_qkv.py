@@ -147,3 +147,39 @@ def test_qkv_rejects_bad_arguments():
     with pytest.raises(saga.SagaError) as e:
         saga.saga_qkv_project(shape, x[:1], w, q[:1], kc[:1], vc[:1], 4)
     assert e.value.code == saga.SAGA_ERR_ARG
+
+
+@pytest.mark.parametrize("B", [1, 4])
+def test_qkv_graph_replay_with_device_length(B):
+    """Captured once in a CUDA graph with the position read from a device length; replayed at two
+    lengths, each replay writes its own cache row and leaves the other rows alone."""
+    h_q, h_k, h_v, d, D, l_cap = 12, 1, 4, 128, 1536, 16
+    x, w, kc0, vc0 = _inputs(B, D, h_q, h_k, h_v, d, l_cap, seed=123 + B)
+    shape = saga.SagaShape(B, h_q, h_k, h_v, d, l_cap)
+    xg, wg, kcg, vcg = x.cuda(), w.cuda(), kc0.cuda(), vc0.cuda()
+    q = torch.zeros((B, h_q, d), dtype=torch.bfloat16, device="cuda")
+    sl = torch.tensor([5], dtype=torch.int32, device="cuda")
+    ws = saga.alloc_qkv_workspace(shape, D)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        saga.saga_qkv_project(shape, xg, wg, q, kcg, vcg, 4, workspace=ws, seq_len_dev=sl, stream=stream)
+    stream.synchronize()
+    kcg.copy_(kc0.cuda())
+    vcg.copy_(vc0.cuda())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        saga.saga_qkv_project(shape, xg, wg, q, kcg, vcg, 4, workspace=ws, seq_len_dev=sl, stream=stream)
+    xf, wf = x.double().numpy(), w.double().numpy()
+    qe, ke, ve = qkv_oracle.project(xf, wf, h_q, h_k, h_v, d)
+    bound_k = _bound(xf, wf[h_q * d:(h_q + h_k) * d], ke.reshape(B, -1), B, D)
+    for length in (9, 14):
+        sl.fill_(length)
+        graph.replay()
+        torch.cuda.synchronize()
+        row = kcg[:, :, length - 1].cpu().double().numpy().reshape(B, -1)
+        assert np.all(np.abs(row - ke.reshape(B, -1)) <= bound_k), length
+    untouched = [r for r in range(l_cap) if r not in (8, 13)]
+    assert torch.equal(kcg.cpu()[:, :, untouched], kc0[:, :, untouched])
+    assert torch.equal(vcg.cpu()[:, :, untouched], vc0[:, :, untouched])
+    assert saga.saga_get_status(ws) == 0
+    del graph
