@@ -135,6 +135,13 @@ SAGA_API int saga_kv_append(const saga_shape* s, void* k_cache, void* v_cache, c
  * leaves it ready for the next); word 0 is a sticky status word read by
  * saga_get_status (SAGA_STATUS_TIMEOUT if a bounded wait gave up); calls on
  * one workspace must not overlap in time.  The caller owns every buffer.
+ * The kernels start loading w_qkv before their programmatic dependency wait
+ * (the weight stream overlaps the end of the preceding kernel): w_qkv must
+ * not be written by work that can still be running when this call's kernels
+ * start, i.e. by a kernel launched earlier on the stream that releases its
+ * dependents early (programmatic launch completion).  Weights written by a
+ * copy, by an ordinary kernel or on another synchronized stream are fine; x,
+ * the caches and the device length are read after the wait.
  * Errors: SAGA_ERR_ARG / SAGA_ERR_UNSUPPORTED / SAGA_ERR_WORKSPACE before
  * anything is enqueued; SAGA_ERR_CUDA if the launch fails. */
 SAGA_API int saga_qkv_project(const saga_shape* s, int hidden, const void* x, const void* w_qkv, void* q_out,
