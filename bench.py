@@ -314,9 +314,10 @@ def run_reference(args, wl, rank, world):
     return 0
 
 
-def make_session(wl, dev, rank, total_steps):
+def make_session(wl, dev, rank, total_steps, layer_batched=False):
     """A DecodeSession holding every layer of `wl` (caches prefilled with the seeded synthetic rows, one
-    rank's seed per rank) and the per-step inputs of `total_steps` decode steps, stacked [steps, layers, ...]."""
+    rank's seed per rank) and the per-step inputs of `total_steps` decode steps, stacked [steps, layers, ...].
+    layer_batched: all layers of a step in one call (batch = layers x B)."""
     import torch
 
     from long_context_decoding_saga_b200 import saga, workload
@@ -325,7 +326,7 @@ def make_session(wl, dev, rank, total_steps):
     l_cap = wl.l_kv + total_steps
     n_top = wl.n_for_kernel(l_cap)
     shape = saga.SagaShape.of(wl.batch, wl.h_q, wl.h_k, wl.h_v, wl.d, l_cap)
-    sess = DecodeSession(shape, wl.layers, n_top, wl.refresh, device=dev)
+    sess = DecodeSession(shape, wl.layers, n_top, wl.refresh, device=dev, layer_batched=layer_batched)
     qs, ks, vs = [], [], []
     for i in range(wl.layers):
         inp = workload.make_layer(wl.with_(seed=wl.seed + 7919 * rank), i, device=dev, steps=total_steps)
@@ -422,6 +423,15 @@ EXTRA_WORKLOADS = (
     ("sweep_l131072_b16_hk8_n256_r16", 4),
 )
 
+# The same step with every layer in one call (the layers as a batch of layers x B: one kernel hand-off
+# chain per step instead of one per layer; needs all layers' queries of the step at once).
+LAYER_BATCHED_WORKLOADS = (
+    "qwen2.5-1.5b_saga_128k",
+    "llama3.2-1b_saga_32k",
+    "llama3.2-1b_dense_gqa_128k",
+    "sweep_l4096_b1_hk2_n256_r16",
+)
+
 
 def time_key_head_merge(dev, tokens=4096, hidden=2048, d=64, h_q=32, h_k=8, repeats=3):
     """The closed-form key-head merge on a Llama-3.2-1B-shaped teacher (8 key heads merged into 4), synthetic
@@ -509,14 +519,14 @@ def time_qkv_projection(dev, peak_gbs, layers=24, replays=5):
     return out
 
 
-def time_extra_workload(wl, dev, rank, args, peak, l2_bytes):
+def time_extra_workload(wl, dev, rank, args, peak, l2_bytes, layer_batched=False):
     """One entry of the `workloads` object: graph-replayed decode steps of `wl` (K = max(16, R) when R is
     at most 64, so the window holds refresh and reuse steps in their proportion), inputs resident."""
     import torch
     W = 3
     K = wl.refresh if wl.refresh <= 64 and wl.refresh > 16 else 16
     plan = step_plan(W, K, wl.refresh, e2e=False)
-    sess, inputs, _, _, _ = make_session(wl, dev, rank, plan["total"])
+    sess, inputs, _, _, _ = make_session(wl, dev, rank, plan["total"], layer_batched=layer_batched)
     q_all, k_all, v_all = inputs
     sess.step(q_all[0], k_all[0], v_all[0])
     sess.capture(torch.cuda.Stream(dev))
@@ -538,7 +548,8 @@ def time_extra_workload(wl, dev, rank, args, peak, l2_bytes):
              "n_top": wl.n_top if not wl.dense else "dense", "refresh": wl.refresh, "steps": K,
              "refresh_steps": int(sum(kinds)), "us_per_step": ms / K * 1e3, "gb_s": gbs, "frac": gbs / peak,
              "step_us": step_means(step_ms, kinds, wl.refresh), "l2": l2_note(flush, step_bytes, l2_bytes),
-             "clocks": clocks, "status_word": None}
+             "clocks": clocks, "status_word": None, "layers_in_one_call": layer_batched,
+             "launches_per_step": {"reuse": sess.launches_per_step(False), "refresh": sess.launches_per_step(True)}}
     from long_context_decoding_saga_b200 import saga
     entry["status_word"] = saga.saga_get_status(sess.workspace)
     del sess, inputs, q_all, k_all, v_all, scratch
@@ -751,6 +762,14 @@ def run_saga(args, wl, rank, world, local_rank):
             except Exception as exc:  # noqa: BLE001  (reported, never fatal to the benchmark line)
                 extras[name] = {"error": str(exc)[:300]}
         line["workloads"] = extras
+        batched = {}
+        for name in LAYER_BATCHED_WORKLOADS:
+            try:
+                batched[name] = time_extra_workload(workload.by_name(name), dev, 0, args, peak, l2_bytes,
+                                                    layer_batched=True)
+            except Exception as exc:  # noqa: BLE001  (reported, never fatal to the benchmark line)
+                batched[name] = {"error": str(exc)[:300]}
+        line["layers_in_one_call"] = batched
         try:
             line["qkv_projection"] = time_qkv_projection(dev, peak)
         except Exception as exc:  # noqa: BLE001  (reported, never fatal to the benchmark line)

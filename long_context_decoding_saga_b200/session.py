@@ -12,6 +12,15 @@ refresh step and a reuse step).  The graphs read the sequence length from a
 device int (the length argument the C ABI takes for graph replays) that a
 one-element add at the start of each replay advances; inputs are staged into
 static buffers before each replay.
+
+With `layer_batched=True` the layers' caches, thresholds, inputs and outputs
+are slices of layer-major buffers, and a step is ONE saga_decode_step call
+with batch = layers x B: every (layer, batch) row is an independent row of
+the batched call, so the results are those of the per-layer calls, and the
+step pays one kernel hand-off chain instead of one per layer.  This needs
+every layer's query of the step at once, as this session's step() takes
+them; a model whose next layer's query depends on this layer's output calls
+the layers one by one.
 """
 from __future__ import annotations
 
@@ -24,19 +33,27 @@ from . import saga
 
 class DecodeSession:
     def __init__(self, shape: saga.SagaShape, layers: int, n_top: int, refresh: int, device="cuda",
-                 out_dtype=torch.float32, track_selection: bool = False):
+                 out_dtype=torch.float32, track_selection: bool = False, layer_batched: bool = False):
         self.shape = shape
         self.layers = layers
         self.n_top = n_top
         self.refresh = refresh
         self.device = torch.device(device)
+        self.layer_batched = layer_batched
         B, hq, hk, hv, d, lc = shape.astuple()
         bf = torch.bfloat16
-        self.k_cache = [torch.zeros((B, hk, lc, d), dtype=bf, device=device) for _ in range(layers)]
-        self.v_cache = [torch.zeros((B, hv, lc, d), dtype=bf, device=device) for _ in range(layers)]
+        if layer_batched:
+            self.batched_shape = saga.SagaShape.of(layers * B, hq, hk, hv, d, lc)
+            self.k_all = torch.zeros((layers, B, hk, lc, d), dtype=bf, device=device)
+            self.v_all = torch.zeros((layers, B, hv, lc, d), dtype=bf, device=device)
+            self.k_cache = [self.k_all[i] for i in range(layers)]
+            self.v_cache = [self.v_all[i] for i in range(layers)]
+        else:
+            self.k_cache = [torch.zeros((B, hk, lc, d), dtype=bf, device=device) for _ in range(layers)]
+            self.v_cache = [torch.zeros((B, hv, lc, d), dtype=bf, device=device) for _ in range(layers)]
         self.tau = torch.zeros((layers, B, hq), dtype=torch.float32, device=device)
         self.out = torch.zeros((layers, B, hq, d), dtype=out_dtype, device=device)
-        self.workspace = saga.alloc_workspace(shape, device)
+        self.workspace = saga.alloc_workspace(self.batched_shape if layer_batched else shape, device)
         self.sel_count = self.sel_idx = None
         if track_selection:
             self.sel_count = torch.zeros((layers, B, hq), dtype=torch.int32, device=device)
@@ -63,13 +80,28 @@ class DecodeSession:
                               sel_count=None if self.sel_count is None else self.sel_count[i],
                               sel_idx=None if self.sel_idx is None else self.sel_idx[i], seq_len_dev=seq_len_dev)
 
+    def _all_layers_step(self, q, k_new, v_new, seq_len, step, seq_len_dev=None):
+        """Every layer in one call: the layer-major buffers viewed as a batch of layers x B."""
+        B, hq, hk, hv, d, lc = self.shape.astuple()
+        LB = self.layers * B
+        saga.saga_decode_step(self.batched_shape, q.reshape(LB, hq, d), k_new.reshape(LB, hk, d),
+                              v_new.reshape(LB, hv, d), self.k_all.view(LB, hk, lc, d),
+                              self.v_all.view(LB, hv, lc, d), seq_len, self.n_top, self.refresh, step,
+                              self.tau.view(LB, hq), self.out.view(LB, hq, d), self.workspace,
+                              sel_count=None if self.sel_count is None else self.sel_count.view(LB, hq),
+                              sel_idx=None if self.sel_idx is None else self.sel_idx.view(LB, hq, lc),
+                              seq_len_dev=seq_len_dev)
+
     def step(self, q, k_new, v_new):
         """One decode step of every layer with host-side lengths (q: [layers, B, h_q, d], ...)."""
         if self.length >= self.shape.l_cap:
             raise RuntimeError("cache capacity exhausted")
         L = self.length + 1
-        for i in range(self.layers):
-            self._layer_step(i, q[i], k_new[i], v_new[i], L, self.t)
+        if self.layer_batched:
+            self._all_layers_step(q.contiguous(), k_new.contiguous(), v_new.contiguous(), L, self.t)
+        else:
+            for i in range(self.layers):
+                self._layer_step(i, q[i], k_new[i], v_new[i], L, self.t)
         self.length = L
         self.t += 1
         return self.out
@@ -85,9 +117,13 @@ class DecodeSession:
             torch.cuda.synchronize(self.device)
             with torch.cuda.graph(g, stream=stream):
                 self.seq_len_dev.add_(1)
-                for i in range(self.layers):
-                    self._layer_step(i, self.q_buf[i], self.k_buf[i], self.v_buf[i], L_est, step,
-                                     seq_len_dev=self.seq_len_dev)
+                if self.layer_batched:
+                    self._all_layers_step(self.q_buf, self.k_buf, self.v_buf, L_est, step,
+                                          seq_len_dev=self.seq_len_dev)
+                else:
+                    for i in range(self.layers):
+                        self._layer_step(i, self.q_buf[i], self.k_buf[i], self.v_buf[i], L_est, step,
+                                         seq_len_dev=self.seq_len_dev)
             self.graphs[kind] = g
         self.seq_len_dev.fill_(self.length)
         torch.cuda.synchronize(self.device)
@@ -116,4 +152,4 @@ class DecodeSession:
             per_layer = 3  # threshold fill, split (+append), combine
         else:
             per_layer = 2  # split (+append), combine
-        return self.layers * per_layer
+        return per_layer if self.layer_batched else self.layers * per_layer

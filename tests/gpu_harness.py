@@ -239,14 +239,15 @@ def layer_inputs_on_gpu(wl, steps):
     return layers
 
 
-def run_full_all(wl, inputs, steps, track=False, record_idx=False):
+def run_full_all(wl, inputs, steps, track=False, record_idx=False, layer_batched=False):
     """All layers of `wl` per step through CUDA-graph replays with a device-side length (the benchmark's
     launch configuration) for `steps` steps.  Returns, per layer, per step: out, tau and (track) the kept
-    counts and (record_idx) each row's kept positions."""
+    counts and (record_idx) each row's kept positions.  layer_batched: every layer of a step in one call."""
     l_cap = wl.l_kv + steps
     n_top = wl.n_for_kernel(l_cap)
     shape = saga.SagaShape.of(wl.batch, wl.h_q, wl.h_k, wl.h_v, wl.d, l_cap)
-    sess = DecodeSession(shape, wl.layers, n_top, wl.refresh, device="cuda", track_selection=track)
+    sess = DecodeSession(shape, wl.layers, n_top, wl.refresh, device="cuda", track_selection=track,
+                         layer_batched=layer_batched)
     for i, inp in enumerate(inputs):
         sess.prefill(i, inp["K0"], inp["V0"])
     q_all = torch.stack([inp["q"] for inp in inputs], 1)

@@ -10,6 +10,9 @@ one layer per worker process.  A first run without index tracking (the timed
 configuration) gives the outputs; a second run with tracking must give the
 same bits, and its index lists are checked.
 
+Llama-SAGA 32K and Qwen-SAGA 128K also run with every layer of a step in one call (batch = layers x B)
+and are checked the same way.
+
 The sweep (Llama-3.2-1B shapes) covers every (h_k, N, R) triple at 128K
 context with batch 1, and mixed points at every context length and batch,
 each on two of its 16 layers (the layers are drawn independently, so any two
@@ -59,6 +62,21 @@ def test_every_layer_and_step_matches_oracle(wl):
     if not wl.dense:
         assert sum(s["index_sets_checked"] for s in summaries) == wl.layers * steps * wl.batch * wl.h_q
         assert all(s["refresh_steps"] == (steps + wl.refresh - 1) // wl.refresh for s in summaries)
+
+
+@pytest.mark.parametrize("wl", [workload.LLAMA_SAGA_32K, workload.QWEN_SAGA_128K], ids=lambda w: w.name)
+def test_layers_in_one_call_match_oracle(wl):
+    """The same steps with every layer of a step in one call (batch = layers x B): every layer of every step
+    against the stepping oracle, index sets included."""
+    steps = wl.steps
+    inputs = gpu_harness.layer_inputs_on_gpu(wl, steps)
+    tracked, n_top, l_cap = gpu_harness.run_full_all(wl, inputs, steps, track=True, record_idx=True,
+                                                    layer_batched=True)
+    del inputs
+    torch.cuda.empty_cache()
+    summaries = gpu_harness.check_full_all(wl, tracked, n_top, l_cap, steps)
+    assert len(summaries) == wl.layers
+    assert sum(s["index_sets_checked"] for s in summaries) == wl.layers * steps * wl.batch * wl.h_q
 
 
 # Every (h_k, N, R) triple at 128K with batch 1, plus points that bring in every context length and batch.
