@@ -345,6 +345,17 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   p.v_new = nr.v_new;
   p.scores_out = reinterpret_cast<float*>(pr.base + pr.ws.scores);
   p.hist_out = hist;
+  // One CTA per row (one kernel, the row scanned by its CTA) when the rows
+  // fill the GPU or are short; else each row in chunks over many CTAs (three
+  // kernels).  Measured on refresh steps: rows of 32K scores (32 rows) 688 vs
+  // 746 us per step and 512 rows of 128K 10.95 vs 11.94 ms with one kernel;
+  // 32 rows of 128K 1145 vs 1281 us and 12 rows of 128K 1690 vs 1704 us with
+  // the chunked kernels.  The one-kernel select recounts a row whose dumped
+  // histogram misses the N-th largest, so the dump may count only the bins
+  // near the stale threshold (the chunked kernels need every bin).
+  const bool one_cta_per_row = rows >= (size_t)pr.sms || seq_len <= 32768;
+  p.hist_floor = one_cta_per_row ? 1 : 0;
+  p.tau = tau;  // the stale threshold, read by the dump before the select overwrites it
   p.nsplit = S;
   e = launch_split(s->d, NP, kSplitDump, tf, tp, p, dim3(S * hsplit, s->h_k, s->batch), st, nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "score dump launch");
@@ -362,13 +373,6 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   sp.cand_cnt = reinterpret_cast<int*>(hist + rows * 512);
   sp.cand = reinterpret_cast<uint32_t*>(pr.base + pr.ws.cand);
   sp.cand_cap = kCandCap;
-  // One CTA per row (one kernel, the row scanned by its CTA) when the rows
-  // fill the GPU or are short; else each row in chunks over many CTAs (three
-  // kernels).  Measured on refresh steps: rows of 32K scores (32 rows) 688 vs
-  // 746 us per step and 512 rows of 128K 10.95 vs 11.94 ms with one kernel;
-  // 32 rows of 128K 1145 vs 1281 us and 12 rows of 128K 1690 vs 1704 us with
-  // the chunked kernels.
-  const bool one_cta_per_row = rows >= (size_t)pr.sms || seq_len <= 32768;
   e = one_cta_per_row ? launch_select(sp, (int)rows, st) : launch_select_parallel(sp, (int)rows, st);
   if (e != cudaSuccess) return cuda_fail(e, "radix select launch");
   return SAGA_OK;

@@ -76,6 +76,7 @@ struct SplitParams {
   const float* scores_in;   // from-scores mode: [B*h_q, ld_scores]
   float* scores_out;        // dump mode
   uint32_t* hist_out;       // dump mode: [B*h_q, 256]
+  int hist_floor;           // dump mode: count only top-byte bins from two below the stale tau's bin up
   float* part_o;
   float* part_m;
   float* part_l;

@@ -894,9 +894,10 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
         qv[k] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.h_q + j0 + n) * D + col));
     }
     tv = load_tau<NP>(eth, p, b, j0, !DUMP);
+    if (DUMP && p.hist_floor != 0 && p.tau != nullptr && eth < p.G) tv = __ldg(p.tau + (size_t)b * p.h_q + j0 + eth);
   }
   // the epilogue compares raw dot products (scaled only once listed)
-  if (warp >= 2 && eth < NP) tv = raw_threshold(tv, p.scale);
+  if (!DUMP && warp >= 2 && eth < NP) tv = raw_threshold(tv, p.scale);
   const int L = device_seq_len(p.seq_len_dev, p.seq_len, p.l_cap, (s == 0 && h == 0 && b == 0) ? p.status : nullptr);
   int start, end;
   split_range(p.seq_len, p.nsplit, s, L, &start, &end);
@@ -989,6 +990,21 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     acc.init();
     ListState ls{0, 0, -1, 0};
     const size_t srow = ((size_t)b * p.h_q + j0) * (size_t)p.ld_scores;
+    // dump mode: the histogram only needs exact counts from the bin holding the N-th largest up, so with
+    // hist_floor it counts the top-byte bins from two below the stale threshold's bin (four times smaller
+    // magnitudes) up; the select checks that the counted bins hold N scores and otherwise recounts the row
+    uint32_t bfl[NP];
+#pragma unroll
+    for (int jl = 0; jl < NP; ++jl) {
+      bfl[jl] = 0u;
+      if (DUMP && p.hist_floor != 0 && jl < p.G) {
+        const float ts = es.tau[jl];  // the stale threshold (scaled, as the dumped scores)
+        if (ts != -INFINITY && ts == ts) {
+          const uint32_t tb = float_key(ts) >> 24;
+          bfl[jl] = tb > 2u ? tb - 2u : 0u;
+        }
+      }
+    }
     int t = 0;
     if (!DUMP && p.test_wait_ns != 0u) {
       bool ok = __all_sync(0xffffffffu, mbar_wait(never, 0, abort_flag, p.test_wait_ns));
@@ -1029,9 +1045,12 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
         for (int jl = 0; jl < NP; ++jl) {
           if (jl < p.G) {
             if (valid) p.scores_out[srow + (size_t)jl * p.ld_scores + tok] = sc[jl];
-            const uint32_t bin = valid ? (float_key(sc[jl]) >> 24) : 256u;
-            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-            if (valid && lane == __ffs(peers) - 1) atomicAdd(&hist[jl * 256 + bin], (uint32_t)__popc(peers));
+            const uint32_t bin = float_key(sc[jl]) >> 24;
+            const bool counted = valid && bin >= bfl[jl];
+            if (__any_sync(0xffffffffu, counted)) {
+              const uint32_t peers = __match_any_sync(0xffffffffu, counted ? bin : 256u);
+              if (counted && lane == __ffs(peers) - 1) atomicAdd(&hist[jl * 256 + bin], (uint32_t)__popc(peers));
+            }
           }
         }
       } else {
@@ -1755,16 +1774,26 @@ __global__ void __launch_bounds__(kSelectThreads) atopn_select_kernel(const Sele
   }
   const float* row = p.scores + (size_t)r * p.ld;
 
-  for (int i = threadIdx.x; i < 256; i += kSelectThreads)
-    hist[i] = p.hist != nullptr ? p.hist[(size_t)r * 256 + i] : 0u;
+  // a given top-digit histogram may count only the bins from some floor up
+  // (the score dump counts from just below the stale threshold): it serves
+  // when its bins hold at least N scores, else the row is counted here
+  __shared__ uint32_t counted;
   if (threadIdx.x == 0) {
     ncand = 0;
     s_bin = 0;
     s_rank = 1;
     s_cnt = 0;
+    counted = 0u;
   }
   __syncthreads();
-  if (p.hist == nullptr) {  // top digit histogram
+  for (int i = threadIdx.x; i < 256; i += kSelectThreads) {
+    hist[i] = p.hist != nullptr ? p.hist[(size_t)r * 256 + i] : 0u;
+    if (hist[i] != 0u) atomicAdd(&counted, hist[i]);
+  }
+  __syncthreads();
+  if (p.hist == nullptr || counted < (uint32_t)p.n_top) {  // top digit histogram of the whole row
+    for (int i = threadIdx.x; i < 256; i += kSelectThreads) hist[i] = 0u;
+    __syncthreads();
     scan_row(row, L, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
     __syncthreads();
   }

@@ -151,6 +151,30 @@ def test_refresh_threshold_entry_point():
     assert np.max(np.abs(tau.cpu().numpy() - expect)) <= gpu_harness.BAND
 
 
+@pytest.mark.parametrize("stale", ["huge", "tiny", "nan", "mixed"])
+def test_refresh_with_any_stale_threshold_is_exact(stale):
+    """The score dump counts only the top-byte bins from just below the stale threshold up, and the select
+    recounts a row whose counted bins hold fewer than N scores: whatever the stale values in tau (above every
+    score, below every score, NaN, or mixed per row), the refreshed threshold is the same bits as with a
+    stale threshold of 0, and the oracle's."""
+    wl = small("refresh_stale", h_q=12, h_k=1, h_v=4, d=128, l_kv=5000, n_top=77)
+    inp = workload.make_layer(wl, 0, steps=1)
+    shape = saga.SagaShape.of(1, 12, 1, 4, 128, 5000)
+    kc = inp["K0"].cuda().contiguous()
+    q = inp["q"][0].cuda().contiguous()
+    ws = saga.alloc_workspace(shape)
+    base = torch.zeros((1, 12), device="cuda")
+    saga.atopn_refresh_threshold(shape, q, kc, 5000, 77, base, ws)
+    tau = {"huge": torch.full((1, 12), 1e30, device="cuda"), "tiny": torch.full((1, 12), -1e30, device="cuda"),
+           "nan": torch.full((1, 12), float("nan"), device="cuda"),
+           "mixed": torch.tensor([[1e30, 0.0, -1e30, 5.0, float("nan"), 1e-30] * 2], device="cuda")}[stale]
+    saga.atopn_refresh_threshold(shape, q, kc, 5000, 77, tau, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(tau, base)
+    expect = saga_oracle.refresh_threshold(inp["q"][0].float().numpy(), inp["K0"].float().numpy(), 5000, 77)
+    assert np.max(np.abs(tau.cpu().numpy() - expect)) <= gpu_harness.BAND
+
+
 def test_empty_selection_gives_zero():
     """A stale threshold above every score of a later step keeps nothing: output 0, count 0."""
     shape = saga.SagaShape.of(1, 8, 1, 8, 64, 600)
