@@ -21,7 +21,7 @@ cudaError_t launch_dense(int D, int NP, const CUtensorMap& kf, const CUtensorMap
                          const CUtensorMap& vp, const SplitParams& p, dim3 grid, cudaStream_t st, int* occ);
 cudaError_t launch_combine(int D, const CombineParams& p, cudaStream_t st);
 cudaError_t launch_select(const SelectParams& p, int rows, cudaStream_t st);
-cudaError_t launch_select_parallel(const SelectParams& p, int rows, cudaStream_t st);
+cudaError_t launch_select_cluster(const SelectParams& p, int rows, cudaStream_t st);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t st);
 cudaError_t launch_qkv(const QkvParams& p, const CUtensorMap& tw, cudaStream_t st);
 cudaError_t launch_fill(float* dst, float v, int n, cudaStream_t st);
@@ -147,9 +147,7 @@ WsLayout ws_layout(const saga_shape* s, int sms) {
   w.scores = off;
   off = align256(off + (size_t)rows * w.ld_scores * 4);
   w.hist = off;
-  off = align256(off + (size_t)rows * (2 * 256 + 1) * 4);
-  w.cand = off;
-  off = align256(off + (size_t)rows * kCandCap * 4);
+  off = align256(off + (size_t)rows * 256 * 4);
   w.idx = off;
   off = align256(off + (size_t)rows * s->l_cap * 4);
   w.total = off;
@@ -335,7 +333,7 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
     cudaError_t et = trace_record(ev_start, st);
     if (et != cudaSuccess) return cuda_fail(et, "trace event record");
   }
-  cudaError_t e = cudaMemsetAsync(hist, 0, rows * (2 * 256 + 1) * 4, st);
+  cudaError_t e = cudaMemsetAsync(hist, 0, rows * 256 * 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(hist)");
   SplitParams p;
   fill_split_common(p, s, pr, q, k_cache, seq_len, seq_len_dev, true);
@@ -345,16 +343,16 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   p.v_new = nr.v_new;
   p.scores_out = reinterpret_cast<float*>(pr.base + pr.ws.scores);
   p.hist_out = hist;
-  // One CTA per row (one kernel, the row scanned by its CTA) when the rows
-  // fill the GPU or are short; else each row in chunks over many CTAs (three
-  // kernels).  Measured on refresh steps: rows of 32K scores (32 rows) 688 vs
-  // 746 us per step and 512 rows of 128K 10.95 vs 11.94 ms with one kernel;
-  // 32 rows of 128K 1145 vs 1281 us and 12 rows of 128K 1690 vs 1704 us with
-  // the chunked kernels.  The one-kernel select recounts a row whose dumped
-  // histogram misses the N-th largest, so the dump may count only the bins
-  // near the stale threshold (the chunked kernels need every bin).
+  // One CTA per row scanning the whole row when the rows fill the GPU or are
+  // short; else one thread-block cluster of CTAs per row, each CTA a chunk.
+  // Measured on refresh steps: rows of 32K scores (32 rows) 688 vs 746 us and
+  // 512 rows of 128K 10.95 vs 11.94 ms per step with one CTA per row than with
+  // rows in chunks over three kernels; for 12 and 32 rows of 128K the cluster
+  // kernel against those three kernels: 1546 vs 1730 us and 1048 vs 1158 us.
+  // Both recount a row whose dumped histogram misses the N-th largest, so the
+  // dump counts only the bins near the stale threshold.
   const bool one_cta_per_row = rows >= (size_t)pr.sms || seq_len <= 32768;
-  p.hist_floor = one_cta_per_row ? 1 : 0;
+  p.hist_floor = 1;
   p.tau = tau;  // the stale threshold, read by the dump before the select overwrites it
   p.nsplit = S;
   e = launch_split(s->d, NP, kSplitDump, tf, tp, p, dim3(S * hsplit, s->h_k, s->batch), st, nullptr);
@@ -369,11 +367,7 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   sp.row_len = seq_len;
   sp.l_cap = s->l_cap;
   sp.n_top = n_top;
-  sp.hist2 = hist + rows * 256;
-  sp.cand_cnt = reinterpret_cast<int*>(hist + rows * 512);
-  sp.cand = reinterpret_cast<uint32_t*>(pr.base + pr.ws.cand);
-  sp.cand_cap = kCandCap;
-  e = one_cta_per_row ? launch_select(sp, (int)rows, st) : launch_select_parallel(sp, (int)rows, st);
+  e = one_cta_per_row ? launch_select(sp, (int)rows, st) : launch_select_cluster(sp, (int)rows, st);
   if (e != cudaSuccess) return cuda_fail(e, "radix select launch");
   return SAGA_OK;
 }

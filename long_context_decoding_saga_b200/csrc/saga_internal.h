@@ -20,7 +20,6 @@ constexpr int kMaxNvh = 32;      // value heads per key-head group
 constexpr int kMaxCtasPerSm = 4; // bound used to size the split partials
 constexpr int kSelectThreads = 1024;
 constexpr int kSelectCap = 16384; // radix-select candidates kept in shared memory
-constexpr int kCandCap = 16384;   // parallel refresh select: candidates per row (global)
 
 // Token range [start, end) of split s out of S.  The boundaries partition P
 // tokens (the host's length at launch, fixed for a captured graph) at
@@ -56,8 +55,7 @@ struct WsLayout {
   size_t part_l;    // float [B*h_q, S_cap]
   size_t part_cnt;  // int   [B*h_q, S_cap]
   size_t scores;    // float [B*h_q, ld_scores]
-  size_t hist;      // uint32 [B*h_q, 256] top byte, [B*h_q, 256] second byte, int [B*h_q] candidate counts
-  size_t cand;      // uint32 [B*h_q, kCandCap] refresh-select candidates
+  size_t hist;      // uint32 [B*h_q, 256] top-byte histograms of the dumped scores
   size_t idx;       // int   [B*h_q, l_cap]
   size_t total;
   int s_cap;
@@ -123,13 +121,7 @@ struct CombineParams {
 struct SelectParams {
   const float* scores;
   long long ld;
-  const uint32_t* hist;  // nullable: precomputed top-byte histogram [rows, 256]
-  // parallel refresh select (with hist): second-byte histogram of the
-  // threshold's top-byte bin, candidates matching the top 16 bits, counts
-  uint32_t* hist2;       // [rows, 256], zero before the first kernel
-  int* cand_cnt;         // [rows], zero before the first kernel
-  uint32_t* cand;        // [rows, cand_cap]
-  int cand_cap;
+  const uint32_t* hist;  // nullable: precomputed top-byte histogram [rows, 256] (may count only upper bins)
   float* tau;
   unsigned* status;
   const int* seq_len_dev;  // nullable: row length from the device

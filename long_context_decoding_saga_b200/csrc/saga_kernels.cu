@@ -1837,19 +1837,9 @@ __global__ void __launch_bounds__(kSelectThreads) atopn_select_kernel(const Sele
   if (threadIdx.x == 0) p.tau[r] = key_float(prefix);
 }
 
-// ---------------------------------------------------------------------------- parallel refresh select
-// With the top-byte histogram of every row already counted by the score dump,
-// the rest of the exact N-th largest runs on many CTAs per row:
-//   1. (rows x P CTAs) each CTA finds the threshold's top-byte bin from the
-//      histogram and counts the second byte of the scores in that bin over
-//      its chunk of the row (global histogram);
-//   2. (rows x P CTAs) with both bytes known, the scores matching the top
-//      16 bits are collected into a per-row candidate buffer (their number is
-//      known from the second histogram; above the buffer size nothing is
-//      collected);
-//   3. (one CTA per row) the last two bytes are resolved in shared memory
-//      from the candidates, or, when they did not fit, by the single-CTA
-//      digit scans over the row.
+// ---------------------------------------------------------------------------- cluster select
+// Few long rows: the row in chunks over the CTAs of one thread-block cluster
+// (atopn_cluster_select_kernel below).
 
 // Calls f(key, valid) for the elements [begin, end) of row (begin a multiple
 // of 4, row 16-byte aligned) with warp-uniform trip counts.
@@ -1886,157 +1876,122 @@ __device__ __forceinline__ void scan_range(const float* row, int begin, int end,
   }
 }
 
-constexpr int kSelPartThreads = 256;
-
 __device__ __forceinline__ void sel_chunk(int L, int part, int P, int* b, int* e) {
   const int chunk = (((L + P - 1) / P) + 3) & ~3;
   *b = min(L, part * chunk);
   *e = min(L, *b + chunk);
 }
 
-__global__ void __launch_bounds__(kSelPartThreads) atopn_hist2_kernel(const SelectParams p) {
-  __shared__ uint32_t h[256];
-  __shared__ uint32_t s_bin, s_rank, s_cnt;
-  const int r = blockIdx.x;
-  pdl_trigger();
-  pdl_wait();
-  int L = p.row_len;
-  if (p.seq_len_dev != nullptr) L = device_seq_len(p.seq_len_dev, p.row_len, p.l_cap, nullptr);
-  if (p.n_top >= L) return;
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) h[i] = 0u;
-  if (threadIdx.x == 0) {
-    s_bin = 0;
-    s_rank = 1;
-    s_cnt = 0;
-  }
-  __syncthreads();
-  find_bin(p.hist + (size_t)r * 256, (uint32_t)p.n_top, &s_bin, &s_rank, &s_cnt);
-  __syncthreads();
-  const uint32_t b1 = s_bin;
-  int beg, end;
-  sel_chunk(L, blockIdx.y, gridDim.y, &beg, &end);
-  scan_range(p.scores + (size_t)r * p.ld, beg, end, [&](uint32_t k, bool ok) {
-    const bool m = ok && (k >> 24) == b1;
-    hist_add(h, m ? (k >> 16) & 255u : 0u, m);
-  });
-  __syncthreads();
-  for (int i = threadIdx.x; i < 256; i += blockDim.x)
-    if (h[i] != 0u) atomicAdd(&p.hist2[(size_t)r * 256 + i], h[i]);
-}
+// Exact N-th largest of a few long rows: one thread-block cluster per row,
+// each CTA scanning a contiguous chunk.  Per 8-bit digit (MSB first) every
+// CTA histograms the keys of its chunk that match the digits found so far;
+// after a cluster barrier each CTA adds the cluster's histograms over
+// distributed shared memory (so every CTA holds the same sums and takes the
+// same decision) and finds the digit's bin.  Once the keys matching the
+// prefix fit, each CTA keeps its own in shared memory and the remaining
+// digits are resolved over those.  A given top-digit histogram (from the
+// score dump) is used when its bins hold N scores.  Cluster barriers are
+// hardware barriers every CTA reaches on every path.
+constexpr int kSelCluster = 8;          // CTAs per row
+constexpr int kSelClusterThreads = 512;
 
-// Bins of the first two bytes: (b1, rank within it), then (b2, rank, count).
-__device__ __forceinline__ void two_bins(const SelectParams& p, int r, uint32_t* s_bin, uint32_t* s_rank,
-                                         uint32_t* s_cnt, uint32_t* b1, uint32_t* b2, uint32_t* rank2,
-                                         uint32_t* cnt2) {
-  if (threadIdx.x == 0) {
-    *s_bin = 0;
-    *s_rank = 1;
-    *s_cnt = 0;
-  }
-  __syncthreads();
-  find_bin(p.hist + (size_t)r * 256, (uint32_t)p.n_top, s_bin, s_rank, s_cnt);
-  __syncthreads();
-  *b1 = *s_bin;
-  const uint32_t rank1 = *s_rank;
-  __syncthreads();
-  find_bin(p.hist2 + (size_t)r * 256, rank1, s_bin, s_rank, s_cnt);
-  __syncthreads();
-  *b2 = *s_bin;
-  *rank2 = *s_rank;
-  *cnt2 = *s_cnt;
-}
-
-__global__ void __launch_bounds__(kSelPartThreads) atopn_collect_kernel(const SelectParams p) {
-  __shared__ uint32_t s_bin, s_rank, s_cnt;
-  const int r = blockIdx.x;
-  pdl_trigger();
-  pdl_wait();
-  int L = p.row_len;
-  if (p.seq_len_dev != nullptr) L = device_seq_len(p.seq_len_dev, p.row_len, p.l_cap, nullptr);
-  if (p.n_top >= L) return;
-  uint32_t b1, b2, rank2, cnt2;
-  two_bins(p, r, &s_bin, &s_rank, &s_cnt, &b1, &b2, &rank2, &cnt2);
-  if (cnt2 > (uint32_t)p.cand_cap) return;  // resolved by the digit scans instead
-  const uint32_t prefix = (b1 << 8) | b2;
-  int beg, end;
-  sel_chunk(L, blockIdx.y, gridDim.y, &beg, &end);
-  uint32_t* cand = p.cand + (size_t)r * p.cand_cap;
-  const int lane = threadIdx.x & 31;
-  scan_range(p.scores + (size_t)r * p.ld, beg, end, [&](uint32_t k, bool ok) {
-    const bool m = ok && (k >> 16) == prefix;
-    const uint32_t bal = __ballot_sync(0xffffffffu, m);
-    if (bal != 0u) {  // warp-uniform: one atomic per warp
-      int base = 0;
-      if (lane == __ffs(bal) - 1) base = atomicAdd(&p.cand_cnt[r], __popc(bal));
-      base = __shfl_sync(0xffffffffu, base, __ffs(bal) - 1);
-      const int pos = base + __popc(bal & ((1u << lane) - 1u));
-      if (m && pos < p.cand_cap) cand[pos] = k;
-    }
-  });
-}
-
-__global__ void __launch_bounds__(kSelectThreads) atopn_resolve_kernel(const SelectParams p) {
-  extern __shared__ uint32_t cand_s[];  // kSelectCap keys
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t s_bin, s_rank, s_cnt;
+__global__ void __launch_bounds__(kSelClusterThreads) atopn_cluster_select_kernel(const SelectParams p) {
+  extern __shared__ uint32_t ccand[];  // this CTA's candidates (kSelectCap keys)
+  __shared__ uint32_t hist[256], tot[256];
+  __shared__ uint32_t s_bin, s_rank, s_cnt, counted;
   __shared__ int ncand;
-  const int r = blockIdx.x;
+  const int c = blockIdx.x, r = blockIdx.y;  // rank in the cluster, row
   pdl_trigger();
   pdl_wait();
   int L = p.row_len;
   if (p.seq_len_dev != nullptr) L = device_seq_len(p.seq_len_dev, p.row_len, p.l_cap, nullptr);
-  if (p.n_top >= L) {
-    if (threadIdx.x == 0) p.tau[r] = -INFINITY;
+  if (p.n_top >= L) {  // uniform over the cluster: no CTA reaches a cluster barrier
+    if (c == 0 && threadIdx.x == 0) p.tau[r] = -INFINITY;
     return;
   }
-  uint32_t b1, b2, rank, cnt;
-  two_bins(p, r, &s_bin, &s_rank, &s_cnt, &b1, &b2, &rank, &cnt);
-  uint32_t prefix = (b1 << 24) | (b2 << 16), mask = 0xFFFF0000u;
   const float* row = p.scores + (size_t)r * p.ld;
-  const bool collected = cnt <= (uint32_t)p.cand_cap && cnt <= (uint32_t)kSelectCap;
-  if (threadIdx.x == 0) ncand = 0;
-  __syncthreads();
-  if (collected) {
-    const uint32_t* cg = p.cand + (size_t)r * p.cand_cap;
-    for (int i = threadIdx.x; i < (int)cnt; i += blockDim.x) cand_s[i] = __ldcg(cg + i);
-    if (threadIdx.x == 0) ncand = (int)cnt;
+  int beg, end;
+  sel_chunk(L, c, kSelCluster, &beg, &end);
+  // adds the cluster's histograms into tot (every CTA), then finds the bin of `rank`
+  auto cluster_bin = [&](uint32_t rank) {
+    __syncthreads();
+    cluster_sync_all();
+    for (int i = threadIdx.x; i < 256; i += kSelClusterThreads) {
+      uint32_t sum = 0u;
+#pragma unroll
+      for (int cc = 0; cc < kSelCluster; ++cc) sum += ld_dsmem_u32(&hist[i], cc);
+      tot[i] = sum;
+    }
+    cluster_sync_all();  // every CTA has read every histogram before any is cleared
+    if (threadIdx.x == 0) {
+      s_bin = 0;
+      s_rank = 1;
+      s_cnt = 0;
+    }
+    __syncthreads();
+    find_bin(tot, rank, &s_bin, &s_rank, &s_cnt);
+    __syncthreads();
+  };
+  if (threadIdx.x == 0) {
+    ncand = 0;
+    counted = 0u;
   }
   __syncthreads();
-  bool in_smem = collected;
-  for (int shift = 8; shift >= 0; shift -= 8) {
-    if (!in_smem && cnt <= (uint32_t)kSelectCap) {
-      scan_row(row, L, [&](uint32_t k, bool ok) {
+  // top digit: the dumped histogram when its bins hold N scores, else counted here
+  for (int i = threadIdx.x; i < 256; i += kSelClusterThreads) {
+    tot[i] = p.hist != nullptr ? p.hist[(size_t)r * 256 + i] : 0u;
+    if (tot[i] != 0u) atomicAdd(&counted, tot[i]);
+  }
+  __syncthreads();
+  if (p.hist == nullptr || counted < (uint32_t)p.n_top) {  // uniform: every CTA read the same histogram
+    for (int i = threadIdx.x; i < 256; i += kSelClusterThreads) hist[i] = 0u;
+    __syncthreads();
+    scan_range(row, beg, end, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
+    cluster_bin((uint32_t)p.n_top);
+  } else {
+    if (threadIdx.x == 0) {
+      s_bin = 0;
+      s_rank = 1;
+      s_cnt = 0;
+    }
+    __syncthreads();
+    find_bin(tot, (uint32_t)p.n_top, &s_bin, &s_rank, &s_cnt);
+    __syncthreads();
+  }
+  uint32_t prefix = s_bin << 24, mask = 0xFF000000u, rank = s_rank, cnt = s_cnt;
+  bool in_smem = false;
+  for (int shift = 16; shift >= 0; shift -= 8) {
+    if (!in_smem && cnt <= (uint32_t)kSelectCap) {  // this CTA's matches are at most the cluster's cnt
+      scan_range(row, beg, end, [&](uint32_t k, bool ok) {
         if (ok && (k & mask) == prefix) {
           const int pos = atomicAdd(&ncand, 1);
-          if (pos < kSelectCap) cand_s[pos] = k;
+          if (pos < kSelectCap) ccand[pos] = k;
         }
       });
       in_smem = true;
     }
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0u;
+    for (int i = threadIdx.x; i < 256; i += kSelClusterThreads) hist[i] = 0u;
     __syncthreads();
     if (in_smem) {
       const int n = min(ncand, kSelectCap);
-      for (int i = threadIdx.x; i < ((n + 31) & ~31); i += blockDim.x) {
-        const bool ok = i < n && (cand_s[i] & mask) == prefix;
-        hist_add(hist, ok ? (cand_s[i] >> shift) & 255u : 0u, ok);
+      for (int i = threadIdx.x; i < ((n + 31) & ~31); i += kSelClusterThreads) {
+        const bool ok = i < n && (ccand[i] & mask) == prefix;
+        hist_add(hist, ok ? (ccand[i] >> shift) & 255u : 0u, ok);
       }
     } else {
-      scan_row(row, L, [&](uint32_t k, bool ok) {
+      scan_range(row, beg, end, [&](uint32_t k, bool ok) {
         const bool m = ok && (k & mask) == prefix;
         hist_add(hist, m ? (k >> shift) & 255u : 0u, m);
       });
     }
-    __syncthreads();
-    find_bin(hist, rank, &s_bin, &s_rank, &s_cnt);
-    __syncthreads();
+    cluster_bin(rank);
     prefix |= s_bin << shift;
     mask |= 0xFFu << shift;
     rank = s_rank;
     cnt = s_cnt;
     __syncthreads();
   }
-  if (threadIdx.x == 0) p.tau[r] = key_float(prefix);
+  if (c == 0 && threadIdx.x == 0) p.tau[r] = key_float(prefix);
 }
 
 // ============================================================================ append + fill
@@ -2486,24 +2441,27 @@ cudaError_t launch_select(const SelectParams& p, int rows, cudaStream_t st) {
   return launch_k(atopn_select_kernel, dim3(rows), dim3(kSelectThreads), bytes, st, p);
 }
 
-// The refresh path's select (needs p.hist, p.hist2, p.cand_cnt zeroed, p.cand).
-cudaError_t launch_select_parallel(const SelectParams& p, int rows, cudaStream_t st) {
+// The refresh path's select for a few long rows: one cluster of CTAs per row.
+cudaError_t launch_select_cluster(const SelectParams& p, int rows, cudaStream_t st) {
   static std::atomic<uint64_t> prepared{0};
   const int bytes = kSelectCap * 4;
-  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(atopn_resolve_kernel), bytes, prepared);
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(atopn_cluster_select_kernel), bytes, prepared);
   if (e != cudaSuccess) return e;
-  // parts per row: about 8K scores each, at most 32
-  const int parts = max(1, min(32, (p.row_len + 8191) / 8192));
-  static std::atomic<uint64_t> prep_h{0}, prep_c{0};
-  e = ensure_smem(reinterpret_cast<const void*>(atopn_hist2_kernel), 0, prep_h);
-  if (e != cudaSuccess) return e;
-  e = ensure_smem(reinterpret_cast<const void*>(atopn_collect_kernel), 0, prep_c);
-  if (e != cudaSuccess) return e;
-  e = launch_k(atopn_hist2_kernel, dim3(rows, parts), dim3(kSelPartThreads), 0, st, p);
-  if (e != cudaSuccess) return e;
-  e = launch_k(atopn_collect_kernel, dim3(rows, parts), dim3(kSelPartThreads), 0, st, p);
-  if (e != cudaSuccess) return e;
-  return launch_k(atopn_resolve_kernel, dim3(rows), dim3(kSelectThreads), bytes, st, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kSelCluster, rows);
+  cfg.blockDim = dim3(kSelClusterThreads);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSelCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, atopn_cluster_select_kernel, p);
 }
 
 template <int NB>

@@ -147,7 +147,7 @@ class DecodeSession:
         """Kernels of this library launched per decode step (the append is fused into the first of them)."""
         dense = self.n_top >= self.shape.l_cap
         if refresh_step and not dense:
-            per_layer = 6  # score dump (+append), three radix-select kernels, from-scores, combine
+            per_layer = 4  # score dump (+append), radix select, from-scores, combine
         elif refresh_step and dense:
             per_layer = 3  # threshold fill, split (+append), combine
         else:

@@ -175,6 +175,27 @@ def test_refresh_with_any_stale_threshold_is_exact(stale):
     assert np.max(np.abs(tau.cpu().numpy() - expect)) <= gpu_harness.BAND
 
 
+@pytest.mark.parametrize("stale", ["zero", "huge", "mixed"])
+def test_refresh_of_long_rows_is_exact(stale):
+    """Rows longer than 32K scores, fewer rows than SMs: one thread-block cluster per row finds the N-th
+    largest; any stale threshold gives the same bits and the oracle's threshold."""
+    wl = small("refresh_long", h_q=12, h_k=1, h_v=4, d=128, l_kv=40000, n_top=300)
+    inp = workload.make_layer(wl, 0, steps=1)
+    shape = saga.SagaShape.of(1, 12, 1, 4, 128, 40000)
+    kc = inp["K0"].cuda().contiguous()
+    q = inp["q"][0].cuda().contiguous()
+    ws = saga.alloc_workspace(shape)
+    base = torch.zeros((1, 12), device="cuda")
+    saga.atopn_refresh_threshold(shape, q, kc, 40000, 300, base, ws)
+    tau = {"zero": torch.zeros((1, 12), device="cuda"), "huge": torch.full((1, 12), 1e30, device="cuda"),
+           "mixed": torch.tensor([[1e30, 0.0, -1e30, 5.0, float("nan"), 1e-30] * 2], device="cuda")}[stale]
+    saga.atopn_refresh_threshold(shape, q, kc, 40000, 300, tau, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(tau, base)
+    expect = saga_oracle.refresh_threshold(inp["q"][0].float().numpy(), inp["K0"].float().numpy(), 40000, 300)
+    assert np.max(np.abs(tau.cpu().numpy() - expect)) <= gpu_harness.BAND
+
+
 def test_empty_selection_gives_zero():
     """A stale threshold above every score of a later step keeps nothing: output 0, count 0."""
     shape = saga.SagaShape.of(1, 8, 1, 8, 64, 600)
