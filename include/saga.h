@@ -97,7 +97,7 @@ typedef struct saga_shape {
 
 /* Bytes of scratch that atopn_refresh_threshold and saga_decode_attn need for
  * this shape on the current device (split partials, the score rows of a
- * refresh step, radix histograms, per-split index lists, a status word).
+ * refresh step, per-split index lists, a status word).
  * The buffer is caller-owned device memory, 256-byte aligned, zero-filled
  * once before first use; calls on one workspace must not overlap in time.
  * Returns 0 for an invalid shape. */

@@ -146,8 +146,6 @@ WsLayout ws_layout(const saga_shape* s, int sms) {
   off = align256(off + (size_t)rows * w.s_cap * 4);
   w.scores = off;
   off = align256(off + (size_t)rows * w.ld_scores * 4);
-  w.hist = off;
-  off = align256(off + (size_t)rows * 256 * 4);
   w.idx = off;
   off = align256(off + (size_t)rows * s->l_cap * 4);
   w.total = off;
@@ -308,7 +306,7 @@ int clear_status_word(const Prepared& pr, cudaStream_t st) {
   return SAGA_OK;
 }
 
-// Scores of every cached token, their top-byte histograms, and the exact
+// Scores of every cached token and the exact
 // threshold (refresh).  clear_status zeroes the status word first.
 int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const void* k_cache, int seq_len,
                 const int* seq_len_dev, int n_top, float* tau, cudaStream_t st, cudaEvent_t ev_start = nullptr,
@@ -324,7 +322,6 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   rc = splits_for(s, pr, seq_len, NP, hsplit, kSplitDump, tf, tp, &S);
   if (rc) return rc;
   const size_t rows = (size_t)s->batch * s->h_q;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(pr.base + pr.ws.hist);
   if (clear_status) {
     rc = clear_status_word(pr, st);
     if (rc) return rc;
@@ -333,8 +330,6 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
     cudaError_t et = trace_record(ev_start, st);
     if (et != cudaSuccess) return cuda_fail(et, "trace event record");
   }
-  cudaError_t e = cudaMemsetAsync(hist, 0, rows * 256 * 4, st);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(hist)");
   SplitParams p;
   fill_split_common(p, s, pr, q, k_cache, seq_len, seq_len_dev, true);
   p.k_cache_w = nr.k_cache;
@@ -342,25 +337,23 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   p.k_new = nr.k_new;
   p.v_new = nr.v_new;
   p.scores_out = reinterpret_cast<float*>(pr.base + pr.ws.scores);
-  p.hist_out = hist;
-  // One CTA per row scanning the whole row when the rows fill the GPU or are
-  // short; else one thread-block cluster of CTAs per row, each CTA a chunk.
-  // Measured on refresh steps: rows of 32K scores (32 rows) 688 vs 746 us and
-  // 512 rows of 128K 10.95 vs 11.94 ms per step with one CTA per row than with
-  // rows in chunks over three kernels; for 12 and 32 rows of 128K the cluster
-  // kernel against those three kernels: 1546 vs 1730 us and 1048 vs 1158 us.
-  // Both recount a row whose dumped histogram misses the N-th largest, so the
-  // dump counts only the bins near the stale threshold.
+  // The select: one CTA per row scanning the whole row when the rows fill the
+  // GPU or are short; else one thread-block cluster of CTAs per row, each CTA
+  // a chunk.  Measured on refresh steps: rows of 32K scores (32 rows) 688 vs
+  // 746 us and 512 rows of 128K 10.95 vs 11.94 ms per step with one CTA per
+  // row than with rows in chunks over three kernels; for 12 and 32 rows of
+  // 128K the cluster kernel against those three kernels: 1546 vs 1730 us and
+  // 1048 vs 1158 us.  The selects count every digit themselves: a top-byte
+  // histogram fused into the dump cost the dump two thirds of its time with
+  // the layers of a step in one call (485 vs 175 us), more than the select's
+  // own pass (148 vs 55 us).
   const bool one_cta_per_row = rows >= (size_t)pr.sms || seq_len <= 32768;
-  p.hist_floor = 1;
-  p.tau = tau;  // the stale threshold, read by the dump before the select overwrites it
   p.nsplit = S;
-  e = launch_split(s->d, NP, kSplitDump, tf, tp, p, dim3(S * hsplit, s->h_k, s->batch), st, nullptr);
+  cudaError_t e = launch_split(s->d, NP, kSplitDump, tf, tp, p, dim3(S * hsplit, s->h_k, s->batch), st, nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "score dump launch");
   SelectParams sp{};
   sp.scores = p.scores_out;
   sp.ld = pr.ws.ld_scores;
-  sp.hist = hist;
   sp.tau = tau;
   sp.status = p.status;
   sp.seq_len_dev = seq_len_dev;
@@ -516,7 +509,6 @@ int atopn_select_threshold(const float* scores, int rows, int row_len, long long
   SelectParams sp{};
   sp.scores = scores;
   sp.ld = row_stride;
-  sp.hist = nullptr;
   sp.tau = tau;
   sp.status = static_cast<unsigned*>(workspace);
   sp.seq_len_dev = nullptr;

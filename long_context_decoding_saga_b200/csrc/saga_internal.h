@@ -55,7 +55,6 @@ struct WsLayout {
   size_t part_l;    // float [B*h_q, S_cap]
   size_t part_cnt;  // int   [B*h_q, S_cap]
   size_t scores;    // float [B*h_q, ld_scores]
-  size_t hist;      // uint32 [B*h_q, 256] top-byte histograms of the dumped scores
   size_t idx;       // int   [B*h_q, l_cap]
   size_t total;
   int s_cap;
@@ -73,8 +72,6 @@ struct SplitParams {
   const float* tau;         // [B, h_q]
   const float* scores_in;   // from-scores mode: [B*h_q, ld_scores]
   float* scores_out;        // dump mode
-  uint32_t* hist_out;       // dump mode: [B*h_q, 256]
-  int hist_floor;           // dump mode: count only top-byte bins from two below the stale tau's bin up
   float* part_o;
   float* part_m;
   float* part_l;
@@ -121,7 +118,6 @@ struct CombineParams {
 struct SelectParams {
   const float* scores;
   long long ld;
-  const uint32_t* hist;  // nullable: precomputed top-byte histogram [rows, 256] (may count only upper bins)
   float* tau;
   unsigned* status;
   const int* seq_len_dev;  // nullable: row length from the device

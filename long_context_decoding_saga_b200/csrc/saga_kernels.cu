@@ -13,9 +13,10 @@
 //                    softmax and value sum of eq. 7 online over the h_v
 //                    value heads, writing one (max, sum, o) partial per split.
 //   dump variant   : refresh steps (Atop-N step 2) - the same scores are
-//                    written out with a per-head histogram of their top byte.
+//                    written out.
 //   select kernels : exact N-th largest score per row by radix selection
-//                    (many CTAs per row on refresh steps).
+//                    (one CTA per row, or one thread-block cluster per row
+//                    for a few long rows).
 //   from-scores    : refresh steps - compare/gather from the dumped scores.
 //   dense kernel   : every token kept, one value head per group - value
 //                    tiles by TMA, online softmax per tile, no lists.
@@ -740,7 +741,6 @@ struct SplitSmem {
   static_assert(ALLOC <= kSmemLimit, "shared memory over the per-CTA limit");
   static_assert(!TWO || ALLOC <= kSmemHalf, "two CTAs per SM must fit in half the shared memory");
   static_assert(merge_floats<D, NP>() * 4 <= NSTAGE * STAGE_BYTES, "merge buffer must fit in the key stages");
-  static_assert(NP * 256 * 4 <= (int)sizeof(WarpList<NP>) * 8, "dump histogram must fit in the warp lists");
 };
 
 // Fused append: row pos of key head h and of the group's value heads, from
@@ -811,7 +811,6 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
   uint8_t* qsm = smem + SM::Q_OFF;
   EpiShared<NP>& es = *reinterpret_cast<EpiShared<NP>*>(smem + SM::EPI_OFF);
   uint16_t* vstage = reinterpret_cast<uint16_t*>(smem + SM::VST_OFF);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(&es.list[0][0]);  // dump mode: [NP][256]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFF);
   uint64_t* empty = full + NSTAGE;
   uint64_t* accf = empty + NSTAGE;
@@ -894,7 +893,6 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
         qv[k] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.h_q + j0 + n) * D + col));
     }
     tv = load_tau<NP>(eth, p, b, j0, !DUMP);
-    if (DUMP && p.hist_floor != 0 && p.tau != nullptr && eth < p.G) tv = __ldg(p.tau + (size_t)b * p.h_q + j0 + eth);
   }
   // the epilogue compares raw dot products (scaled only once listed)
   if (!DUMP && warp >= 2 && eth < NP) tv = raw_threshold(tv, p.scale);
@@ -932,8 +930,6 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
         }
       }
     }
-    if (DUMP)
-      for (int i = eth; i < NP * 256; i += kEpiThreads) hist[i] = 0u;
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
@@ -990,21 +986,6 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     acc.init();
     ListState ls{0, 0, -1, 0};
     const size_t srow = ((size_t)b * p.h_q + j0) * (size_t)p.ld_scores;
-    // dump mode: the histogram only needs exact counts from the bin holding the N-th largest up, so with
-    // hist_floor it counts the top-byte bins from two below the stale threshold's bin (four times smaller
-    // magnitudes) up; the select checks that the counted bins hold N scores and otherwise recounts the row
-    uint32_t bfl[NP];
-#pragma unroll
-    for (int jl = 0; jl < NP; ++jl) {
-      bfl[jl] = 0u;
-      if (DUMP && p.hist_floor != 0 && jl < p.G) {
-        const float ts = es.tau[jl];  // the stale threshold (scaled, as the dumped scores)
-        if (ts != -INFINITY && ts == ts) {
-          const uint32_t tb = float_key(ts) >> 24;
-          bfl[jl] = tb > 2u ? tb - 2u : 0u;
-        }
-      }
-    }
     int t = 0;
     if (!DUMP && p.test_wait_ns != 0u) {
       bool ok = __all_sync(0xffffffffu, mbar_wait(never, 0, abort_flag, p.test_wait_ns));
@@ -1043,15 +1024,7 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
       if (DUMP) {
 #pragma unroll
         for (int jl = 0; jl < NP; ++jl) {
-          if (jl < p.G) {
-            if (valid) p.scores_out[srow + (size_t)jl * p.ld_scores + tok] = sc[jl];
-            const uint32_t bin = float_key(sc[jl]) >> 24;
-            const bool counted = valid && bin >= bfl[jl];
-            if (__any_sync(0xffffffffu, counted)) {
-              const uint32_t peers = __match_any_sync(0xffffffffu, counted ? bin : 256u);
-              if (counted && lane == __ffs(peers) - 1) atomicAdd(&hist[jl * 256 + bin], (uint32_t)__popc(peers));
-            }
-          }
+          if (jl < p.G && valid) p.scores_out[srow + (size_t)jl * p.ld_scores + tok] = sc[jl];
         }
       } else {
         tile_epilogue<D, NP>(es, acc, ea, ls, q, lane, et, sc, tok, valid, counting, p, b, j0, start, vstage_w);
@@ -1074,13 +1047,6 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     if (warp == 0 && lane == 0) {
       // wait (bounded) for the last copy issued into each stage
       for (int t = max(0, issued - NSTAGE); t < issued; ++t) mbar_wait_drain(&full[t % NSTAGE], (t / NSTAGE) & 1);
-    }
-  }
-  if (DUMP && warp >= 2) {
-    const int et = threadIdx.x - 64;
-    for (int i = et; i < p.G * 256; i += kEpiThreads) {
-      const uint32_t c = hist[i];
-      if (c) atomicAdd(&p.hist_out[((size_t)b * p.h_q + j0 + i / 256) * 256 + (i % 256)], c);
     }
   }
   __syncthreads();
@@ -1774,29 +1740,17 @@ __global__ void __launch_bounds__(kSelectThreads) atopn_select_kernel(const Sele
   }
   const float* row = p.scores + (size_t)r * p.ld;
 
-  // a given top-digit histogram may count only the bins from some floor up
-  // (the score dump counts from just below the stale threshold): it serves
-  // when its bins hold at least N scores, else the row is counted here
-  __shared__ uint32_t counted;
   if (threadIdx.x == 0) {
     ncand = 0;
     s_bin = 0;
     s_rank = 1;
     s_cnt = 0;
-    counted = 0u;
   }
+  for (int i = threadIdx.x; i < 256; i += kSelectThreads) hist[i] = 0u;
   __syncthreads();
-  for (int i = threadIdx.x; i < 256; i += kSelectThreads) {
-    hist[i] = p.hist != nullptr ? p.hist[(size_t)r * 256 + i] : 0u;
-    if (hist[i] != 0u) atomicAdd(&counted, hist[i]);
-  }
+  // top digit: a histogram of the whole row
+  scan_row(row, L, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
   __syncthreads();
-  if (p.hist == nullptr || counted < (uint32_t)p.n_top) {  // top digit histogram of the whole row
-    for (int i = threadIdx.x; i < 256; i += kSelectThreads) hist[i] = 0u;
-    __syncthreads();
-    scan_row(row, L, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
-    __syncthreads();
-  }
   find_bin(hist, (uint32_t)p.n_top, &s_bin, &s_rank, &s_cnt);
   __syncthreads();
   uint32_t prefix = s_bin << 24, mask = 0xFF000000u, rank = s_rank, cnt = s_cnt;
@@ -1889,16 +1843,15 @@ __device__ __forceinline__ void sel_chunk(int L, int part, int P, int* b, int* e
 // distributed shared memory (so every CTA holds the same sums and takes the
 // same decision) and finds the digit's bin.  Once the keys matching the
 // prefix fit, each CTA keeps its own in shared memory and the remaining
-// digits are resolved over those.  A given top-digit histogram (from the
-// score dump) is used when its bins hold N scores.  Cluster barriers are
-// hardware barriers every CTA reaches on every path.
+// digits are resolved over those.  Cluster barriers are hardware barriers
+// every CTA reaches on every path.
 constexpr int kSelCluster = 8;          // CTAs per row
 constexpr int kSelClusterThreads = 512;
 
 __global__ void __launch_bounds__(kSelClusterThreads) atopn_cluster_select_kernel(const SelectParams p) {
   extern __shared__ uint32_t ccand[];  // this CTA's candidates (kSelectCap keys)
   __shared__ uint32_t hist[256], tot[256];
-  __shared__ uint32_t s_bin, s_rank, s_cnt, counted;
+  __shared__ uint32_t s_bin, s_rank, s_cnt;
   __shared__ int ncand;
   const int c = blockIdx.x, r = blockIdx.y;  // rank in the cluster, row
   pdl_trigger();
@@ -1932,32 +1885,12 @@ __global__ void __launch_bounds__(kSelClusterThreads) atopn_cluster_select_kerne
     find_bin(tot, rank, &s_bin, &s_rank, &s_cnt);
     __syncthreads();
   };
-  if (threadIdx.x == 0) {
-    ncand = 0;
-    counted = 0u;
-  }
+  if (threadIdx.x == 0) ncand = 0;
+  for (int i = threadIdx.x; i < 256; i += kSelClusterThreads) hist[i] = 0u;
   __syncthreads();
-  // top digit: the dumped histogram when its bins hold N scores, else counted here
-  for (int i = threadIdx.x; i < 256; i += kSelClusterThreads) {
-    tot[i] = p.hist != nullptr ? p.hist[(size_t)r * 256 + i] : 0u;
-    if (tot[i] != 0u) atomicAdd(&counted, tot[i]);
-  }
-  __syncthreads();
-  if (p.hist == nullptr || counted < (uint32_t)p.n_top) {  // uniform: every CTA read the same histogram
-    for (int i = threadIdx.x; i < 256; i += kSelClusterThreads) hist[i] = 0u;
-    __syncthreads();
-    scan_range(row, beg, end, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
-    cluster_bin((uint32_t)p.n_top);
-  } else {
-    if (threadIdx.x == 0) {
-      s_bin = 0;
-      s_rank = 1;
-      s_cnt = 0;
-    }
-    __syncthreads();
-    find_bin(tot, (uint32_t)p.n_top, &s_bin, &s_rank, &s_cnt);
-    __syncthreads();
-  }
+  // top digit: this CTA's chunk counted, the cluster's counts summed
+  scan_range(row, beg, end, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
+  cluster_bin((uint32_t)p.n_top);
   uint32_t prefix = s_bin << 24, mask = 0xFF000000u, rank = s_rank, cnt = s_cnt;
   bool in_smem = false;
   for (int shift = 16; shift >= 0; shift -= 8) {
