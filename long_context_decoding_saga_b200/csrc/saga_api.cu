@@ -146,6 +146,8 @@ WsLayout ws_layout(const saga_shape* s, int sms) {
   off = align256(off + (size_t)rows * w.s_cap * 4);
   w.scores = off;
   off = align256(off + (size_t)rows * w.ld_scores * 4);
+  w.hist = off;
+  off = align256(off + (size_t)rows * 256 * 4);
   w.idx = off;
   off = align256(off + (size_t)rows * s->l_cap * 4);
   w.total = off;
@@ -343,10 +345,22 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   // 746 us and 512 rows of 128K 10.95 vs 11.94 ms per step with one CTA per
   // row than with rows in chunks over three kernels; for 12 and 32 rows of
   // 128K the cluster kernel against those three kernels: 1546 vs 1730 us and
-  // 1048 vs 1158 us.  The selects count every digit themselves: a top-byte
-  // histogram fused into the dump cost the dump two thirds of its time with
-  // the layers of a step in one call (485 vs 175 us), more than the select's
-  // own pass (148 vs 55 us).
+  // 1048 vs 1158 us.  For groups of at most kDumpHistMaxNp heads the dump
+  // also counts the top byte of the scores from two bins below the stale
+  // threshold's up, and the select skips its first pass when those bins hold
+  // N scores (else it counts the row itself, so any tau is exact).  With 12
+  // heads per CTA that counting had cost the dump two thirds of its time (485
+  // vs 175 us for 28 layers in one call), more than the pass it saves (148 vs
+  // 55 us); with 4 heads the refresh steps are 11-16 % faster with it.
+  uint32_t* hist = nullptr;
+  if (NP <= kDumpHistMaxNp) {
+    hist = reinterpret_cast<uint32_t*>(pr.base + pr.ws.hist);
+    cudaError_t em = cudaMemsetAsync(hist, 0, rows * 256 * 4, st);
+    if (em != cudaSuccess) return cuda_fail(em, "cudaMemsetAsync(hist)");
+    p.hist_out = hist;
+    p.hist_floor = 1;
+    p.tau = tau;  // the stale threshold, read by the dump before the select overwrites it
+  }
   const bool one_cta_per_row = rows >= (size_t)pr.sms || seq_len <= 32768;
   p.nsplit = S;
   cudaError_t e = launch_split(s->d, NP, kSplitDump, tf, tp, p, dim3(S * hsplit, s->h_k, s->batch), st, nullptr);
@@ -354,6 +368,7 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   SelectParams sp{};
   sp.scores = p.scores_out;
   sp.ld = pr.ws.ld_scores;
+  sp.hist = hist;
   sp.tau = tau;
   sp.status = p.status;
   sp.seq_len_dev = seq_len_dev;

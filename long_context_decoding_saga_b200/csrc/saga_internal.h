@@ -55,6 +55,7 @@ struct WsLayout {
   size_t part_l;    // float [B*h_q, S_cap]
   size_t part_cnt;  // int   [B*h_q, S_cap]
   size_t scores;    // float [B*h_q, ld_scores]
+  size_t hist;      // uint32 [B*h_q, 256] top-byte counts of the dumped scores (groups of <= 4 heads)
   size_t idx;       // int   [B*h_q, l_cap]
   size_t total;
   int s_cap;
@@ -72,6 +73,8 @@ struct SplitParams {
   const float* tau;         // [B, h_q]
   const float* scores_in;   // from-scores mode: [B*h_q, ld_scores]
   float* scores_out;        // dump mode
+  uint32_t* hist_out;       // dump mode, padded groups of <= 4 heads: [B*h_q, 256], else null
+  int hist_floor;           // dump mode: count only top-byte bins from two below the stale tau's bin up
   float* part_o;
   float* part_m;
   float* part_l;
@@ -115,9 +118,17 @@ struct CombineParams {
   int out_bf16;
 };
 
+// The score dump also counts the top byte of the scores near the stale
+// threshold (so the select can skip its first pass) only for padded groups of
+// at most this many heads: there the counting costs little next to the key
+// stream; with 8 or 16 heads per CTA it took half the dump's time or more.
+constexpr int kDumpHistMaxNp = 4;
+
 struct SelectParams {
   const float* scores;
   long long ld;
+  const uint32_t* hist;  // nullable: top-byte counts [rows, 256] that may hold only the upper bins; a row
+                         // whose counted bins hold fewer than n_top scores is counted again
   float* tau;
   unsigned* status;
   const int* seq_len_dev;  // nullable: row length from the device

@@ -13,7 +13,8 @@
 //                    softmax and value sum of eq. 7 online over the h_v
 //                    value heads, writing one (max, sum, o) partial per split.
 //   dump variant   : refresh steps (Atop-N step 2) - the same scores are
-//                    written out.
+//                    written out (for groups of up to 4 heads, with counts
+//                    of their top byte near the stale threshold).
 //   select kernels : exact N-th largest score per row by radix selection
 //                    (one CTA per row, or one thread-block cluster per row
 //                    for a few long rows).
@@ -741,6 +742,8 @@ struct SplitSmem {
   static_assert(ALLOC <= kSmemLimit, "shared memory over the per-CTA limit");
   static_assert(!TWO || ALLOC <= kSmemHalf, "two CTAs per SM must fit in half the shared memory");
   static_assert(merge_floats<D, NP>() * 4 <= NSTAGE * STAGE_BYTES, "merge buffer must fit in the key stages");
+  static_assert(NP > kDumpHistMaxNp || NP * 256 * 4 <= (int)sizeof(WarpList<NP>) * 8,
+                "dump counts must fit in the warp lists");
 };
 
 // Fused append: row pos of key head h and of the group's value heads, from
@@ -796,6 +799,8 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     saga_split_kernel(const __grid_constant__ CUtensorMap tmap_full, const __grid_constant__ CUtensorMap tmap_part,
                       const SplitParams p) {
   static_assert(UMMA, "scores come from tcgen05 for every group size");
+  // dump of a small group: also count the top byte of the scores near the stale threshold
+  constexpr bool DHIST = DUMP && NP <= kDumpHistMaxNp;
   using SM = SplitSmem<D, NP, UMMA>;
   constexpr int NATOM = SM::NATOM;
   constexpr int NSTAGE = SM::NSTAGE;
@@ -811,6 +816,7 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
   uint8_t* qsm = smem + SM::Q_OFF;
   EpiShared<NP>& es = *reinterpret_cast<EpiShared<NP>*>(smem + SM::EPI_OFF);
   uint16_t* vstage = reinterpret_cast<uint16_t*>(smem + SM::VST_OFF);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(&es.list[0][0]);  // DHIST: [NP][256]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFF);
   uint64_t* empty = full + NSTAGE;
   uint64_t* accf = empty + NSTAGE;
@@ -893,6 +899,7 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
         qv[k] = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.h_q + j0 + n) * D + col));
     }
     tv = load_tau<NP>(eth, p, b, j0, !DUMP);
+    if (DHIST && p.hist_out != nullptr && p.tau != nullptr && eth < p.G) tv = __ldg(p.tau + (size_t)b * p.h_q + j0 + eth);
   }
   // the epilogue compares raw dot products (scaled only once listed)
   if (!DUMP && warp >= 2 && eth < NP) tv = raw_threshold(tv, p.scale);
@@ -930,6 +937,8 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
         }
       }
     }
+    if (DHIST)
+      for (int i = eth; i < NP * 256; i += kEpiThreads) hist[i] = 0u;
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   tc_fence_before();
@@ -986,6 +995,21 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     acc.init();
     ListState ls{0, 0, -1, 0};
     const size_t srow = ((size_t)b * p.h_q + j0) * (size_t)p.ld_scores;
+    // DHIST: the select needs exact counts only from the bin of the N-th largest up, so the top-byte
+    // bins from two below the stale threshold's bin (a fourth of its magnitude) up are counted; the
+    // select checks that the counted bins hold N scores and otherwise counts the row itself
+    uint32_t bfl[NP];
+#pragma unroll
+    for (int jl = 0; jl < NP; ++jl) {
+      bfl[jl] = 0u;
+      if (DHIST && p.hist_floor != 0 && jl < p.G) {
+        const float ts = es.tau[jl];  // the stale threshold (scaled, as the dumped scores)
+        if (ts != -INFINITY && ts == ts) {
+          const uint32_t tb = float_key(ts) >> 24;
+          bfl[jl] = tb > 2u ? tb - 2u : 0u;
+        }
+      }
+    }
     int t = 0;
     if (!DUMP && p.test_wait_ns != 0u) {
       bool ok = __all_sync(0xffffffffu, mbar_wait(never, 0, abort_flag, p.test_wait_ns));
@@ -1024,7 +1048,17 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
       if (DUMP) {
 #pragma unroll
         for (int jl = 0; jl < NP; ++jl) {
-          if (jl < p.G && valid) p.scores_out[srow + (size_t)jl * p.ld_scores + tok] = sc[jl];
+          if (jl < p.G) {
+            if (valid) p.scores_out[srow + (size_t)jl * p.ld_scores + tok] = sc[jl];
+            if (DHIST && p.hist_out != nullptr) {
+              const uint32_t bin = float_key(sc[jl]) >> 24;
+              const bool counted = valid && bin >= bfl[jl];
+              if (__any_sync(0xffffffffu, counted)) {
+                const uint32_t peers = __match_any_sync(0xffffffffu, counted ? bin : 256u);
+                if (counted && lane == __ffs(peers) - 1) atomicAdd(&hist[jl * 256 + bin], (uint32_t)__popc(peers));
+              }
+            }
+          }
         }
       } else {
         tile_epilogue<D, NP>(es, acc, ea, ls, q, lane, et, sc, tok, valid, counting, p, b, j0, start, vstage_w);
@@ -1047,6 +1081,13 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     if (warp == 0 && lane == 0) {
       // wait (bounded) for the last copy issued into each stage
       for (int t = max(0, issued - NSTAGE); t < issued; ++t) mbar_wait_drain(&full[t % NSTAGE], (t / NSTAGE) & 1);
+    }
+  }
+  if (DHIST && p.hist_out != nullptr && warp >= 2) {
+    const int et = threadIdx.x - 64;
+    for (int i = et; i < p.G * 256; i += kEpiThreads) {
+      const uint32_t c = hist[i];
+      if (c) atomicAdd(&p.hist_out[((size_t)b * p.h_q + j0 + i / 256) * 256 + (i % 256)], c);
     }
   }
   __syncthreads();
@@ -1740,17 +1781,29 @@ __global__ void __launch_bounds__(kSelectThreads) atopn_select_kernel(const Sele
   }
   const float* row = p.scores + (size_t)r * p.ld;
 
+  // given top-digit counts may hold only the bins from some floor up (the
+  // score dump counts from just below the stale threshold): they serve when
+  // their bins hold at least N scores, else the row is counted here
+  __shared__ uint32_t counted;
   if (threadIdx.x == 0) {
     ncand = 0;
     s_bin = 0;
     s_rank = 1;
     s_cnt = 0;
+    counted = 0u;
   }
-  for (int i = threadIdx.x; i < 256; i += kSelectThreads) hist[i] = 0u;
   __syncthreads();
-  // top digit: a histogram of the whole row
-  scan_row(row, L, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
+  for (int i = threadIdx.x; i < 256; i += kSelectThreads) {
+    hist[i] = p.hist != nullptr ? p.hist[(size_t)r * 256 + i] : 0u;
+    if (hist[i] != 0u) atomicAdd(&counted, hist[i]);
+  }
   __syncthreads();
+  if (p.hist == nullptr || counted < (uint32_t)p.n_top) {  // top digit: a histogram of the whole row
+    for (int i = threadIdx.x; i < 256; i += kSelectThreads) hist[i] = 0u;
+    __syncthreads();
+    scan_row(row, L, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
+    __syncthreads();
+  }
   find_bin(hist, (uint32_t)p.n_top, &s_bin, &s_rank, &s_cnt);
   __syncthreads();
   uint32_t prefix = s_bin << 24, mask = 0xFF000000u, rank = s_rank, cnt = s_cnt;
@@ -1843,15 +1896,16 @@ __device__ __forceinline__ void sel_chunk(int L, int part, int P, int* b, int* e
 // distributed shared memory (so every CTA holds the same sums and takes the
 // same decision) and finds the digit's bin.  Once the keys matching the
 // prefix fit, each CTA keeps its own in shared memory and the remaining
-// digits are resolved over those.  Cluster barriers are hardware barriers
-// every CTA reaches on every path.
+// digits are resolved over those.  Given top-digit counts (from the score
+// dump) are used when their bins hold N scores.  Cluster barriers are
+// hardware barriers every CTA reaches on every path.
 constexpr int kSelCluster = 8;          // CTAs per row
 constexpr int kSelClusterThreads = 512;
 
 __global__ void __launch_bounds__(kSelClusterThreads) atopn_cluster_select_kernel(const SelectParams p) {
   extern __shared__ uint32_t ccand[];  // this CTA's candidates (kSelectCap keys)
   __shared__ uint32_t hist[256], tot[256];
-  __shared__ uint32_t s_bin, s_rank, s_cnt;
+  __shared__ uint32_t s_bin, s_rank, s_cnt, counted;
   __shared__ int ncand;
   const int c = blockIdx.x, r = blockIdx.y;  // rank in the cluster, row
   pdl_trigger();
@@ -1885,12 +1939,33 @@ __global__ void __launch_bounds__(kSelClusterThreads) atopn_cluster_select_kerne
     find_bin(tot, rank, &s_bin, &s_rank, &s_cnt);
     __syncthreads();
   };
-  if (threadIdx.x == 0) ncand = 0;
-  for (int i = threadIdx.x; i < 256; i += kSelClusterThreads) hist[i] = 0u;
+  if (threadIdx.x == 0) {
+    ncand = 0;
+    counted = 0u;
+  }
   __syncthreads();
-  // top digit: this CTA's chunk counted, the cluster's counts summed
-  scan_range(row, beg, end, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
-  cluster_bin((uint32_t)p.n_top);
+  // top digit: the given counts when their bins hold N scores, else this
+  // CTA's chunk counted and the cluster's counts summed
+  for (int i = threadIdx.x; i < 256; i += kSelClusterThreads) {
+    tot[i] = p.hist != nullptr ? p.hist[(size_t)r * 256 + i] : 0u;
+    if (tot[i] != 0u) atomicAdd(&counted, tot[i]);
+  }
+  __syncthreads();
+  if (p.hist == nullptr || counted < (uint32_t)p.n_top) {  // uniform: every CTA read the same counts
+    for (int i = threadIdx.x; i < 256; i += kSelClusterThreads) hist[i] = 0u;
+    __syncthreads();
+    scan_range(row, beg, end, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
+    cluster_bin((uint32_t)p.n_top);
+  } else {
+    if (threadIdx.x == 0) {
+      s_bin = 0;
+      s_rank = 1;
+      s_cnt = 0;
+    }
+    __syncthreads();
+    find_bin(tot, (uint32_t)p.n_top, &s_bin, &s_rank, &s_cnt);
+    __syncthreads();
+  }
   uint32_t prefix = s_bin << 24, mask = 0xFF000000u, rank = s_rank, cnt = s_cnt;
   bool in_smem = false;
   for (int shift = 16; shift >= 0; shift -= 8) {

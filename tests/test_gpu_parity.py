@@ -151,23 +151,35 @@ def test_refresh_threshold_entry_point():
     assert np.max(np.abs(tau.cpu().numpy() - expect)) <= gpu_harness.BAND
 
 
+def _stale_tau(kind, h_q):
+    mixed = ([1e30, 0.0, -1e30, 5.0, float("nan"), 1e-30] * 4)[:h_q]
+    return {"zero": torch.zeros((1, h_q), device="cuda"), "huge": torch.full((1, h_q), 1e30, device="cuda"),
+            "tiny": torch.full((1, h_q), -1e30, device="cuda"),
+            "nan": torch.full((1, h_q), float("nan"), device="cuda"),
+            "mixed": torch.tensor([mixed], device="cuda")}[kind]
+
+
+# (h_q, h_k, h_v): 12 heads per key head (the select counts every digit itself) and 4 (the score dump also
+# counts the top byte of the scores near the stale threshold, which the select uses when it holds N scores)
+STALE_HEADS = [(12, 1, 4), (8, 2, 4)]
+
+
+@pytest.mark.parametrize("heads", STALE_HEADS, ids=lambda h: f"g{h[0] // h[1]}")
 @pytest.mark.parametrize("stale", ["huge", "tiny", "nan", "mixed"])
-def test_refresh_with_any_stale_threshold_is_exact(stale):
-    """The score dump counts only the top-byte bins from just below the stale threshold up, and the select
-    recounts a row whose counted bins hold fewer than N scores: whatever the stale values in tau (above every
-    score, below every score, NaN, or mixed per row), the refreshed threshold is the same bits as with a
-    stale threshold of 0, and the oracle's."""
-    wl = small("refresh_stale", h_q=12, h_k=1, h_v=4, d=128, l_kv=5000, n_top=77)
+def test_refresh_with_any_stale_threshold_is_exact(stale, heads):
+    """Whatever the stale values in tau (above every score, below every score, NaN, or mixed per row), the
+    refreshed threshold is the same bits as with a stale threshold of 0, and the oracle's: counts of the top
+    byte taken from just below the stale threshold up are used only when they hold N scores."""
+    h_q, h_k, h_v = heads
+    wl = small("refresh_stale", h_q=h_q, h_k=h_k, h_v=h_v, d=128, l_kv=5000, n_top=77)
     inp = workload.make_layer(wl, 0, steps=1)
-    shape = saga.SagaShape.of(1, 12, 1, 4, 128, 5000)
+    shape = saga.SagaShape.of(1, h_q, h_k, h_v, 128, 5000)
     kc = inp["K0"].cuda().contiguous()
     q = inp["q"][0].cuda().contiguous()
     ws = saga.alloc_workspace(shape)
-    base = torch.zeros((1, 12), device="cuda")
+    base = torch.zeros((1, h_q), device="cuda")
     saga.atopn_refresh_threshold(shape, q, kc, 5000, 77, base, ws)
-    tau = {"huge": torch.full((1, 12), 1e30, device="cuda"), "tiny": torch.full((1, 12), -1e30, device="cuda"),
-           "nan": torch.full((1, 12), float("nan"), device="cuda"),
-           "mixed": torch.tensor([[1e30, 0.0, -1e30, 5.0, float("nan"), 1e-30] * 2], device="cuda")}[stale]
+    tau = _stale_tau(stale, h_q)
     saga.atopn_refresh_threshold(shape, q, kc, 5000, 77, tau, ws)
     torch.cuda.synchronize()
     assert torch.equal(tau, base)
@@ -175,20 +187,21 @@ def test_refresh_with_any_stale_threshold_is_exact(stale):
     assert np.max(np.abs(tau.cpu().numpy() - expect)) <= gpu_harness.BAND
 
 
+@pytest.mark.parametrize("heads", STALE_HEADS, ids=lambda h: f"g{h[0] // h[1]}")
 @pytest.mark.parametrize("stale", ["zero", "huge", "mixed"])
-def test_refresh_of_long_rows_is_exact(stale):
+def test_refresh_of_long_rows_is_exact(stale, heads):
     """Rows longer than 32K scores, fewer rows than SMs: one thread-block cluster per row finds the N-th
     largest; any stale threshold gives the same bits and the oracle's threshold."""
-    wl = small("refresh_long", h_q=12, h_k=1, h_v=4, d=128, l_kv=40000, n_top=300)
+    h_q, h_k, h_v = heads
+    wl = small("refresh_long", h_q=h_q, h_k=h_k, h_v=h_v, d=128, l_kv=40000, n_top=300)
     inp = workload.make_layer(wl, 0, steps=1)
-    shape = saga.SagaShape.of(1, 12, 1, 4, 128, 40000)
+    shape = saga.SagaShape.of(1, h_q, h_k, h_v, 128, 40000)
     kc = inp["K0"].cuda().contiguous()
     q = inp["q"][0].cuda().contiguous()
     ws = saga.alloc_workspace(shape)
-    base = torch.zeros((1, 12), device="cuda")
+    base = torch.zeros((1, h_q), device="cuda")
     saga.atopn_refresh_threshold(shape, q, kc, 40000, 300, base, ws)
-    tau = {"zero": torch.zeros((1, 12), device="cuda"), "huge": torch.full((1, 12), 1e30, device="cuda"),
-           "mixed": torch.tensor([[1e30, 0.0, -1e30, 5.0, float("nan"), 1e-30] * 2], device="cuda")}[stale]
+    tau = _stale_tau(stale, h_q)
     saga.atopn_refresh_threshold(shape, q, kc, 40000, 300, tau, ws)
     torch.cuda.synchronize()
     assert torch.equal(tau, base)
