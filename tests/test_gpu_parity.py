@@ -28,8 +28,9 @@ def small(name, **kw):
     return W(**base)
 
 
-# Shapes spanning both scoring paths (CUDA cores for h_q/h_k <= 4, tcgen05 above), d = 64 and 128, value
-# heads above / equal to / below the key heads, batch > 1, ragged lengths (not multiples of 32 or 128).
+# Shapes spanning groups of 1 to 64 query heads per key head (groups of up to 4 also take the score dump's
+# top-byte counts on refresh steps), d = 64 and 128, value heads above / equal to / below the key heads,
+# batch > 1, ragged lengths (not multiples of 32 or 128).
 CASES = [
     small("g8_d64", h_q=8, h_k=1, h_v=8, d=64, l_kv=1000),
     small("g12_d128_hv4", h_q=12, h_k=1, h_v=4, d=128, l_kv=2085, n_top=50),
