@@ -63,11 +63,38 @@ def layer_bytes(wl, L):
     return 2 * wl.batch * wl.d * (keys + vals) + 2 * wl.batch * wl.h_q * wl.d + 4 * wl.batch * wl.h_q * wl.d
 
 
+def code_tokens(text):
+    """C/CUDA source with comments removed and whitespace collapsed (string and character literals kept
+    as written), so that a comment edit leaves the kernel's hash unchanged."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+            out.append(" ")
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash():
+    """Hash of the split kernel's sources (code only): the key of the recorded DRAM-traffic figure."""
     h = hashlib.sha256()
     for f in ("saga_kernels.cu", "saga_device.cuh", "saga_internal.h"):
-        with open(os.path.join(ROOT, "long_context_decoding_saga_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "long_context_decoding_saga_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(code_tokens(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

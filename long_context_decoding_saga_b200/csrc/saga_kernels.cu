@@ -996,8 +996,9 @@ __global__ void __launch_bounds__(192, SplitSmem<D, NP, UMMA>::CTAS_PER_SM)
     ListState ls{0, 0, -1, 0};
     const size_t srow = ((size_t)b * p.h_q + j0) * (size_t)p.ld_scores;
     // DHIST: the select needs exact counts only from the bin of the N-th largest up, so the top-byte
-    // bins from two below the stale threshold's bin (a fourth of its magnitude) up are counted; the
-    // select checks that the counted bins hold N scores and otherwise counts the row itself
+    // bins from two below the stale threshold's bin up are counted (a bin spans two binades, so for a
+    // positive threshold that reaches scores 16 to 64 times smaller); the select checks that the
+    // counted bins hold N scores and otherwise counts the row itself
     uint32_t bfl[NP];
 #pragma unroll
     for (int jl = 0; jl < NP; ++jl) {

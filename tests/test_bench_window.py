@@ -1,7 +1,8 @@
 """The benchmark's timed window (CPU only): it holds refresh and reuse steps
 in the proportion of the refresh schedule (the nearest whole number of
 refresh steps to K / R; exactly K / R when R divides K), and the per-kind
-means amortize over one refresh period."""
+means amortize over one refresh period.  Also the key of the recorded
+DRAM-traffic figure (the kernels' code without comments)."""
 import os
 import sys
 
@@ -58,3 +59,14 @@ def test_step_plan(warmup, steps, refresh, e2e):
         if e2e:
             assert bench.refresh_count(p["e2e_first"], p["E"], refresh) == int(p["E"] / refresh + 0.5)
     assert (p["E"] == 0) == (not e2e)
+
+
+def test_traffic_key_ignores_comments_only():
+    """The recorded DRAM-traffic figure is keyed by the kernels' code: comment and whitespace edits keep the
+    key, any code edit (a string literal's text included) changes it."""
+    src = 'int a = 1; // count\n/* two\n lines */ asm volatile("mov.u32 %0, 1; // x" : "=r"(a));\nchar c = \'/\';'
+    same = 'int a = 1;   /* another comment */\nasm volatile("mov.u32 %0, 1; // x" : "=r"(a)); // trailing\nchar c = \'/\';'
+    assert bench.code_tokens(src) == bench.code_tokens(same)
+    assert bench.code_tokens(src) != bench.code_tokens(src.replace("a = 1", "a = 2"))
+    assert bench.code_tokens(src) != bench.code_tokens(src.replace("// x", "// y"))
+    assert "//" in bench.code_tokens(src) and "count" not in bench.code_tokens(src)
