@@ -370,6 +370,7 @@ int run_refresh(const saga_shape* s, const Prepared& pr, const void* q, const vo
   sp.ld = pr.ws.ld_scores;
   sp.hist = hist;
   sp.tau = tau;
+  sp.spec = 1;  // tau holds the stale thresholds until the select writes the new ones
   sp.status = p.status;
   sp.seq_len_dev = seq_len_dev;
   sp.row_len = seq_len;

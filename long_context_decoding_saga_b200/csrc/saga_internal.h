@@ -135,6 +135,8 @@ struct SelectParams {
   int row_len;
   int l_cap;               // clamp bound for a device length
   int n_top;
+  int spec;                // tau holds the stale thresholds: the top-digit pass also keeps the keys from the
+                           // stale threshold's top-byte bin up, and skips the collection pass when they serve
 };
 
 // Decode-step QKV projection (eq. 1) fused with the KV-cache append.

@@ -1698,6 +1698,30 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool vali
   if (valid && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
 }
 
+// Appends k to cand when take (warp-aggregated: one shared atomic per warp);
+// *ncand counts every taken key, also those past kSelectCap.  Full warp.
+__device__ __forceinline__ void cand_add(uint32_t* cand, int* ncand, uint32_t k, bool take) {
+  const uint32_t m = __ballot_sync(0xffffffffu, take);
+  if (m == 0u) return;
+  const int lane = threadIdx.x & 31, first = __ffs(m) - 1;
+  int base = 0;
+  if (lane == first) base = atomicAdd(ncand, __popc(m));
+  base = __shfl_sync(0xffffffffu, base, first);
+  const int pos = base + __popc(m & ((1u << lane) - 1u));
+  if (take && pos < kSelectCap) cand[pos] = k;
+}
+
+// Top-byte bin of row r's stale threshold, from which the top-digit pass also
+// keeps candidates (the N-th largest mostly stays in its bin from one refresh
+// to the next); 256 = none: not asked, or a threshold that is not a positive
+// finite number (from 0 down the kept keys would take in every positive
+// score, as at a session's first refresh, whose thresholds start at 0).
+__device__ __forceinline__ uint32_t spec_floor(const SelectParams& p, int r) {
+  if (p.spec == 0) return 256u;
+  const float t = p.tau[r];
+  return isfinite(t) && t > 0.f ? float_key(t) >> 24 : 256u;
+}
+
 // Float4 loads each thread keeps in flight in the row scans.
 constexpr int kScanUnroll = 4;
 
@@ -1781,6 +1805,7 @@ __global__ void __launch_bounds__(kSelectThreads) atopn_select_kernel(const Sele
     return;
   }
   const float* row = p.scores + (size_t)r * p.ld;
+  const uint32_t fl = spec_floor(p, r);  // read before this CTA writes tau[r]
 
   // given top-digit counts may hold only the bins from some floor up (the
   // score dump counts from just below the stale threshold): they serve when
@@ -1799,16 +1824,30 @@ __global__ void __launch_bounds__(kSelectThreads) atopn_select_kernel(const Sele
     if (hist[i] != 0u) atomicAdd(&counted, hist[i]);
   }
   __syncthreads();
+  bool spec = false;  // uniform: the top-digit pass also kept the keys from bin fl up
   if (p.hist == nullptr || counted < (uint32_t)p.n_top) {  // top digit: a histogram of the whole row
     for (int i = threadIdx.x; i < 256; i += kSelectThreads) hist[i] = 0u;
     __syncthreads();
-    scan_row(row, L, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
+    if (fl < 256u) {
+      spec = true;
+      scan_row(row, L, [&](uint32_t k, bool ok) {
+        hist_add(hist, k >> 24, ok);
+        cand_add(cand, &ncand, k, ok && (k >> 24) >= fl);
+      });
+    } else {
+      scan_row(row, L, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
+    }
     __syncthreads();
   }
   find_bin(hist, (uint32_t)p.n_top, &s_bin, &s_rank, &s_cnt);
   __syncthreads();
   uint32_t prefix = s_bin << 24, mask = 0xFF000000u, rank = s_rank, cnt = s_cnt;
-  bool in_smem = false;
+  // the kept keys hold every key of the N-th largest's bin when that bin is fl
+  // or above and none was dropped; else they are discarded and collected below
+  bool in_smem = spec && s_bin >= fl && ncand <= kSelectCap;
+  __syncthreads();  // every thread has read ncand
+  if (!in_smem && threadIdx.x == 0) ncand = 0;
+  __syncthreads();
   for (int shift = 16; shift >= 0; shift -= 8) {
     if (!in_smem && cnt <= (uint32_t)kSelectCap) {
       scan_row(row, L, [&](uint32_t k, bool ok) {
@@ -1898,8 +1937,10 @@ __device__ __forceinline__ void sel_chunk(int L, int part, int P, int* b, int* e
 // same decision) and finds the digit's bin.  Once the keys matching the
 // prefix fit, each CTA keeps its own in shared memory and the remaining
 // digits are resolved over those.  Given top-digit counts (from the score
-// dump) are used when their bins hold N scores.  Cluster barriers are
-// hardware barriers every CTA reaches on every path.
+// dump) are used when their bins hold N scores.  On refresh steps the
+// top-digit pass also keeps the keys from the stale threshold's bin up, which
+// saves the collection pass when the N-th largest stays in or above that bin.
+// Cluster barriers are hardware barriers every CTA reaches on every path.
 constexpr int kSelCluster = 8;          // CTAs per row
 constexpr int kSelClusterThreads = 512;
 
@@ -1918,6 +1959,8 @@ __global__ void __launch_bounds__(kSelClusterThreads) atopn_cluster_select_kerne
     return;
   }
   const float* row = p.scores + (size_t)r * p.ld;
+  // read before the first cluster barrier, so before CTA 0 can write tau[r]
+  const uint32_t fl = spec_floor(p, r);
   int beg, end;
   sel_chunk(L, c, kSelCluster, &beg, &end);
   // adds the cluster's histograms into tot (every CTA), then finds the bin of `rank`
@@ -1952,10 +1995,19 @@ __global__ void __launch_bounds__(kSelClusterThreads) atopn_cluster_select_kerne
     if (tot[i] != 0u) atomicAdd(&counted, tot[i]);
   }
   __syncthreads();
+  bool spec = false;  // uniform: the top-digit pass also kept this chunk's keys from bin fl up
   if (p.hist == nullptr || counted < (uint32_t)p.n_top) {  // uniform: every CTA read the same counts
     for (int i = threadIdx.x; i < 256; i += kSelClusterThreads) hist[i] = 0u;
     __syncthreads();
-    scan_range(row, beg, end, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
+    if (fl < 256u) {
+      spec = true;
+      scan_range(row, beg, end, [&](uint32_t k, bool ok) {
+        hist_add(hist, k >> 24, ok);
+        cand_add(ccand, &ncand, k, ok && (k >> 24) >= fl);
+      });
+    } else {
+      scan_range(row, beg, end, [&](uint32_t k, bool ok) { hist_add(hist, k >> 24, ok); });
+    }
     cluster_bin((uint32_t)p.n_top);
   } else {
     if (threadIdx.x == 0) {
@@ -1968,7 +2020,13 @@ __global__ void __launch_bounds__(kSelClusterThreads) atopn_cluster_select_kerne
     __syncthreads();
   }
   uint32_t prefix = s_bin << 24, mask = 0xFF000000u, rank = s_rank, cnt = s_cnt;
-  bool in_smem = false;
+  // this CTA's kept keys hold every key of its chunk in the N-th largest's bin
+  // when that bin is fl or above and none was dropped (decided per CTA: the
+  // cluster barriers below do not depend on it)
+  bool in_smem = spec && s_bin >= fl && ncand <= kSelectCap;
+  __syncthreads();  // every thread has read ncand
+  if (!in_smem && threadIdx.x == 0) ncand = 0;
+  __syncthreads();
   for (int shift = 16; shift >= 0; shift -= 8) {
     if (!in_smem && cnt <= (uint32_t)kSelectCap) {  // this CTA's matches are at most the cluster's cnt
       scan_range(row, beg, end, [&](uint32_t k, bool ok) {

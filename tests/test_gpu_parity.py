@@ -210,6 +210,25 @@ def test_refresh_of_long_rows_is_exact(stale, heads):
     assert np.max(np.abs(tau.cpu().numpy() - expect)) <= gpu_harness.BAND
 
 
+def test_refresh_with_overflowing_kept_keys_is_exact():
+    """A stale threshold below every score makes each CTA of the cluster select keep every key of its chunk
+    during the top-digit pass: with 140000 scores a row (17500 a CTA) they overflow the candidate store, and
+    the select collects the N-th largest's bin again; the threshold is the oracle's."""
+    L, N = 140000, 300
+    wl = small("refresh_overflow", h_q=12, h_k=1, h_v=4, d=128, l_kv=L, n_top=N)
+    inp = workload.make_layer(wl, 0, steps=1)
+    shape = saga.SagaShape.of(1, 12, 1, 4, 128, L)
+    kc = inp["K0"].cuda().contiguous()
+    q = inp["q"][0].cuda().contiguous()
+    ws = saga.alloc_workspace(shape)
+    tau = torch.full((1, 12), -1e30, device="cuda")
+    saga.atopn_refresh_threshold(shape, q, kc, L, N, tau, ws)
+    torch.cuda.synchronize()
+    expect = saga_oracle.refresh_threshold(inp["q"][0].float().numpy(), inp["K0"].float().numpy(), L, N)
+    assert np.max(np.abs(tau.cpu().numpy() - expect)) <= gpu_harness.BAND
+    assert saga.saga_get_status(ws) == 0
+
+
 def test_empty_selection_gives_zero():
     """A stale threshold above every score of a later step keeps nothing: output 0, count 0."""
     shape = saga.SagaShape.of(1, 8, 1, 8, 64, 600)
