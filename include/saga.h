@@ -156,7 +156,11 @@ SAGA_API size_t saga_qkv_workspace_bytes(const saga_shape* s, int hidden);
  * tokens"): tau[b, j] = the n_top-th largest of the fp32 scores
  * A[b, j, 0..seq_len) (eq. 2), counted with multiplicity; -inf when
  * n_top >= seq_len.  Exact: radix selection over order-preserving 32-bit
- * images of the scores, no sort.  n_top >= 1. */
+ * images of the scores, no sort.  n_top >= 1.
+ * tau is in/out: its incoming values (the stale thresholds of the last
+ * refresh) only steer the work - the selection keeps the scores from the
+ * stale threshold's top-byte bin up while it counts the top digit - and any
+ * value, NaN and +-inf included, gives the same result bits. */
 SAGA_API int atopn_refresh_threshold(const saga_shape* s, const void* q, const void* k_cache, int seq_len,
                             const int* seq_len_dev, int n_top, float* tau, void* workspace, size_t ws_bytes,
                             void* stream);
