@@ -126,8 +126,10 @@ SAGA_API int saga_kv_append(const saga_shape* s, void* k_cache, void* v_cache, c
  * tensor cores, the hidden dimension split across CTAs and the fp32 partials
  * added in a fixed order, so results are reproducible run to run); each
  * output is rounded once to bf16 (nearest even).  If seq_len_dev is not NULL,
- * pos is read on the device as (*seq_len_dev - 1), clamped into [0, l_cap),
- * and the host pos only needs to be in range.  Requirements: 1 <= batch <=
+ * pos is read on the device as (*seq_len_dev - 1), clamped into [0, l_cap)
+ * (the clamp is not flagged in the status word: the attention call that
+ * reads the same device length flags it), and the host pos only needs to be
+ * in range.  Requirements: 1 <= batch <=
  * 16, hidden a positive multiple of 8, 0 <= pos < l_cap, all tensor pointers
  * device memory 16-byte aligned, q_out and the cache rows not overlapping x
  * or w_qkv.  workspace: device memory of saga_qkv_workspace_bytes(s, hidden)
