@@ -39,7 +39,7 @@ def _worker(rank, world, port, results):
 
 def test_two_ranks_gather_and_combine():
     world = 2
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         results = mgr.dict()
         mp.start_processes(_worker, args=(world, _free_port(), results), nprocs=world, join=True,
                            start_method="spawn")
